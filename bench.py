@@ -1,0 +1,493 @@
+#!/usr/bin/env python
+"""Benchmark of one sparse decode step (top-k token-level sparse attention under GQA, JSSA-style).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload NAME]
+
+A step is the whole hot path for one batch: projection-and-append of the newest key, then the
+decode step (group-mean query, projected score scan with top-k per KV head, gather-free split-K
+attention and combine) through the C ABI.  Inputs are seeded synthetic tensors resident in
+HBM.  Rank 0 prints one JSON line.  Multi-GPU runs (torchrun) are independent replicas of
+the workload on every rank (no data-path collective): weak scaling, time = max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "sparse decode steps/s & achieved HBM GB/s at N=128K, B=1/16; speedup vs dense"
+UNIT = "steps/s"
+DEFAULT_WORKLOAD = "long-128k-b16"
+SECONDARY_WORKLOAD = "long-128k-b1"
+L2_BYTES = 126 * 1024 * 1024
+
+
+# ------------------------------------------------------------------------------ accounting
+def roofline_bytes(B, Hq, Hkv, d, r, seqlens, ks, lam):
+    """Algorithmic HBM bytes of one step, per kernel and in total.
+
+    Per (sequence b, KV head): N_b*r*2 (projected cache scan) + k_b*2*d*2 (selected K and V
+    rows) + G*d*2 (queries) + G*d*4 (fp32 output) [+ N_b*4 gate inputs when lambda != 0].
+    """
+    G = Hq // Hkv
+    kproj = sum(int(n) * r * 2 for n in seqlens) * Hkv
+    kv = sum(min(int(k), int(n)) * 2 * d * 2 for n, k in zip(seqlens, ks)) * Hkv
+    q = B * Hq * d * 2
+    out = B * Hq * d * 4
+    lg = sum(int(n) * 4 for n in seqlens) * Hkv if lam != 0.0 else 0
+    lg_sel = sum(min(int(k), int(n)) * 4 for n, k in zip(seqlens, ks)) * Hkv if lam != 0.0 else 0
+    return {
+        "select": kproj + q + lg,
+        "attend": kv + q + out + lg_sel,
+        "step": kproj + kv + q + out + lg,
+        "kproj": kproj, "kv": kv,
+    }
+
+
+def dense_bytes(B, Hq, Hkv, d, seqlens):
+    return sum(int(n) * 2 * d * 2 for n in seqlens) * Hkv + B * Hq * d * 2 + B * Hq * d * 4
+
+
+def measured_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            j = json.load(f)
+        return float(j["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+def kernel_source_sha(name):
+    path = os.path.join(ROOT, "token_level_sparse_head_b200", "csrc", name)
+    h = hashlib.sha256()
+    for p in (path, os.path.join(ROOT, "token_level_sparse_head_b200", "csrc", "sas_device.cuh")):
+        with open(p, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel_file, workload):
+    """DRAM bytes per launch from the committed ncu summary, if it matches the current source."""
+    try:
+        with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+            t = json.load(f)
+        e = t[kernel_file][workload]
+        if e.get("source_sha") == kernel_source_sha(kernel_file):
+            return float(e["dram_bytes_per_launch"])
+    except Exception:
+        pass
+    return None
+
+
+# ------------------------------------------------------------------------------ clocks
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples while the timed region runs."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_id: str):
+        self.proc = None
+        self.tmp = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", device_id, f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "50"], stdout=self.tmp, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.06)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.tmp.flush()
+        rows = []
+        with open(self.tmp.name) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) >= 8:
+                    rows.append(parts)
+        os.unlink(self.tmp.name)
+        if not rows:
+            return None
+        sm = [float(r[0]) for r in rows if r[0].replace(".", "").isdigit()]
+        mx = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[4 + i].lower().startswith("active")})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+def smi_device_id(torch, dev):
+    try:
+        u = str(torch.cuda.get_device_properties(dev).uuid)
+        return u if u.startswith("GPU-") else "GPU-" + u
+    except Exception:
+        vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
+        return vis.split(",")[dev] if vis else str(dev)
+
+
+# ------------------------------------------------------------------------------ our arm
+class Workload:
+    def __init__(self, name, device, torch):
+        from synth import CONFIGS, make_config
+        from token_level_sparse_head_b200 import DecodeSession, lib, shape_of
+
+        self.name = name
+        self.torch = torch
+        self.lib = lib
+        p = make_config(name, device=device)
+        self.p = p
+        self.shape = shape_of(p)
+        self.sess = DecodeSession(self.shape, p.k_max, device=device)
+        if p.paged:
+            self.kproj = torch.zeros(p.num_pages, p.Hkv, 64, p.r, dtype=torch.bfloat16, device=device)
+        else:
+            self.kproj = torch.zeros(p.B, p.Hkv, p.n_cap, p.r, dtype=torch.bfloat16, device=device)
+        lib.sas_build_proj_cache(self.shape, p.K, p.M, self.kproj, p.page_table, p.seqlens)
+        # the newest key of every sequence (position N_b - 1), for the append of each step
+        sl = p.seqlens.tolist()
+        knew = torch.empty(p.B, p.Hkv, p.d, dtype=torch.bfloat16, device=device)
+        for b, n in enumerate(sl):
+            if p.paged:
+                pg = int(p.page_table[b, (n - 1) // 64])
+                knew[b] = p.K[pg, :, (n - 1) % 64]
+            else:
+                knew[b] = p.K[b, :, n - 1]
+        self.knew = knew
+        self.seqlens_h = sl
+        self.ks_h = p.k.tolist()
+        self.bytes = roofline_bytes(p.B, p.Hq, p.Hkv, p.d, p.r, sl, self.ks_h, p.lam)
+        self.dense_bytes = dense_bytes(p.B, p.Hq, p.Hkv, p.d, sl)
+        self.cfg = dict(CONFIGS[name])
+
+    def step(self):
+        p, L = self.p, self.lib
+        L.sas_append_proj(self.shape, self.knew, p.M, self.kproj, p.page_table, p.seqlens)
+        L.sas_decode_step(self.shape, p.q, p.M, self.kproj, p.K, p.V, p.page_table, p.seqlens, p.k, p.k_max,
+                          p.lam, p.log_g, self.sess.out, self.sess.idx, self.sess.workspace, self.sess.ws_bytes)
+
+    def step_parts(self, ev):
+        """The same step through the component entry points, with events between kernels."""
+        p, L, s = self.p, self.lib, self.sess
+        ev[0].record()
+        L.sas_append_proj(self.shape, self.knew, p.M, self.kproj, p.page_table, p.seqlens)
+        ev[1].record()
+        L.sas_select_topk(self.shape, p.q, p.M, self.kproj, p.page_table, p.seqlens, p.k, p.k_max, p.lam,
+                          p.log_g, s.idx, None, s.workspace, s.ws_bytes)
+        ev[2].record()
+        L.sas_sparse_attention(self.shape, p.q, p.K, p.V, p.page_table, p.seqlens, s.idx, p.k, p.k_max, p.lam,
+                               p.log_g, s.out, s.workspace, s.ws_bytes)
+        ev[3].record()
+
+    def dense(self):
+        p = self.p
+        self.lib.sas_dense_decode(self.shape, p.q, p.K, p.V, p.page_table, p.seqlens, self.sess.out,
+                                  self.sess.workspace, self.sess.ws_bytes)
+
+    def free(self):
+        del self.p, self.kproj, self.sess, self.knew
+        self.torch.cuda.empty_cache()
+
+
+def timed_block(torch, fn, steps, dist=None):
+    """Time `steps` calls of fn as one block: barrier + sync on both sides, CUDA events on the
+    current stream; returns the max over ranks of the elapsed seconds."""
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        fn()
+    e1.record()
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    t = e0.elapsed_time(e1) / 1e3
+    if dist is not None:
+        tt = torch.tensor([t], dtype=torch.float64, device="cuda")
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        t = float(tt.item())
+    return t
+
+
+def flushed_steps(torch, fn, steps, flush_buf):
+    """Per-step event timing with an L2 flush (a write larger than L2) between steps."""
+    ts = []
+    for _ in range(steps):
+        flush_buf.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        fn()
+        e1.record()
+        torch.cuda.synchronize()
+        ts.append(e0.elapsed_time(e1) / 1e3)
+    return statistics.median(ts)
+
+
+def run_ours(args):
+    import torch
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as tdist
+
+        tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                 device_id=torch.device("cuda", local))
+        dist = tdist
+    dev = f"cuda:{local}"
+    peak, peak_kind = measured_peaks()
+
+    wl = Workload(args.workload, dev, torch)
+    p = wl.p
+    for _ in range(args.warmup):
+        wl.step()
+    torch.cuda.synchronize()
+
+    # --- headline: K steps through sas_append_proj + sas_decode_step, inputs resident in HBM
+    sampler = ClockSampler(smi_device_id(torch, local))
+    t = timed_block(torch, wl.step, args.steps, dist)
+    clocks = sampler.stop()
+    ms = t / args.steps * 1e3
+    value = args.steps * world / t
+
+    # --- per-kernel durations (component entry points, events between the kernels)
+    nk = max(3, min(args.steps, 200))
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(nk)]
+    torch.cuda.synchronize()
+    for i in range(nk):
+        wl.step_parts(evs[i])
+    torch.cuda.synchronize()
+    k_ms = {
+        "append": statistics.mean(e[0].elapsed_time(e[1]) for e in evs),
+        "select": statistics.mean(e[1].elapsed_time(e[2]) for e in evs),
+        "attend": statistics.mean(e[2].elapsed_time(e[3]) for e in evs),
+    }
+    dom = "select" if k_ms["select"] >= k_ms["attend"] else "attend"
+    dom_bytes = wl.bytes[dom]
+    head_bytes = dict(wl.bytes)
+    head_dense_bytes = wl.dense_bytes
+    achieved = dom_bytes / (k_ms[dom] * 1e-3) / 1e9
+    traffic = recorded_traffic("select.cu" if dom == "select" else "attend.cu", args.workload)
+
+    # --- dense full-KV baseline on the same workload
+    for _ in range(2):
+        wl.dense()
+    nd = max(3, min(args.steps // 10, 50))
+    td = timed_block(torch, wl.dense, nd, dist)
+    dense_ms = td / nd * 1e3
+
+    # --- end to end through the C ABI with host buffers (pinned), copies inside the timed region
+    q_host = torch.empty_like(p.q, device="cpu").pin_memory()
+    q_host.copy_(p.q)
+    knew_host = torch.empty_like(wl.knew, device="cpu").pin_memory()
+    knew_host.copy_(wl.knew)
+    out_host = torch.empty_like(wl.sess.out, device="cpu").pin_memory()
+
+    def e2e_step():
+        p.q.copy_(q_host, non_blocking=True)
+        wl.knew.copy_(knew_host, non_blocking=True)
+        wl.step()
+        out_host.copy_(wl.sess.out, non_blocking=True)
+        torch.cuda.current_stream().synchronize()
+
+    for _ in range(3):
+        e2e_step()
+    ne = max(3, min(args.steps, 200))
+    te = timed_block(torch, e2e_step, ne, dist)
+    e2e = {"value": ne * world / te, "unit": UNIT,
+           "h2d_bytes_per_step": q_host.numel() * 2 + knew_host.numel() * 2,
+           "d2h_bytes_per_step": out_host.numel() * 4}
+
+    # --- secondary workload: B = 1 at 128K (L2 flushed between steps; its 84 MB fit in L2)
+    secondary = None
+    if not args.no_secondary and args.workload == DEFAULT_WORKLOAD:
+        wl.free()
+        del wl
+        w1 = Workload(SECONDARY_WORKLOAD, dev, torch)
+        flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
+        for _ in range(3):
+            w1.step()
+        t1 = flushed_steps(torch, w1.step, max(10, min(args.steps, 100)), flush)
+        td1 = flushed_steps(torch, w1.dense, 10, flush)
+        secondary = {"workload": SECONDARY_WORKLOAD, "ms_per_step": t1 * 1e3, "steps_per_s": 1.0 / t1,
+                     "hbm_gbs": w1.bytes["step"] / t1 / 1e9, "dense_ms_per_step": td1 * 1e3,
+                     "speedup_vs_dense": td1 / t1, "l2": "flushed between steps (2x L2 write)"}
+        wl = w1
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(args.workload, budget_s=args.cpu_seconds)
+
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    c = CONFIGS_VIEW(args.workload)
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32", "storage_dtype": "bf16", "data": "synthetic",
+        "config": dict(workload=args.workload, **c, l2="inputs larger than L2: each step reads "
+                       f"{head_bytes['step'] / 1e9:.2f} GB, L2 is 0.13 GB", parallelism=f"replicas x{world}"),
+        "hbm_gbs": None, "speedup_vs_dense": dense_ms / ms,
+        "dense": {"ms_per_step": dense_ms, "steps_per_s": 1e3 / dense_ms},
+        "kernels_ms": k_ms,
+        "roofline": {"kernel": dom, "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "peak_kind": peak_kind,
+                     "algorithmic_bytes_per_launch": dom_bytes, "traffic": traffic},
+        "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": 3 * args.steps, "clocks": clocks,
+    }
+    line["hbm_gbs"] = head_bytes["step"] / (ms * 1e-3) / 1e9
+    line["step_roofline_frac"] = line["hbm_gbs"] / peak
+    line["dense"]["hbm_gbs"] = head_dense_bytes / (dense_ms * 1e-3) / 1e9
+    if secondary:
+        line["b1"] = secondary
+    print(json.dumps(line), flush=True)
+
+
+def CONFIGS_VIEW(name):
+    from synth import CONFIGS
+
+    c = dict(CONFIGS[name])
+    return {k: c[k] for k in ("B", "Hq", "Hkv", "d", "r", "N", "k") if k in c} | (
+        {"lam": c["lam"]} if "lam" in c else {})
+
+
+# ------------------------------------------------------------------------------ oracle arm
+def _threads_used():
+    try:
+        from threadpoolctl import threadpool_info
+
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return 1
+
+
+def oracle_head_problem(name, seed):
+    """One (sequence, KV head) of the named workload, drawn on the CPU (heads are independent
+    and identically distributed), with its projected cache built by the oracle."""
+    from oracle import sas_oracle as O
+    from synth import CONFIGS, make_problem
+
+    c = CONFIGS[name]
+    G = c["Hq"] // c["Hkv"]
+    n = c["N"] if c["N"] else (c["n_lo"] + c["n_hi"]) // 2
+    k = c["k"] if c["k"] else n // c["k_div"]
+    p = make_problem(B=1, Hq=G, Hkv=1, d=c["d"], r=c["r"], seqlens=[n], k=[k], lam=c.get("lam", 0.0),
+                     basis=c["basis"], aniso=c["aniso"], seed=seed)
+    f = lambda t: None if t is None else t.to(__import__("torch").float64).numpy()
+    q, K, V, M = f(p.q)[0], f(p.K)[0, 0, :n], f(p.V)[0, 0, :n], f(p.M)[0]
+    lg = None if p.log_g is None else f(p.log_g)[0, 0, :n]
+    kp = O.project_keys(K, M)
+    return dict(q=q, K=K, V=V, M=M, kp=kp, lg=lg, k=k, lam=c.get("lam", 0.0))
+
+
+def oracle_head_seconds(h):
+    from oracle import sas_oracle as O
+
+    t0 = time.perf_counter()
+    O.decode_head(h["q"], h["M"], h["kp"], h["K"], h["V"], h["k"], h["lam"], h["lg"])
+    return time.perf_counter() - t0
+
+
+def cpu_baseline(name, budget_s=15.0):
+    """The oracle, as it stands, on a bounded sample of the workload: whole heads (one sequence x
+    one KV head each) until about budget_s seconds of oracle time; steps/s extrapolates to all
+    B*Hkv heads of a step."""
+    from synth import CONFIGS
+
+    c = CONFIGS[name]
+    heads_per_step = c["B"] * c["Hkv"]
+    ts = []
+    i = 0
+    while sum(ts) < budget_s and i < 64:
+        h = oracle_head_problem(name, seed=1000 + i)
+        ts.append(oracle_head_seconds(h))
+        i += 1
+    per_head = statistics.mean(ts)
+    return {"value": 1.0 / (per_head * heads_per_step), "unit": UNIT, "cores": _threads_used(),
+            "kind": "oracle", "sample": f"{len(ts)} of {heads_per_step} (sequence, KV head) pairs of one "
+            f"step ({sum(ts):.1f} s of oracle time), extrapolated to the whole step"}
+
+
+def run_reference(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    from synth import CONFIGS
+
+    c = CONFIGS[args.workload]
+    heads_per_step = c["B"] * c["Hkv"]
+    h = oracle_head_problem(args.workload, seed=2000)
+    for _ in range(max(0, min(args.warmup, 3))):
+        oracle_head_seconds(h)
+    ts = []
+    t_start = time.perf_counter()
+    for i in range(args.steps):
+        ts.append(oracle_head_seconds(h))
+        if time.perf_counter() - t_start > args.cpu_seconds * 4:
+            break
+    per_head = statistics.mean(ts)
+    value = 1.0 / (per_head * heads_per_step)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": per_head * heads_per_step * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": dict(workload=args.workload, **CONFIGS_VIEW(args.workload)),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": _threads_used(), "kind": "oracle",
+                         "sample": f"{len(ts)} timed oracle runs of one (sequence, KV head) pair of "
+                                   f"the workload; each step = {heads_per_step} such pairs"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--no-secondary", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

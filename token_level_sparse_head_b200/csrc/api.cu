@@ -1,0 +1,325 @@
+// C ABI of libsas (declared in include/sas.h): host-side validation, workspace layout and
+// kernel launches.  Nothing here allocates device memory or synchronises, except the
+// debugging call sas_check_workspace.
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+
+#include "sas.h"
+#include "sas_kernels.h"
+
+namespace {
+
+thread_local char g_detail[512] = {0};
+
+sas_status fail(sas_status s, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_detail, sizeof(g_detail), fmt, ap);
+  va_end(ap);
+  return s;
+}
+
+sas_status cuda_fail(cudaError_t e, const char* where) {
+  return fail(SAS_ERR_CUDA, "%s: %s", where, cudaGetErrorString(e));
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int cap_of(const sas_shape* s) { return s->page_size ? s->max_pages * s->page_size : s->n_cap; }
+
+sas_status check_shape(const sas_shape* s) {
+  if (s == nullptr) return fail(SAS_ERR_INVALID_ARG, "shape is NULL");
+  if (s->B < 1 || s->Hq < 1 || s->Hkv < 1) return fail(SAS_ERR_INVALID_ARG, "B, Hq, Hkv must be >= 1");
+  if (s->Hq % s->Hkv) return fail(SAS_ERR_INVALID_ARG, "Hq (%d) is not a multiple of Hkv (%d)", s->Hq, s->Hkv);
+  if (s->d != 64 && s->d != 128) return fail(SAS_ERR_UNSUPPORTED, "head dim d=%d (supported: 64, 128)", s->d);
+  if (s->r != 16 && s->r != 32 && s->r != 64) return fail(SAS_ERR_UNSUPPORTED, "rank r=%d (supported: 16, 32, 64)", s->r);
+  if (s->r > s->d) return fail(SAS_ERR_INVALID_ARG, "rank r=%d exceeds d=%d", s->r, s->d);
+  if (s->kproj_dtype != SAS_KPROJ_BF16) return fail(SAS_ERR_UNSUPPORTED, "kproj_dtype %d", s->kproj_dtype);
+  if (s->page_size == 0) {
+    if (s->n_cap < 4 || (s->n_cap % 4)) return fail(SAS_ERR_INVALID_ARG, "n_cap=%d must be a positive multiple of 4", s->n_cap);
+    if ((long long)s->B * s->Hkv * s->n_cap >= (1LL << 32)) return fail(SAS_ERR_UNSUPPORTED, "cache rows exceed 2^32");
+  } else if (s->page_size == 64) {
+    if (s->max_pages < 1 || s->num_pages < 1) return fail(SAS_ERR_INVALID_ARG, "paged layout needs max_pages, num_pages >= 1");
+    if ((long long)s->num_pages * s->Hkv * 64 >= (1LL << 32)) return fail(SAS_ERR_UNSUPPORTED, "cache rows exceed 2^32");
+  } else {
+    return fail(SAS_ERR_UNSUPPORTED, "page_size=%d (supported: 0 contiguous, 64 paged)", s->page_size);
+  }
+  if (cap_of(s) > SAS_MAX_CAPACITY) return fail(SAS_ERR_UNSUPPORTED, "capacity %d exceeds %d", cap_of(s), SAS_MAX_CAPACITY);
+  if ((long long)s->B * s->Hkv > 65535) return fail(SAS_ERR_UNSUPPORTED, "B*Hkv exceeds 65535");
+  return SAS_OK;
+}
+
+sas_status check_ptr(const void* p, const char* name, bool required = true) {
+  if (p == nullptr) return required ? fail(SAS_ERR_INVALID_ARG, "%s is NULL", name) : SAS_OK;
+  if (!aligned16(p)) return fail(SAS_ERR_INVALID_ARG, "%s is not 16-byte aligned", name);
+  return SAS_OK;
+}
+
+#define SAS_TRY(expr)                 \
+  do {                                \
+    const sas_status _s = (expr);     \
+    if (_s != SAS_OK) return _s;      \
+  } while (0)
+
+int num_sms() {
+  int dev = 0, n = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n;
+}
+
+// Workspace: [0,256) error word | counters (uint32, 256-aligned) | partials (fp32)
+constexpr size_t kErrBytes = 256;
+
+sas::AttendParams attend_plan(const sas_shape* s, int count_max) {
+  sas::AttendParams a = {};
+  a.B = s->B; a.Hq = s->Hq; a.Hkv = s->Hkv; a.G = s->Hq / s->Hkv; a.d = s->d;
+  a.cap = cap_of(s);
+  sas::plan_attend(a, count_max);
+  return a;
+}
+
+size_t ws_bytes_for(const sas::AttendParams& a) {
+  size_t cnt = (size_t)a.B * a.Hkv * a.ngz * 4;
+  cnt = (cnt + 255) & ~(size_t)255;
+  return kErrBytes + cnt + sas::attend_workspace_floats(a) * 4;
+}
+
+void bind_workspace(sas::AttendParams& a, void* ws) {
+  unsigned char* w = static_cast<unsigned char*>(ws);
+  size_t cnt = (size_t)a.B * a.Hkv * a.ngz * 4;
+  cnt = (cnt + 255) & ~(size_t)255;
+  a.err = reinterpret_cast<uint32_t*>(w);
+  a.counters = reinterpret_cast<uint32_t*>(w + kErrBytes);
+  a.partials = reinterpret_cast<float*>(w + kErrBytes + cnt);
+}
+
+sas_status check_cache_ptrs(const sas_shape* s, const int32_t* page_table, const int32_t* seqlens) {
+  SAS_TRY(check_ptr(seqlens, "seqlens"));
+  if (s->page_size) SAS_TRY(check_ptr(page_table, "page_table"));
+  return SAS_OK;
+}
+
+sas_status do_select(const sas_shape* s, const void* q, const float* M, const void* Kproj,
+                     const int32_t* page_table, const int32_t* seqlens, const int32_t* k, int32_t k_max,
+                     float lambda, const float* log_g, int32_t* idx_out, float* scores_out, uint32_t* err,
+                     cudaStream_t st) {
+  sas::SelectParams sp = {};
+  sp.q = static_cast<const __nv_bfloat16*>(q);
+  sp.M = M;
+  sp.kproj = static_cast<const __nv_bfloat16*>(Kproj);
+  sp.page_table = s->page_size ? page_table : nullptr;
+  sp.seqlens = seqlens;
+  sp.kvec = k;
+  sp.log_g = (lambda != 0.0f) ? log_g : nullptr;
+  sp.idx_out = idx_out;
+  sp.scores_out = scores_out;
+  sp.err = err;
+  sp.B = s->B; sp.Hq = s->Hq; sp.Hkv = s->Hkv; sp.G = s->Hq / s->Hkv; sp.d = s->d; sp.r = s->r;
+  sp.cap = cap_of(s);
+  sp.max_pages = s->max_pages; sp.num_pages = s->num_pages; sp.paged = s->page_size ? 1 : 0;
+  sp.k_max = k_max;
+  sp.sigma = 1.0f / sqrtf((float)s->d);
+  sp.lam = lambda;
+  if (!sas::plan_select(sp, num_sms())) return fail(SAS_ERR_UNSUPPORTED, "no selection plan for this shape");
+  const cudaError_t e = sas::launch_select(sp, st);
+  if (e != cudaSuccess) return cuda_fail(e, "select kernel launch");
+  return SAS_OK;
+}
+
+sas_status do_attend(const sas_shape* s, const void* q, const void* K, const void* V, const int32_t* page_table,
+                     const int32_t* seqlens, const int32_t* idx, const int32_t* k, int32_t count_max,
+                     float lambda, const float* log_g, float* out, void* ws, cudaStream_t st) {
+  sas::AttendParams a = attend_plan(s, count_max);
+  bind_workspace(a, ws);
+  a.q = static_cast<const __nv_bfloat16*>(q);
+  a.K = static_cast<const __nv_bfloat16*>(K);
+  a.V = static_cast<const __nv_bfloat16*>(V);
+  a.page_table = s->page_size ? page_table : nullptr;
+  a.seqlens = seqlens;
+  a.idx = idx;
+  a.kvec = k;
+  a.log_g = (idx != nullptr && lambda != 0.0f) ? log_g : nullptr;
+  a.out = out;
+  a.max_pages = s->max_pages; a.num_pages = s->num_pages; a.paged = s->page_size ? 1 : 0;
+  a.k_max = count_max;
+  a.sigma = 1.0f / sqrtf((float)s->d);
+  a.lam = lambda;
+  const cudaError_t e = sas::launch_attend(a, st);
+  if (e != cudaSuccess) return cuda_fail(e, "attention kernel launch");
+  return SAS_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int sas_abi_version(void) { return SAS_ABI_VERSION; }
+
+const char* sas_status_string(sas_status s) {
+  switch (s) {
+    case SAS_OK: return "SAS_OK";
+    case SAS_ERR_INVALID_ARG: return "SAS_ERR_INVALID_ARG";
+    case SAS_ERR_UNSUPPORTED: return "SAS_ERR_UNSUPPORTED";
+    case SAS_ERR_CUDA: return "SAS_ERR_CUDA";
+    case SAS_ERR_DEVICE_CHECK: return "SAS_ERR_DEVICE_CHECK";
+  }
+  return "SAS_UNKNOWN_STATUS";
+}
+
+const char* sas_last_error_detail(void) { return g_detail; }
+
+size_t sas_decode_workspace_bytes(const sas_shape* shape, int32_t k_max) {
+  if (check_shape(shape) != SAS_OK || k_max < 1) return 0;
+  return ws_bytes_for(attend_plan(shape, k_max));
+}
+
+size_t sas_dense_workspace_bytes(const sas_shape* shape) {
+  if (check_shape(shape) != SAS_OK) return 0;
+  return ws_bytes_for(attend_plan(shape, cap_of(shape)));
+}
+
+sas_status sas_workspace_init(void* workspace, size_t ws_bytes, void* stream) {
+  SAS_TRY(check_ptr(workspace, "workspace"));
+  if (ws_bytes < kErrBytes) return fail(SAS_ERR_INVALID_ARG, "workspace smaller than %zu bytes", kErrBytes);
+  const cudaError_t e = cudaMemsetAsync(workspace, 0, ws_bytes, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? SAS_OK : cuda_fail(e, "workspace memset");
+}
+
+sas_status sas_check_workspace(void* workspace, size_t ws_bytes, void* stream, uint32_t* code_out,
+                               uint32_t* where_out) {
+  SAS_TRY(check_ptr(workspace, "workspace"));
+  if (ws_bytes < kErrBytes) return fail(SAS_ERR_INVALID_ARG, "workspace smaller than %zu bytes", kErrBytes);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint32_t w[2] = {0, 0};
+  cudaError_t e = cudaMemcpyAsync(w, workspace, sizeof(w), cudaMemcpyDeviceToHost, st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  if (e == cudaSuccess) e = cudaMemsetAsync(workspace, 0, sizeof(w), st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return cuda_fail(e, "reading the workspace error word");
+  if (code_out) *code_out = w[0];
+  if (where_out) *where_out = w[1];
+  return w[0] ? SAS_ERR_DEVICE_CHECK : SAS_OK;
+}
+
+sas_status sas_build_proj_cache(const sas_shape* shape, const void* K, const float* M, void* Kproj,
+                                const int32_t* page_table, const int32_t* seqlens, void* stream) {
+  SAS_TRY(check_shape(shape));
+  SAS_TRY(check_ptr(K, "K"));
+  SAS_TRY(check_ptr(M, "M"));
+  SAS_TRY(check_ptr(Kproj, "Kproj"));
+  SAS_TRY(check_cache_ptrs(shape, page_table, seqlens));
+  sas::ProjParams p = {};
+  p.K = static_cast<const __nv_bfloat16*>(K);
+  p.M = M;
+  p.Kproj = static_cast<__nv_bfloat16*>(Kproj);
+  p.page_table = shape->page_size ? page_table : nullptr;
+  p.seqlens = seqlens;
+  p.err = nullptr;
+  p.B = shape->B; p.Hkv = shape->Hkv; p.d = shape->d; p.r = shape->r; p.cap = cap_of(shape);
+  p.max_pages = shape->max_pages; p.num_pages = shape->num_pages; p.paged = shape->page_size ? 1 : 0;
+  p.append = 0;
+  const cudaError_t e = sas::launch_proj(p, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? SAS_OK : cuda_fail(e, "projection build launch");
+}
+
+sas_status sas_append_proj(const sas_shape* shape, const void* K_new, const float* M, void* Kproj,
+                           const int32_t* page_table, const int32_t* seqlens, void* stream) {
+  SAS_TRY(check_shape(shape));
+  SAS_TRY(check_ptr(K_new, "K_new"));
+  SAS_TRY(check_ptr(M, "M"));
+  SAS_TRY(check_ptr(Kproj, "Kproj"));
+  SAS_TRY(check_cache_ptrs(shape, page_table, seqlens));
+  sas::ProjParams p = {};
+  p.K = static_cast<const __nv_bfloat16*>(K_new);
+  p.M = M;
+  p.Kproj = static_cast<__nv_bfloat16*>(Kproj);
+  p.page_table = shape->page_size ? page_table : nullptr;
+  p.seqlens = seqlens;
+  p.B = shape->B; p.Hkv = shape->Hkv; p.d = shape->d; p.r = shape->r; p.cap = cap_of(shape);
+  p.max_pages = shape->max_pages; p.num_pages = shape->num_pages; p.paged = shape->page_size ? 1 : 0;
+  p.append = 1;
+  const cudaError_t e = sas::launch_proj(p, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? SAS_OK : cuda_fail(e, "projection append launch");
+}
+
+sas_status sas_select_topk(const sas_shape* shape, const void* q, const float* M, const void* Kproj,
+                           const int32_t* page_table, const int32_t* seqlens, const int32_t* k, int32_t k_max,
+                           float lambda, const float* log_g, int32_t* idx_out, float* scores_out, void* workspace,
+                           size_t ws_bytes, void* stream) {
+  SAS_TRY(check_shape(shape));
+  if (k_max < 1) return fail(SAS_ERR_INVALID_ARG, "k_max must be >= 1");
+  SAS_TRY(check_ptr(q, "q"));
+  SAS_TRY(check_ptr(M, "M"));
+  SAS_TRY(check_ptr(Kproj, "Kproj"));
+  SAS_TRY(check_ptr(k, "k"));
+  SAS_TRY(check_ptr(idx_out, "idx_out"));
+  SAS_TRY(check_ptr(scores_out, "scores_out", false));
+  SAS_TRY(check_cache_ptrs(shape, page_table, seqlens));
+  if (lambda != 0.0f) SAS_TRY(check_ptr(log_g, "log_g"));
+  SAS_TRY(check_ptr(workspace, "workspace"));
+  if (ws_bytes < sas_decode_workspace_bytes(shape, k_max)) return fail(SAS_ERR_INVALID_ARG, "workspace too small");
+  return do_select(shape, q, M, Kproj, page_table, seqlens, k, k_max, lambda, log_g, idx_out, scores_out,
+                   static_cast<uint32_t*>(workspace), static_cast<cudaStream_t>(stream));
+}
+
+sas_status sas_sparse_attention(const sas_shape* shape, const void* q, const void* K, const void* V,
+                                const int32_t* page_table, const int32_t* seqlens, const int32_t* idx,
+                                const int32_t* k, int32_t k_max, float lambda, const float* log_g, float* out,
+                                void* workspace, size_t ws_bytes, void* stream) {
+  SAS_TRY(check_shape(shape));
+  if (k_max < 1) return fail(SAS_ERR_INVALID_ARG, "k_max must be >= 1");
+  SAS_TRY(check_ptr(q, "q"));
+  SAS_TRY(check_ptr(K, "K"));
+  SAS_TRY(check_ptr(V, "V"));
+  SAS_TRY(check_ptr(idx, "idx"));
+  SAS_TRY(check_ptr(k, "k"));
+  SAS_TRY(check_ptr(out, "out"));
+  SAS_TRY(check_cache_ptrs(shape, page_table, seqlens));
+  if (lambda != 0.0f) SAS_TRY(check_ptr(log_g, "log_g"));
+  SAS_TRY(check_ptr(workspace, "workspace"));
+  if (ws_bytes < sas_decode_workspace_bytes(shape, k_max)) return fail(SAS_ERR_INVALID_ARG, "workspace too small");
+  return do_attend(shape, q, K, V, page_table, seqlens, idx, k, k_max, lambda, log_g, out, workspace,
+                   static_cast<cudaStream_t>(stream));
+}
+
+sas_status sas_decode_step(const sas_shape* shape, const void* q, const float* M, const void* Kproj, const void* K,
+                           const void* V, const int32_t* page_table, const int32_t* seqlens, const int32_t* k,
+                           int32_t k_max, float lambda, const float* log_g, float* out, int32_t* idx_out,
+                           void* workspace, size_t ws_bytes, void* stream) {
+  SAS_TRY(check_shape(shape));
+  if (k_max < 1) return fail(SAS_ERR_INVALID_ARG, "k_max must be >= 1");
+  SAS_TRY(check_ptr(q, "q"));
+  SAS_TRY(check_ptr(M, "M"));
+  SAS_TRY(check_ptr(Kproj, "Kproj"));
+  SAS_TRY(check_ptr(K, "K"));
+  SAS_TRY(check_ptr(V, "V"));
+  SAS_TRY(check_ptr(k, "k"));
+  SAS_TRY(check_ptr(out, "out"));
+  SAS_TRY(check_ptr(idx_out, "idx_out"));
+  SAS_TRY(check_cache_ptrs(shape, page_table, seqlens));
+  if (lambda != 0.0f) SAS_TRY(check_ptr(log_g, "log_g"));
+  SAS_TRY(check_ptr(workspace, "workspace"));
+  if (ws_bytes < sas_decode_workspace_bytes(shape, k_max)) return fail(SAS_ERR_INVALID_ARG, "workspace too small");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  SAS_TRY(do_select(shape, q, M, Kproj, page_table, seqlens, k, k_max, lambda, log_g, idx_out, nullptr,
+                    static_cast<uint32_t*>(workspace), st));
+  return do_attend(shape, q, K, V, page_table, seqlens, idx_out, k, k_max, lambda, log_g, out, workspace, st);
+}
+
+sas_status sas_dense_decode(const sas_shape* shape, const void* q, const void* K, const void* V,
+                            const int32_t* page_table, const int32_t* seqlens, float* out, void* workspace,
+                            size_t ws_bytes, void* stream) {
+  SAS_TRY(check_shape(shape));
+  SAS_TRY(check_ptr(q, "q"));
+  SAS_TRY(check_ptr(K, "K"));
+  SAS_TRY(check_ptr(V, "V"));
+  SAS_TRY(check_ptr(out, "out"));
+  SAS_TRY(check_cache_ptrs(shape, page_table, seqlens));
+  SAS_TRY(check_ptr(workspace, "workspace"));
+  if (ws_bytes < sas_dense_workspace_bytes(shape)) return fail(SAS_ERR_INVALID_ARG, "workspace too small");
+  return do_attend(shape, q, K, V, page_table, seqlens, nullptr, nullptr, cap_of(shape), 0.0f, nullptr, out,
+                   workspace, static_cast<cudaStream_t>(stream));
+}
+
+}  // extern "C"

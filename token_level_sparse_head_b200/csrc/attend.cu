@@ -1,0 +1,446 @@
+// Gather-free split-K decode attention over per-KV-head index sets (sm_100a).
+//
+// JSSA page, section 原理详解(二) / Triton 内核的三个设计点: one launch per layer serves
+// every KV head, each query head is mapped to the index set its KV head selected, and the K/V
+// rows are read where they live, with no staging copy of the selected cache.  One token's K
+// (or V) head slice is contiguous (section 不规则索引本身不是障碍), so each selected row is
+// fetched as one bulk copy of d*2 bytes on the TMA engine straight into this warp's shared
+// memory ring; the page holding it is resolved per index for the paged layout.
+//
+// Grid: (splits, B*Hkv, G/gt).  A CTA takes a contiguous slice of one (b, h) index list and
+// gt query heads of h; its 4 warps take 8-token tiles of the slice in turn, each warp with its
+// own ring of stages and its own online-softmax state (running max m, sum l, accumulator), in
+// fp32.  Logits z = sigma q.K_i (+ lambda log g_i, SAS page section 2.1).  The warps merge in
+// shared memory, the CTA writes one partial (m, l, acc) per query head to the workspace, and
+// the last CTA of each (b, h, head group) to finish merges all splits in split order
+// (deterministic) and writes the output.  The dense variant (idx = 0..N_b-1) is the full-KV
+// baseline.
+#include "sas_device.cuh"
+#include "sas_kernels.h"
+
+namespace sas {
+namespace {
+
+constexpr int kWarps = 4;
+constexpr int kThreads = kWarps * 32;
+constexpr int kTile = 8;     // tokens per warp tile
+constexpr int kStages = 4;   // ring depth per warp
+
+template <int D, int GT>
+struct Geo {
+  static constexpr int LPR = D / 8;            // lanes per K row (16 bytes each)
+  static constexpr int RPI = 32 / LPR;         // rows per warp instruction
+  static constexpr int NP = kTile / RPI;       // row groups per lane per tile
+  static constexpr int NV = NP * GT;           // partial dot products per lane per tile
+  static constexpr int CPL = D / 32;           // output channels per lane (PV)
+  static constexpr int ROW_BYTES = D * 2;
+  static constexpr int STAGE_BYTES = 2 * kTile * ROW_BYTES;
+  static constexpr int LOG_LPR = (LPR == 16) ? 4 : 3;
+  static constexpr int LOG_NV = (NV >= 16) ? 4 : (NV == 8 ? 3 : (NV == 4 ? 2 : (NV == 2 ? 1 : 0)));
+  // After the reduction a lane's value index is (lane % LPR) >> SHIFT (SHIFT > 0 when NV < LPR).
+  static constexpr int SHIFT = LOG_LPR > LOG_NV ? LOG_LPR - LOG_NV : 0;
+  static constexpr int LOG_GT = GT == 4 ? 2 : (GT == 2 ? 1 : 0);
+};
+
+struct Smem {
+  int off_rows, off_lg, off_ring, off_pbuf, off_sbuf, off_merge, off_bars, off_w, off_flag, total;
+};
+
+template <int D, int GT>
+__host__ __device__ inline Smem smem_layout(int split_len, int splits) {
+  using Gm = Geo<D, GT>;
+  Smem s;
+  int o = 0;
+  s.off_rows = o;  o += split_len * 4;
+  s.off_lg = o;    o += split_len * 4;
+  o = (o + 127) & ~127;
+  s.off_ring = o;  o += kWarps * kStages * Gm::STAGE_BYTES;
+  s.off_pbuf = o;  o += kWarps * kTile * GT * 4;
+  s.off_sbuf = o;  o += kWarps * GT * 4;
+  s.off_merge = o; o += kWarps * GT * (D + 2) * 4;
+  o = (o + 7) & ~7;
+  s.off_bars = o;  o += kWarps * kStages * 8;
+  s.off_w = o;     o += splits * GT * 4 + GT * 8;
+  s.off_flag = o;  o += 16;
+  s.total = o;
+  return s;
+}
+
+template <int D, int GT, bool GATED, bool PAGED, bool DENSE>
+__global__ void __launch_bounds__(kThreads) attend_kernel(const AttendParams p) {
+  using Gm = Geo<D, GT>;
+  extern __shared__ __align__(128) unsigned char smem[];
+  const Smem L = smem_layout<D, GT>(p.split_len, p.splits);
+  uint32_t* rows_s = reinterpret_cast<uint32_t*>(smem + L.off_rows);
+  float* lg_s = reinterpret_cast<float*>(smem + L.off_lg);
+  unsigned char* ring = smem + L.off_ring;
+  float* pbuf_all = reinterpret_cast<float*>(smem + L.off_pbuf);
+  float* sbuf_all = reinterpret_cast<float*>(smem + L.off_sbuf);
+  float* merge = reinterpret_cast<float*>(smem + L.off_merge);
+  uint64_t* bars_all = reinterpret_cast<uint64_t*>(smem + L.off_bars);
+  float* wts = reinterpret_cast<float*>(smem + L.off_w);
+  int* flag = reinterpret_cast<int*>(smem + L.off_flag);
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int split = blockIdx.x;
+  const int bh = blockIdx.y;
+  const int gz = blockIdx.z;
+  const int b = bh / p.Hkv, h = bh % p.Hkv;
+  const int bhz = bh * p.ngz + gz;
+
+  int n = p.seqlens[b];
+  if (n < 0 || n > p.cap) {
+    if (split == 0 && tid == 0 && h == 0 && gz == 0) record_error(p.err, kDevBadSeqlen, (uint32_t)b);
+    n = 0;
+  }
+  int count = n;
+  if (!DENSE) {
+    int kb = p.kvec[b];
+    kb = min(kb, p.k_max);
+    count = max(0, min(kb, n));
+  }
+  const int j0 = split * p.split_len;
+  const int j1 = min(j0 + p.split_len, count);
+  const int cnt = max(0, j1 - j0);
+
+  // ---- resolve the slice's rows (and gate terms) once ----
+  for (int j = tid; j < cnt; j += kThreads) {
+    int i = DENSE ? (j0 + j) : p.idx[(size_t)bh * p.k_max + j0 + j];
+    if (!DENSE && (i < 0 || i >= n)) {
+      record_error(p.err, kDevBadIndex, (uint32_t)bh);
+      i = 0;
+    }
+    uint32_t row;
+    if (PAGED) {
+      int pg = p.page_table[(size_t)b * p.max_pages + (i >> 6)];
+      if (pg < 0 || pg >= p.num_pages) {
+        record_error(p.err, kDevBadPage, (uint32_t)b);
+        pg = 0;
+      }
+      row = ((uint32_t)pg * (uint32_t)p.Hkv + (uint32_t)h) * 64u + (uint32_t)(i & 63);
+    } else {
+      row = (uint32_t)bh * (uint32_t)p.cap + (uint32_t)i;
+    }
+    rows_s[j] = row;
+    if (GATED) lg_s[j] = p.lam * p.log_g[(size_t)bh * p.cap + i];
+  }
+  if (lane == 0) {
+    for (int s = 0; s < kStages; ++s) mbar_init(&bars_all[warp * kStages + s], 1);
+    fence_barrier_init();
+  }
+
+  // ---- query slice in registers: lane holds channels c0..c0+7 of each of its gt heads ----
+  const int rl = lane % Gm::LPR;   // lane within its row
+  const int rs = lane / Gm::LPR;   // row slot within a warp instruction
+  const int c0 = rl * 8;
+  float2 qv[GT][4];
+#pragma unroll
+  for (int g = 0; g < GT; ++g) {
+    const int hq = h * p.G + gz * GT + g;
+    const uint4 w = *reinterpret_cast<const uint4*>(p.q + ((size_t)b * p.Hq + hq) * D + c0);
+    qv[g][0] = make_float2(bf16lo(w.x) * p.sigma, bf16hi(w.x) * p.sigma);
+    qv[g][1] = make_float2(bf16lo(w.y) * p.sigma, bf16hi(w.y) * p.sigma);
+    qv[g][2] = make_float2(bf16lo(w.z) * p.sigma, bf16hi(w.z) * p.sigma);
+    qv[g][3] = make_float2(bf16lo(w.w) * p.sigma, bf16hi(w.w) * p.sigma);
+  }
+  __syncthreads();
+
+  // This lane's logit slot after the reduction: value index vi -> (row group, head).
+  const int vi = rl >> Gm::SHIFT;
+  const int my_rg = vi / GT;
+  const int my_g = vi % GT;
+  const int my_tl = my_rg * Gm::RPI + rs;  // token within the tile
+  const bool owner = (rl & ((1 << Gm::SHIFT) - 1)) == 0;
+
+  unsigned char* wring = ring + (size_t)warp * kStages * Gm::STAGE_BYTES;
+  uint64_t* bars = bars_all + warp * kStages;
+  float* pbuf = pbuf_all + warp * kTile * GT;
+  float* sbuf = sbuf_all + warp * GT;
+
+  const int ntiles = (cnt + kTile - 1) / kTile;
+  const int nt_w = ntiles > warp ? (ntiles - warp + kWarps - 1) / kWarps : 0;
+
+  auto issue = [&](int it) {
+    const int tile = warp + it * kWarps;
+    const int tb = tile * kTile;
+    const int ntok = min(kTile, cnt - tb);
+    const int slot = it % kStages;
+    unsigned char* st = wring + (size_t)slot * Gm::STAGE_BYTES;
+    if (lane == 0) mbar_arrive_expect_tx(&bars[slot], (uint32_t)(ntok * 2 * Gm::ROW_BYTES));
+    __syncwarp();
+    if (lane < 2 * kTile) {
+      const int t = lane & (kTile - 1);
+      if (t < ntok) {
+        const uint32_t row = rows_s[tb + t];
+        const bool isv = lane >= kTile;
+        const __nv_bfloat16* src = (isv ? p.V : p.K) + (size_t)row * D;
+        bulk_g2s(st + (size_t)(isv ? kTile + t : t) * Gm::ROW_BYTES, src, Gm::ROW_BYTES, &bars[slot]);
+      }
+    }
+  };
+
+  for (int it = 0; it < min(kStages, nt_w); ++it) issue(it);
+
+  float m_run = -INFINITY;  // running max of this lane's head
+  float l_part = 0.f;       // this lane's share of the running sum (owner lanes)
+  float acc[GT][Gm::CPL];
+#pragma unroll
+  for (int g = 0; g < GT; ++g)
+#pragma unroll
+    for (int c = 0; c < Gm::CPL; ++c) acc[g][c] = 0.f;
+  bool waited_ok = true;
+
+  for (int it = 0; it < nt_w; ++it) {
+    const int slot = it % kStages;
+    const int tb = (warp + it * kWarps) * kTile;
+    const int ntok = min(kTile, cnt - tb);
+    if (!mbar_wait_bounded(&bars[slot], (uint32_t)(it / kStages) & 1u)) waited_ok = false;
+    const unsigned char* st = wring + (size_t)slot * Gm::STAGE_BYTES;
+
+    // QK: partial dots of this lane's 8 channels, for NP rows x GT heads.
+    float v[Gm::NV];
+#pragma unroll
+    for (int rg = 0; rg < Gm::NP; ++rg) {
+      const int tl = rg * Gm::RPI + rs;
+      const uint4 w = *reinterpret_cast<const uint4*>(st + (size_t)tl * Gm::ROW_BYTES + c0 * 2);
+      const float2 k0 = make_float2(bf16lo(w.x), bf16hi(w.x));
+      const float2 k1 = make_float2(bf16lo(w.y), bf16hi(w.y));
+      const float2 k2 = make_float2(bf16lo(w.z), bf16hi(w.z));
+      const float2 k3 = make_float2(bf16lo(w.w), bf16hi(w.w));
+#pragma unroll
+      for (int g = 0; g < GT; ++g) {
+        float2 a = make_float2(0.f, 0.f);
+        a = ffma2(qv[g][0], k0, a);
+        a = ffma2(qv[g][1], k1, a);
+        a = ffma2(qv[g][2], k2, a);
+        a = ffma2(qv[g][3], k3, a);
+        v[rg * GT + g] = a.x + a.y;
+      }
+    }
+    // Reduce over the LPR lanes of each row: transposing butterfly, then plain butterfly.
+#pragma unroll
+    for (int lvl = 0; lvl < Gm::LOG_LPR; ++lvl) {
+      const int m = Gm::LPR >> (lvl + 1);
+      if (lvl < Gm::LOG_NV) {
+        const int half = Gm::NV >> (lvl + 1);
+        const bool upper = (lane & m) != 0;
+#pragma unroll
+        for (int i = 0; i < half; ++i) {
+          const float send = upper ? v[i] : v[i + half];
+          const float keep = upper ? v[i + half] : v[i];
+          v[i] = keep + __shfl_xor_sync(0xffffffffu, send, m);
+        }
+      } else {
+        v[0] += __shfl_xor_sync(0xffffffffu, v[0], m);
+      }
+    }
+    float z = v[0];
+    if (GATED) z += lg_s[tb + min(my_tl, ntok - 1)];
+    if (my_tl >= ntok) z = -INFINITY;
+
+    // Online softmax for head my_g: max over the lanes holding the same head.
+    float tmax = z;
+#pragma unroll
+    for (int m = 1; m < 32; m <<= 1) {
+      // skip lane bits that encode the head (bits SHIFT .. SHIFT+LOG_GT-1 of rl)
+      const bool head_bit = (m >= (1 << Gm::SHIFT)) && (m < (1 << (Gm::SHIFT + Gm::LOG_GT)));
+      if (!head_bit) tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, m));
+    }
+    const float m_new = fmaxf(m_run, tmax);
+    const float scale = (m_new == -INFINITY) ? 1.f : __expf(m_run - m_new);
+    const float pz = (m_new == -INFINITY) ? 0.f : __expf(z - m_new);
+    m_run = m_new;
+    if (owner) {
+      l_part = l_part * scale + pz;
+      if (my_tl < ntok) pbuf[my_tl * GT + my_g] = pz;
+      if (my_tl == 0) sbuf[my_g] = scale;
+    }
+    __syncwarp();
+
+    // PV: lane owns channels lane*CPL .. +CPL-1 of every head.
+    float sc[GT];
+#pragma unroll
+    for (int g = 0; g < GT; ++g) sc[g] = sbuf[g];
+#pragma unroll
+    for (int g = 0; g < GT; ++g)
+#pragma unroll
+      for (int c = 0; c < Gm::CPL; ++c) acc[g][c] *= sc[g];
+    const unsigned char* vst = st + (size_t)kTile * Gm::ROW_BYTES;
+    for (int tl = 0; tl < ntok; ++tl) {
+      float pw[GT];
+#pragma unroll
+      for (int g = 0; g < GT; ++g) pw[g] = pbuf[tl * GT + g];
+      if constexpr (Gm::CPL == 4) {
+        const uint2 w = *reinterpret_cast<const uint2*>(vst + (size_t)tl * Gm::ROW_BYTES + lane * 8);
+        const float2 v0 = make_float2(bf16lo(w.x), bf16hi(w.x));
+        const float2 v1 = make_float2(bf16lo(w.y), bf16hi(w.y));
+#pragma unroll
+        for (int g = 0; g < GT; ++g) {
+          const float2 pp = make_float2(pw[g], pw[g]);
+          float2 a01 = ffma2(pp, v0, make_float2(acc[g][0], acc[g][1]));
+          float2 a23 = ffma2(pp, v1, make_float2(acc[g][2], acc[g][3]));
+          acc[g][0] = a01.x; acc[g][1] = a01.y; acc[g][2] = a23.x; acc[g][3] = a23.y;
+        }
+      } else {
+        const uint32_t w = *reinterpret_cast<const uint32_t*>(vst + (size_t)tl * Gm::ROW_BYTES + lane * 4);
+        const float2 v0 = make_float2(bf16lo(w), bf16hi(w));
+#pragma unroll
+        for (int g = 0; g < GT; ++g) {
+          const float2 pp = make_float2(pw[g], pw[g]);
+          float2 a01 = ffma2(pp, v0, make_float2(acc[g][0], acc[g][1]));
+          acc[g][0] = a01.x; acc[g][1] = a01.y;
+        }
+      }
+    }
+    __syncwarp();
+    if (it + kStages < nt_w) issue(it + kStages);
+  }
+  if (!waited_ok) record_error(p.err, kDevWaitTimeout, (uint32_t)bh);
+
+  // ---- per-warp totals: l over the owner lanes of each head ----
+  float l_tot = owner ? l_part : 0.f;
+#pragma unroll
+  for (int m = 1; m < 32; m <<= 1) {
+    const bool head_bit = (m >= (1 << Gm::SHIFT)) && (m < (1 << (Gm::SHIFT + Gm::LOG_GT)));
+    if (!head_bit) l_tot += __shfl_xor_sync(0xffffffffu, l_tot, m);
+  }
+  // merge[warp][g][0..D-1] = acc, [D] = m, [D+1] = l
+  float* mw = merge + (size_t)warp * GT * (D + 2);
+#pragma unroll
+  for (int g = 0; g < GT; ++g)
+#pragma unroll
+    for (int c = 0; c < Gm::CPL; ++c) mw[g * (D + 2) + lane * Gm::CPL + c] = acc[g][c];
+  if (owner && my_tl == 0) {
+    mw[my_g * (D + 2) + D] = m_run;
+    mw[my_g * (D + 2) + D + 1] = l_tot;
+  }
+  __syncthreads();
+
+  // ---- CTA partial for this split ----
+  float* part = p.partials + ((size_t)bhz * p.splits + split) * GT * (D + 2);
+  for (int e = tid; e < GT * (D + 2); e += kThreads) {
+    const int g = e / (D + 2), c = e % (D + 2);
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) M = fmaxf(M, merge[(w * GT + g) * (D + 2) + D]);
+    float val = 0.f;
+    if (c == D) {
+      val = M;
+    } else if (M != -INFINITY) {
+#pragma unroll
+      for (int w = 0; w < kWarps; ++w) {
+        const float mwv = merge[(w * GT + g) * (D + 2) + D];
+        const float f = (mwv == -INFINITY) ? 0.f : __expf(mwv - M);
+        val += f * merge[(w * GT + g) * (D + 2) + c];
+      }
+    }
+    part[e] = val;
+  }
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) {
+    const uint32_t prev = atomicAdd(&p.counters[bhz], 1u);
+    flag[0] = (prev == (uint32_t)(p.splits - 1)) ? 1 : 0;
+  }
+  __syncthreads();
+  if (flag[0] == 0) return;
+
+  // ---- last CTA: merge the splits in split order ----
+  __threadfence();
+  const float* base = p.partials + (size_t)bhz * p.splits * GT * (D + 2);
+  if (warp < GT) {
+    const int g = warp;
+    float M = -INFINITY;
+    for (int s = lane; s < p.splits; s += 32) M = fmaxf(M, __ldcg(base + ((size_t)s * GT + g) * (D + 2) + D));
+#pragma unroll
+    for (int o = 16; o; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    float Lsum = 0.f;
+    for (int s = lane; s < p.splits; s += 32) {
+      const float ms = __ldcg(base + ((size_t)s * GT + g) * (D + 2) + D);
+      const float f = (M == -INFINITY || ms == -INFINITY) ? 0.f : __expf(ms - M);
+      wts[s * GT + g] = f;
+      Lsum += f * __ldcg(base + ((size_t)s * GT + g) * (D + 2) + D + 1);
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) Lsum += __shfl_xor_sync(0xffffffffu, Lsum, o);
+    if (lane == 0) wts[p.splits * GT + g] = (Lsum > 0.f) ? 1.f / Lsum : 0.f;
+  }
+  __syncthreads();
+  for (int e = tid; e < GT * D; e += kThreads) {
+    const int g = e / D, c = e % D;
+    float s_acc = 0.f;
+    for (int s = 0; s < p.splits; ++s) s_acc += wts[s * GT + g] * __ldcg(base + ((size_t)s * GT + g) * (D + 2) + c);
+    const int hq = h * p.G + gz * GT + g;
+    p.out[((size_t)b * p.Hq + hq) * D + c] = s_acc * wts[p.splits * GT + g];
+  }
+  if (tid == 0) p.counters[bhz] = 0u;
+}
+
+template <int D, int GT, bool GATED, bool PAGED, bool DENSE>
+cudaError_t launch_t(const AttendParams& p, cudaStream_t stream) {
+  auto kern = attend_kernel<D, GT, GATED, PAGED, DENSE>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, p.smem_bytes);
+  if (e != cudaSuccess) return e;
+  dim3 grid((unsigned)p.splits, (unsigned)(p.B * p.Hkv), (unsigned)p.ngz);
+  kern<<<grid, kThreads, (size_t)p.smem_bytes, stream>>>(p);
+  return cudaGetLastError();
+}
+
+template <int D, int GT>
+cudaError_t launch_dg(const AttendParams& p, cudaStream_t stream) {
+  const bool dense = (p.idx == nullptr);
+  const bool gated = (p.log_g != nullptr);
+  const bool paged = p.paged != 0;
+  if (dense) return paged ? launch_t<D, GT, false, true, true>(p, stream) : launch_t<D, GT, false, false, true>(p, stream);
+  if (gated) return paged ? launch_t<D, GT, true, true, false>(p, stream) : launch_t<D, GT, true, false, false>(p, stream);
+  return paged ? launch_t<D, GT, false, true, false>(p, stream) : launch_t<D, GT, false, false, false>(p, stream);
+}
+
+template <int D>
+cudaError_t launch_d(const AttendParams& p, cudaStream_t stream) {
+  switch (p.gt) {
+    case 4: return launch_dg<D, 4>(p, stream);
+    case 2: return launch_dg<D, 2>(p, stream);
+    case 1: return launch_dg<D, 1>(p, stream);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace
+
+void plan_attend(AttendParams& p, int count_max) {
+  p.gt = (p.G % 4 == 0) ? 4 : ((p.G % 2 == 0) ? 2 : 1);
+  p.ngz = p.G / p.gt;
+  const long heads = (long)p.B * p.Hkv * p.ngz;
+  if (count_max < 1) count_max = 1;
+  long s = (kTargetCtas + heads - 1) / heads;
+  if (s < 1) s = 1;
+  long len = (count_max + s - 1) / s;
+  len = (len + 31) & ~31L;
+  if (len < 32) len = 32;
+  if (len > kMaxSplitLen) len = kMaxSplitLen;
+  p.split_len = (int)len;
+  p.splits = (int)((count_max + len - 1) / len);
+  p.nstages = kStages;
+  Smem L;
+  if (p.d == 128) {
+    L = (p.gt == 4) ? smem_layout<128, 4>(p.split_len, p.splits)
+                    : (p.gt == 2 ? smem_layout<128, 2>(p.split_len, p.splits) : smem_layout<128, 1>(p.split_len, p.splits));
+  } else {
+    L = (p.gt == 4) ? smem_layout<64, 4>(p.split_len, p.splits)
+                    : (p.gt == 2 ? smem_layout<64, 2>(p.split_len, p.splits) : smem_layout<64, 1>(p.split_len, p.splits));
+  }
+  p.smem_bytes = L.total;
+}
+
+size_t attend_workspace_floats(const AttendParams& p) {
+  return (size_t)p.B * p.Hkv * p.ngz * p.splits * p.gt * (p.d + 2);
+}
+
+cudaError_t launch_attend(const AttendParams& p, cudaStream_t stream) {
+  if (p.d == 128) return launch_d<128>(p, stream);
+  if (p.d == 64) return launch_d<64>(p, stream);
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace sas

@@ -1,0 +1,83 @@
+// Kernel parameter blocks and launchers of libsas (internal; the public ABI is include/sas.h).
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+namespace sas {
+
+// ---------------------------------------------------------------------------- projection
+struct ProjParams {
+  const __nv_bfloat16* K;      // build: cache (layout below); append: K_new [B][Hkv][d]
+  const float* M;              // [Hkv][r][d]
+  __nv_bfloat16* Kproj;        // cache layout, width r
+  const int32_t* page_table;   // [B][max_pages] or null (contiguous)
+  const int32_t* seqlens;      // [B]
+  uint32_t* err;               // device error word or null
+  int B, Hkv, d, r, cap, max_pages, num_pages;
+  int paged;                   // 0 / 1 (64-token pages)
+  int append;                  // 0: build rows [0, N_b); 1: project K_new into row N_b - 1
+  int rows_per_cta;            // build: rows of one (b, h) handled by one CTA
+};
+cudaError_t launch_proj(const ProjParams& p, cudaStream_t stream);
+
+// ---------------------------------------------------------------------------- selection
+struct SelectParams {
+  const __nv_bfloat16* q;      // [B][Hq][d]
+  const float* M;              // [Hkv][r][d]
+  const __nv_bfloat16* kproj;  // cache layout, width r
+  const int32_t* page_table;
+  const int32_t* seqlens;
+  const int32_t* kvec;         // [B]
+  const float* log_g;          // [B][Hkv][cap] or null
+  int32_t* idx_out;            // [B][Hkv][k_max]
+  float* scores_out;           // [B][Hkv][cap] or null
+  uint32_t* err;
+  int B, Hq, Hkv, G, d, r, cap, max_pages, num_pages, paged, k_max;
+  float sigma, lam;
+  int cluster;                 // CTAs per (b, h)
+  int chunk;                   // max positions per CTA (multiple of 512)
+  int nstages;                 // bulk-copy ring depth
+  int stage_bytes;             // bytes per ring stage
+  int off_ring, off_q, off_bar, off_ctl, smem_bytes;
+};
+// Chooses cluster size, chunk and ring depth for a shape; returns false if unsupported.
+bool plan_select(SelectParams& p, int num_sms);
+cudaError_t launch_select(const SelectParams& p, cudaStream_t stream);
+
+// ---------------------------------------------------------------------------- attention
+struct AttendParams {
+  const __nv_bfloat16* q;      // [B][Hq][d]
+  const __nv_bfloat16* K;      // cache layout
+  const __nv_bfloat16* V;
+  const int32_t* page_table;
+  const int32_t* seqlens;
+  const int32_t* idx;          // [B][Hkv][k_max]; null for the dense (all positions) variant
+  const int32_t* kvec;         // [B]; null for dense
+  const float* log_g;          // [B][Hkv][cap] or null
+  float* out;                  // [B][Hq][d]
+  float* partials;             // workspace: [B*Hkv*ngz][splits][gt][d + 2]
+  uint32_t* counters;          // workspace: [B*Hkv*ngz]
+  uint32_t* err;
+  int B, Hq, Hkv, G, d, cap, max_pages, num_pages, paged, k_max;
+  float sigma, lam;
+  int gt;                      // query heads per CTA (1, 2 or 4)
+  int ngz;                     // G / gt
+  int splits;                  // CTAs per (b, h, head group)
+  int split_len;               // index-list entries per CTA (multiple of 32)
+  int nstages;
+  int smem_bytes;
+};
+// Split plan for `count_max` index entries per head; pure function of the arguments.
+void plan_attend(AttendParams& p, int count_max);
+size_t attend_workspace_floats(const AttendParams& p);
+cudaError_t launch_attend(const AttendParams& p, cudaStream_t stream);
+
+constexpr int kTargetCtas = 1024;   // attention split planning target (device independent)
+constexpr int kMaxSplitLen = 2048;  // index entries per attention CTA at most
+constexpr int kMaxChunk = 16384;    // positions per selection CTA at most
+constexpr int kMaxCluster = 16;
+
+}  // namespace sas
