@@ -220,7 +220,8 @@ def make_problem(
     else:
         max_pages = 0
         num_pages = 0
-        n_cap_eff = int(n_cap) if n_cap is not None else max(1, max(seqlens))
+        # default capacity: the longest sequence, rounded up to a multiple of 4 rows
+        n_cap_eff = int(n_cap) if n_cap is not None else (max(1, max(seqlens)) + 3) // 4 * 4
         assert n_cap_eff >= max(seqlens)
         kv_shape = (B, Hkv, n_cap_eff, d)
     K = _gauss_bf16(kv_shape, seed, "K", device, scale=scale)

@@ -25,6 +25,28 @@ def bf16_ulp_diff(a, b):
     return np.abs(ordered(a) - ordered(b))
 
 
+def bf16_ulp(x):
+    """Spacing of bf16 values at |x| (2**(e-8) for x = m 2**e, 0.5 <= m < 1)."""
+    _, e = np.frexp(np.abs(np.asarray(x, np.float64)))
+    return np.ldexp(1.0, np.maximum(e - 8, -133))
+
+
+def check_build_rows(kp_g, kp_o, a, p):
+    """GPU projected rows vs the oracle's correctly rounded ones.
+
+    The kernel accumulates d products in fp32 (error at most d * 2**-24 * sum_c |M_jc K_c|)
+    and rounds once to bf16, the oracle rounds the exact sum: they may differ by that error
+    plus one bf16 spacing."""
+    mask = _rows_mask(p, a)
+    Kabs = np.abs(a["K"])[mask]                         # [rows, d]
+    heads = np.nonzero(mask)[1]                         # KV head of each row
+    Mabs = np.abs(a["M"])[heads]                        # [rows, r, d]
+    acc_bound = p.d * 2.0 ** -24 * np.einsum("nrd,nd->nr", Mabs, Kabs)
+    g, o = kp_g[mask], kp_o[mask]
+    tol = bf16_ulp(np.maximum(np.abs(g), np.abs(o))) + 1.01 * acc_bound
+    assert np.all(np.abs(g - o) <= tol), f"build: worst {np.max(np.abs(g - o) / tol):.3f} of bound"
+
+
 def kproj_tensor(kp_np, device):
     return torch.from_numpy(np.ascontiguousarray(kp_np)).to(torch.float32).to(torch.bfloat16).to(device)
 
@@ -95,12 +117,9 @@ def run_small(p_cpu, device="cuda", dense=True, check_build=True):
     if check_build:
         kp_g = torch.zeros_like(kp_in)
         lib.sas_build_proj_cache(shape, p.K, p.M, kp_g, p.page_table, p.seqlens)
-        kg = f64(kp_g)
-        mask = _rows_mask(p, a)
-        ulp = bf16_ulp_diff(kg[mask], kp_o[mask])
-        assert ulp.max(initial=0) <= 1, f"build: {ulp.max()} ulp"
-        stats["build_ulp1_frac"] = float((ulp > 0).mean()) if ulp.size else 0.0
-        assert stats["build_ulp1_frac"] <= 1e-2
+        check_build_rows(f64(kp_g), kp_o, a, p)
+        ulp = bf16_ulp_diff(f64(kp_g)[_rows_mask(p, a)], kp_o[_rows_mask(p, a)])
+        stats["build_ulp_frac"] = float((ulp > 0).mean()) if ulp.size else 0.0
 
     scores = torch.full((p.B, p.Hkv, p.cap), float("nan"), dtype=torch.float32, device=device)
     idx_sel = torch.full((p.B, p.Hkv, p.k_max), -7, dtype=torch.int32, device=device)
@@ -157,8 +176,9 @@ def run_sampled(p, heads, device="cuda", dense_heads=None):
         a = _head_arrays(p, b, h, n, pt, seqlens, ks)
         kp_rows_g = _head_rows(kp, b, h, n, pt)
         kp_rows_o = O.project_keys(a["K"][0, 0, :n], a["M"][0])
-        ulp = bf16_ulp_diff(kp_rows_g, kp_rows_o)
-        assert ulp.max(initial=0) <= 1
+        acc_bound = p.d * 2.0 ** -24 * (np.abs(a["K"][0, 0, :n]) @ np.abs(a["M"][0]).T)
+        tol = bf16_ulp(np.maximum(np.abs(kp_rows_g), np.abs(kp_rows_o))) + 1.01 * acc_bound
+        assert np.all(np.abs(kp_rows_g - kp_rows_o) <= tol), "build rows outside the fp32 bound"
         if np.array_equal(f64(p.M[h]), np.eye(p.d)[: p.r]):
             assert np.array_equal(kp_rows_g, kp_rows_o), "identity basis must copy channels exactly"
         ndiff += compare_head(_HeadView(p), a, 0, 0, kp_rows_o, f64(idx[b, h]), f64(out[b, h * G:(h + 1) * G]))

@@ -107,8 +107,10 @@ __global__ void __launch_bounds__(kThreads) select_topk_kernel(const SelectParam
   const int k_eff = max(0, min(kb, n));
   int32_t* idx = p.idx_out + (size_t)bh * p.k_max;
 
-  // Nothing to rank: empty selection, or every position selected.  Uniform per cluster.
-  if (k_eff == 0 || (k_eff == n && p.scores_out == nullptr)) {
+  // Nothing to rank: empty selection, or every position selected (scores still computed when
+  // they are requested).  Uniform per cluster.
+  const bool want_scores = (p.scores_out != nullptr) && n > 0;
+  if (!want_scores && (k_eff == 0 || k_eff == n)) {
     for (int j = rank * kThreads + tid; j < p.k_max; j += C * kThreads) idx[j] = (j < k_eff) ? j : -1;
     return;
   }
@@ -237,6 +239,11 @@ __global__ void __launch_bounds__(kThreads) select_topk_kernel(const SelectParam
     if (tid == 0 && s + p.nstages < nst) issue(s + p.nstages);
   }
   if (!waited_ok) record_error(p.err, kDevWaitTimeout, (uint32_t)bh);
+
+  if (k_eff == 0) {  // scores were requested, nothing is selected (uniform per cluster)
+    for (int j = rank * kThreads + tid; j < p.k_max; j += C * kThreads) idx[j] = -1;
+    return;
+  }
 
   // ---- 3. radix select across the cluster ----
   for (int i = tid; i < 2 * kBins; i += kThreads) hist_local[i] = 0u;
