@@ -146,14 +146,14 @@ def smi_device_id(torch, dev):
 
 # ------------------------------------------------------------------------------ our arm
 class Workload:
-    def __init__(self, name, device, torch):
+    def __init__(self, name, device, torch, batch=None):
         from synth import CONFIGS, make_config
         from token_level_sparse_head_b200 import DecodeSession, lib, shape_of
 
         self.name = name
         self.torch = torch
         self.lib = lib
-        p = make_config(name, device=device)
+        p = make_config(name, device=device, **({"B": batch} if batch else {}))
         self.p = p
         self.shape = shape_of(p)
         self.sess = DecodeSession(self.shape, p.k_max, device=device)
@@ -262,7 +262,7 @@ def run_ours(args):
     dev = f"cuda:{local}"
     peak, peak_kind = measured_peaks()
 
-    wl = Workload(args.workload, dev, torch)
+    wl = Workload(args.workload, dev, torch, batch=args.batch)
     p = wl.p
     for _ in range(args.warmup):
         wl.step()
@@ -334,9 +334,18 @@ def run_ours(args):
             w1.step()
         t1 = flushed_steps(torch, w1.step, max(10, min(args.steps, 100)), flush)
         td1 = flushed_steps(torch, w1.dense, 10, flush)
+        kt = {"append": [], "select": [], "attend": []}
+        for _ in range(20):
+            flush.zero_()
+            ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+            w1.step_parts(ev)
+            torch.cuda.synchronize()
+            for i, kname in enumerate(("append", "select", "attend")):
+                kt[kname].append(ev[i].elapsed_time(ev[i + 1]))
         secondary = {"workload": SECONDARY_WORKLOAD, "ms_per_step": t1 * 1e3, "steps_per_s": 1.0 / t1,
                      "hbm_gbs": w1.bytes["step"] / t1 / 1e9, "dense_ms_per_step": td1 * 1e3,
-                     "speedup_vs_dense": td1 / t1, "l2": "flushed between steps (2x L2 write)"}
+                     "speedup_vs_dense": td1 / t1, "l2": "flushed between steps (2x L2 write)",
+                     "kernels_ms": {kname: statistics.median(v) for kname, v in kt.items()}}
         wl = w1
 
     cpu = None
@@ -361,7 +370,7 @@ def run_ours(args):
         "roofline": {"kernel": dom, "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "peak_kind": peak_kind,
                      "algorithmic_bytes_per_launch": dom_bytes, "traffic": traffic},
-        "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": 3 * args.steps, "clocks": clocks,
+        "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": 4 * args.steps, "clocks": clocks,
     }
     line["hbm_gbs"] = head_bytes["step"] / (ms * 1e-3) / 1e9
     line["step_roofline_frac"] = line["hbm_gbs"] / peak
@@ -477,6 +486,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--batch", type=int, default=None, help="override the workload's batch (profiling)")
     ap.add_argument("--no-secondary", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)

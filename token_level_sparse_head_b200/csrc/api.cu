@@ -68,7 +68,6 @@ int num_sms() {
   return n;
 }
 
-// Workspace: [0,256) error word | counters (uint32, 256-aligned) | partials (fp32)
 constexpr size_t kErrBytes = 256;
 
 sas::AttendParams attend_plan(const sas_shape* s, int count_max) {
@@ -79,19 +78,37 @@ sas::AttendParams attend_plan(const sas_shape* s, int count_max) {
   return a;
 }
 
-size_t ws_bytes_for(const sas::AttendParams& a) {
-  size_t cnt = (size_t)a.B * a.Hkv * a.ngz * 4;
-  cnt = (cnt + 255) & ~(size_t)255;
-  return kErrBytes + cnt + sas::attend_workspace_floats(a) * 4;
+// Workspace: [0,256) error word | key histograms | counters | attention partials | score keys.
+// The histograms and counters sit at fixed offsets: they must stay zero between calls (the
+// kernels clear them after use), whatever other calls (dense decode, other budgets) share the
+// workspace; partials and keys are rewritten by every call.
+struct WsLayout {
+  size_t hist, counters, partials, keys, total;
+};
+
+WsLayout ws_layout(const sas::AttendParams& a, bool with_keys) {
+  WsLayout w;
+  size_t o = kErrBytes;
+  w.hist = o;
+  o += (size_t)a.B * a.Hkv * 2048 * 4;
+  w.counters = o;
+  o += ((size_t)a.B * a.Hkv * a.ngz * 4 + 255) & ~(size_t)255;
+  w.partials = o;
+  o += (sas::attend_workspace_floats(a) * 4 + 255) & ~(size_t)255;
+  w.keys = o;
+  if (with_keys) o += ((size_t)a.B * a.Hkv * a.cap * 4 + 255) & ~(size_t)255;
+  w.total = o;
+  return w;
 }
+
+size_t ws_bytes_for(const sas::AttendParams& a, bool with_keys) { return ws_layout(a, with_keys).total; }
 
 void bind_workspace(sas::AttendParams& a, void* ws) {
   unsigned char* w = static_cast<unsigned char*>(ws);
-  size_t cnt = (size_t)a.B * a.Hkv * a.ngz * 4;
-  cnt = (cnt + 255) & ~(size_t)255;
+  const WsLayout L = ws_layout(a, false);
   a.err = reinterpret_cast<uint32_t*>(w);
-  a.counters = reinterpret_cast<uint32_t*>(w + kErrBytes);
-  a.partials = reinterpret_cast<float*>(w + kErrBytes + cnt);
+  a.counters = reinterpret_cast<uint32_t*>(w + L.counters);
+  a.partials = reinterpret_cast<float*>(w + L.partials);
 }
 
 sas_status check_cache_ptrs(const sas_shape* s, const int32_t* page_table, const int32_t* seqlens) {
@@ -102,9 +119,14 @@ sas_status check_cache_ptrs(const sas_shape* s, const int32_t* page_table, const
 
 sas_status do_select(const sas_shape* s, const void* q, const float* M, const void* Kproj,
                      const int32_t* page_table, const int32_t* seqlens, const int32_t* k, int32_t k_max,
-                     float lambda, const float* log_g, int32_t* idx_out, float* scores_out, uint32_t* err,
+                     float lambda, const float* log_g, int32_t* idx_out, float* scores_out, void* ws,
                      cudaStream_t st) {
-  sas::SelectParams sp = {};
+  const sas::AttendParams a = attend_plan(s, k_max);
+  const WsLayout L = ws_layout(a, true);
+  unsigned char* w = static_cast<unsigned char*>(ws);
+  const int sms = num_sms();
+
+  sas::ScoreParams sp = {};
   sp.q = static_cast<const __nv_bfloat16*>(q);
   sp.M = M;
   sp.kproj = static_cast<const __nv_bfloat16*>(Kproj);
@@ -112,17 +134,31 @@ sas_status do_select(const sas_shape* s, const void* q, const float* M, const vo
   sp.seqlens = seqlens;
   sp.kvec = k;
   sp.log_g = (lambda != 0.0f) ? log_g : nullptr;
-  sp.idx_out = idx_out;
+  sp.keys = reinterpret_cast<uint32_t*>(w + L.keys);
+  sp.hist = reinterpret_cast<uint32_t*>(w + L.hist);
   sp.scores_out = scores_out;
-  sp.err = err;
+  sp.err = reinterpret_cast<uint32_t*>(w);
   sp.B = s->B; sp.Hq = s->Hq; sp.Hkv = s->Hkv; sp.G = s->Hq / s->Hkv; sp.d = s->d; sp.r = s->r;
   sp.cap = cap_of(s);
   sp.max_pages = s->max_pages; sp.num_pages = s->num_pages; sp.paged = s->page_size ? 1 : 0;
   sp.k_max = k_max;
   sp.sigma = 1.0f / sqrtf((float)s->d);
   sp.lam = lambda;
-  if (!sas::plan_select(sp, num_sms())) return fail(SAS_ERR_UNSUPPORTED, "no selection plan for this shape");
-  const cudaError_t e = sas::launch_select(sp, st);
+  sas::plan_score(sp, sms);
+
+  sas::SelectParams sl = {};
+  sl.keys = sp.keys;
+  sl.hist = sp.hist;
+  sl.seqlens = seqlens;
+  sl.kvec = k;
+  sl.idx_out = idx_out;
+  sl.err = sp.err;
+  sl.B = s->B; sl.Hkv = s->Hkv; sl.cap = sp.cap; sl.k_max = k_max;
+  if (!sas::plan_select(sl, sms)) return fail(SAS_ERR_UNSUPPORTED, "no selection plan for this shape");
+
+  cudaError_t e = sas::launch_score(sp, st);
+  if (e != cudaSuccess) return cuda_fail(e, "score kernel launch");
+  e = sas::launch_select(sl, st);
   if (e != cudaSuccess) return cuda_fail(e, "select kernel launch");
   return SAS_OK;
 }
@@ -171,12 +207,12 @@ const char* sas_last_error_detail(void) { return g_detail; }
 
 size_t sas_decode_workspace_bytes(const sas_shape* shape, int32_t k_max) {
   if (check_shape(shape) != SAS_OK || k_max < 1) return 0;
-  return ws_bytes_for(attend_plan(shape, k_max));
+  return ws_bytes_for(attend_plan(shape, k_max), true);
 }
 
 size_t sas_dense_workspace_bytes(const sas_shape* shape) {
   if (check_shape(shape) != SAS_OK) return 0;
-  return ws_bytes_for(attend_plan(shape, cap_of(shape)));
+  return ws_bytes_for(attend_plan(shape, cap_of(shape)), false);
 }
 
 sas_status sas_workspace_init(void* workspace, size_t ws_bytes, void* stream) {
@@ -260,7 +296,7 @@ sas_status sas_select_topk(const sas_shape* shape, const void* q, const float* M
   SAS_TRY(check_ptr(workspace, "workspace"));
   if (ws_bytes < sas_decode_workspace_bytes(shape, k_max)) return fail(SAS_ERR_INVALID_ARG, "workspace too small");
   return do_select(shape, q, M, Kproj, page_table, seqlens, k, k_max, lambda, log_g, idx_out, scores_out,
-                   static_cast<uint32_t*>(workspace), static_cast<cudaStream_t>(stream));
+                   workspace, static_cast<cudaStream_t>(stream));
 }
 
 sas_status sas_sparse_attention(const sas_shape* shape, const void* q, const void* K, const void* V,
@@ -303,7 +339,7 @@ sas_status sas_decode_step(const sas_shape* shape, const void* q, const float* M
   if (ws_bytes < sas_decode_workspace_bytes(shape, k_max)) return fail(SAS_ERR_INVALID_ARG, "workspace too small");
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   SAS_TRY(do_select(shape, q, M, Kproj, page_table, seqlens, k, k_max, lambda, log_g, idx_out, nullptr,
-                    static_cast<uint32_t*>(workspace), st));
+                    workspace, st));
   return do_attend(shape, q, K, V, page_table, seqlens, idx_out, k, k_max, lambda, log_g, out, workspace, st);
 }
 

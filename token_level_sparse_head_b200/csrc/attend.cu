@@ -103,26 +103,50 @@ __global__ void __launch_bounds__(kThreads) attend_kernel(const AttendParams p) 
   const int j1 = min(j0 + p.split_len, count);
   const int cnt = max(0, j1 - j0);
 
-  // ---- resolve the slice's rows (and gate terms) once ----
-  for (int j = tid; j < cnt; j += kThreads) {
-    int i = DENSE ? (j0 + j) : p.idx[(size_t)bh * p.k_max + j0 + j];
-    if (!DENSE && (i < 0 || i >= n)) {
-      record_error(p.err, kDevBadIndex, (uint32_t)bh);
-      i = 0;
+  // ---- resolve the slice's rows (and gate terms) once; loads batched 4 per thread ----
+  for (int jb = 0; jb < cnt; jb += 4 * kThreads) {
+    int iv[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int j = jb + u * kThreads + tid;
+      iv[u] = (j < cnt) ? (DENSE ? (j0 + j) : p.idx[(size_t)bh * p.k_max + j0 + j]) : 0;
     }
-    uint32_t row;
-    if (PAGED) {
-      int pg = p.page_table[(size_t)b * p.max_pages + (i >> 6)];
-      if (pg < 0 || pg >= p.num_pages) {
-        record_error(p.err, kDevBadPage, (uint32_t)b);
-        pg = 0;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      if (!DENSE && (iv[u] < 0 || iv[u] >= n)) {
+        record_error(p.err, kDevBadIndex, (uint32_t)bh);
+        iv[u] = 0;
       }
-      row = ((uint32_t)pg * (uint32_t)p.Hkv + (uint32_t)h) * 64u + (uint32_t)(i & 63);
-    } else {
-      row = (uint32_t)bh * (uint32_t)p.cap + (uint32_t)i;
     }
-    rows_s[j] = row;
-    if (GATED) lg_s[j] = p.lam * p.log_g[(size_t)bh * p.cap + i];
+    int pg[4] = {0, 0, 0, 0};
+    float lgv[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int j = jb + u * kThreads + tid;
+      if (j < cnt) {
+        if (PAGED) pg[u] = p.page_table[(size_t)b * p.max_pages + (iv[u] >> 6)];
+        if (GATED) lgv[u] = p.log_g[(size_t)bh * p.cap + iv[u]];
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int j = jb + u * kThreads + tid;
+      if (j < cnt) {
+        uint32_t row;
+        if (PAGED) {
+          int g = pg[u];
+          if (g < 0 || g >= p.num_pages) {
+            record_error(p.err, kDevBadPage, (uint32_t)b);
+            g = 0;
+          }
+          row = ((uint32_t)g * (uint32_t)p.Hkv + (uint32_t)h) * 64u + (uint32_t)(iv[u] & 63);
+        } else {
+          row = (uint32_t)bh * (uint32_t)p.cap + (uint32_t)iv[u];
+        }
+        rows_s[j] = row;
+        if (GATED) lg_s[j] = p.lam * lgv[u];
+      }
+    }
   }
   if (lane == 0) {
     for (int s = 0; s < kStages; ++s) mbar_init(&bars_all[warp * kStages + s], 1);
@@ -168,7 +192,15 @@ __global__ void __launch_bounds__(kThreads) attend_kernel(const AttendParams p) 
     unsigned char* st = wring + (size_t)slot * Gm::STAGE_BYTES;
     if (lane == 0) mbar_arrive_expect_tx(&bars[slot], (uint32_t)(ntok * 2 * Gm::ROW_BYTES));
     __syncwarp();
-    if (lane < 2 * kTile) {
+    if (DENSE) {
+      // A tile is 8 consecutive positions starting at a multiple of 8: consecutive rows of the
+      // cache (within one 64-token page for the paged layout), fetched as one copy each.
+      if (lane < 2) {
+        const uint32_t row = rows_s[tb];
+        const __nv_bfloat16* src = (lane ? p.V : p.K) + (size_t)row * D;
+        bulk_g2s(st + (size_t)(lane ? kTile : 0) * Gm::ROW_BYTES, src, (uint32_t)(ntok * Gm::ROW_BYTES), &bars[slot]);
+      }
+    } else if (lane < 2 * kTile) {
       const int t = lane & (kTile - 1);
       if (t < ntok) {
         const uint32_t row = rows_s[tb + t];
@@ -316,8 +348,10 @@ __global__ void __launch_bounds__(kThreads) attend_kernel(const AttendParams p) 
   }
   __syncthreads();
 
-  // ---- CTA partial for this split ----
-  float* part = p.partials + ((size_t)bhz * p.splits + split) * GT * (D + 2);
+  // ---- CTA partial for this split: acc [GT][D] and (m, l) [GT][2] ----
+  const size_t nheads = (size_t)p.B * p.Hkv * p.ngz;
+  float* pacc = p.partials + ((size_t)bhz * p.splits + split) * GT * D;
+  float* pml = p.partials + nheads * p.splits * GT * D + ((size_t)bhz * p.splits + split) * GT * 2;
   for (int e = tid; e < GT * (D + 2); e += kThreads) {
     const int g = e / (D + 2), c = e % (D + 2);
     float M = -INFINITY;
@@ -334,7 +368,8 @@ __global__ void __launch_bounds__(kThreads) attend_kernel(const AttendParams p) 
         val += f * merge[(w * GT + g) * (D + 2) + c];
       }
     }
-    part[e] = val;
+    if (c < D) pacc[g * D + c] = val;
+    else pml[g * 2 + (c - D)] = val;
   }
   __threadfence();
   __syncthreads();
@@ -345,33 +380,71 @@ __global__ void __launch_bounds__(kThreads) attend_kernel(const AttendParams p) 
   __syncthreads();
   if (flag[0] == 0) return;
 
-  // ---- last CTA: merge the splits in split order ----
+  // ---- last CTA: merge the splits (fixed order: deterministic) ----
   __threadfence();
-  const float* base = p.partials + (size_t)bhz * p.splits * GT * (D + 2);
+  const float* bacc = p.partials + (size_t)bhz * p.splits * GT * D;
+  const float* bml = p.partials + nheads * p.splits * GT * D + (size_t)bhz * p.splits * GT * 2;
   if (warp < GT) {
     const int g = warp;
     float M = -INFINITY;
-    for (int s = lane; s < p.splits; s += 32) M = fmaxf(M, __ldcg(base + ((size_t)s * GT + g) * (D + 2) + D));
+    for (int s = lane; s < p.splits; s += 32) M = fmaxf(M, __ldcg(bml + ((size_t)s * GT + g) * 2));
 #pragma unroll
     for (int o = 16; o; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
     float Lsum = 0.f;
     for (int s = lane; s < p.splits; s += 32) {
-      const float ms = __ldcg(base + ((size_t)s * GT + g) * (D + 2) + D);
-      const float f = (M == -INFINITY || ms == -INFINITY) ? 0.f : __expf(ms - M);
+      const float2 ml = __ldcg(reinterpret_cast<const float2*>(bml + ((size_t)s * GT + g) * 2));
+      const float f = (M == -INFINITY || ml.x == -INFINITY) ? 0.f : __expf(ml.x - M);
       wts[s * GT + g] = f;
-      Lsum += f * __ldcg(base + ((size_t)s * GT + g) * (D + 2) + D + 1);
+      Lsum += f * ml.y;
     }
 #pragma unroll
     for (int o = 16; o; o >>= 1) Lsum += __shfl_xor_sync(0xffffffffu, Lsum, o);
     if (lane == 0) wts[p.splits * GT + g] = (Lsum > 0.f) ? 1.f / Lsum : 0.f;
   }
   __syncthreads();
+  // Warp w sums splits w, w+4, ...; lane owns OPL consecutive outputs (one head).
+  constexpr int OPL = GT * D / 32;
+  const int e0 = lane * OPL;
+  const int gl = e0 / D;
+  float racc[OPL];
+#pragma unroll
+  for (int i = 0; i < OPL; ++i) racc[i] = 0.f;
+  int s = warp;
+  if constexpr (OPL % 4 == 0) {
+    for (; s + kWarps < p.splits; s += 2 * kWarps) {
+      const float4* a = reinterpret_cast<const float4*>(bacc + (size_t)s * GT * D + e0);
+      const float4* bb = reinterpret_cast<const float4*>(bacc + (size_t)(s + kWarps) * GT * D + e0);
+      float4 va[OPL / 4], vb[OPL / 4];
+#pragma unroll
+      for (int i = 0; i < OPL / 4; ++i) { va[i] = __ldcg(a + i); vb[i] = __ldcg(bb + i); }
+      const float wa = wts[s * GT + gl], wb = wts[(s + kWarps) * GT + gl];
+#pragma unroll
+      for (int i = 0; i < OPL / 4; ++i) {
+        racc[4 * i + 0] += wa * va[i].x + wb * vb[i].x;
+        racc[4 * i + 1] += wa * va[i].y + wb * vb[i].y;
+        racc[4 * i + 2] += wa * va[i].z + wb * vb[i].z;
+        racc[4 * i + 3] += wa * va[i].w + wb * vb[i].w;
+      }
+    }
+  }
+  for (; s < p.splits; s += kWarps) {
+    const float* a = bacc + (size_t)s * GT * D + e0;
+    const float wa = wts[s * GT + gl];
+#pragma unroll
+    for (int i = 0; i < OPL; ++i) racc[i] += wa * __ldcg(a + i);
+  }
+  float* red = merge;  // reuse: [kWarps][GT * D]
+  __syncthreads();
+#pragma unroll
+  for (int i = 0; i < OPL; ++i) red[warp * GT * D + e0 + i] = racc[i];
+  __syncthreads();
   for (int e = tid; e < GT * D; e += kThreads) {
     const int g = e / D, c = e % D;
-    float s_acc = 0.f;
-    for (int s = 0; s < p.splits; ++s) s_acc += wts[s * GT + g] * __ldcg(base + ((size_t)s * GT + g) * (D + 2) + c);
+    float v = 0.f;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) v += red[w * GT * D + e];
     const int hq = h * p.G + gz * GT + g;
-    p.out[((size_t)b * p.Hq + hq) * D + c] = s_acc * wts[p.splits * GT + g];
+    p.out[((size_t)b * p.Hq + hq) * D + c] = v * wts[p.splits * GT + g];
   }
   if (tid == 0) p.counters[bhz] = 0u;
 }
@@ -417,7 +490,9 @@ void plan_attend(AttendParams& p, int count_max) {
   if (s < 1) s = 1;
   long len = (count_max + s - 1) / s;
   len = (len + 31) & ~31L;
-  if (len < 32) len = 32;
+  if (len < 128) len = 128;
+  const long cm32 = ((long)count_max + 31) & ~31L;
+  if (len > cm32) len = cm32;
   if (len > kMaxSplitLen) len = kMaxSplitLen;
   p.split_len = (int)len;
   p.splits = (int)((count_max + len - 1) / len);

@@ -7,9 +7,10 @@
 //
 // build : every cached row i < N_b of every (b, h), one thread per row, M[h] staged in shared
 //         memory and read as broadcast float4s;
-// append: the newest key of every (b, h), one warp per (b, h), one lane per output element.
-// Both accumulate each output in fp32 in channel order c = 0..d-1 (so an appended row is
-// bit-identical to the same row built), then round to bf16 (nearest even).
+// append: the newest key of every (b, h), one CTA per (b, h), 8 threads per output element.
+// Both use one summation order for each output: 8 partial sums over consecutive blocks of d/8
+// channels (fp32, in channel order), combined as ((p0+p1)+(p2+p3))+((p4+p5)+(p6+p7)), then
+// rounded to bf16 (nearest even); so an appended row is bit-identical to the same row built.
 #include "sas_device.cuh"
 #include "sas_kernels.h"
 
@@ -46,30 +47,40 @@ __global__ void __launch_bounds__(kBuildThreads) build_kernel(const ProjParams p
   } else {
     row = (size_t)bh * p.cap + i;
   }
-  // The key row is re-read (L1-resident) once per block of 16 outputs, 4 channels at a time.
+  // The key row is re-read (L1-resident) for each block of outputs, 4 channels at a time.
   const uint2* src = reinterpret_cast<const uint2*>(p.K + row * D);
+  constexpr int BLK = D / 8;  // channels per partial sum
+  constexpr int JB = 4;       // outputs per pass
   uint32_t outw[R / 2];
-  constexpr int JB = 16;
 #pragma unroll
   for (int jb = 0; jb < R; jb += JB) {
+    float part[JB][8];
+#pragma unroll
+    for (int blk = 0; blk < 8; ++blk) {
+#pragma unroll
+      for (int jj = 0; jj < JB; ++jj) part[jj][blk] = 0.f;
+#pragma unroll
+      for (int c4 = blk * BLK / 4; c4 < (blk + 1) * BLK / 4; ++c4) {
+        const uint2 kk = src[c4];
+        const float k0 = bf16lo(kk.x), k1 = bf16hi(kk.x);
+        const float k2 = bf16lo(kk.y), k3 = bf16hi(kk.y);
+#pragma unroll
+        for (int jj = 0; jj < JB; ++jj) {
+          const float4 m = reinterpret_cast<const float4*>(Ms + (size_t)(jb + jj) * D)[c4];
+          float a = part[jj][blk];
+          a = fmaf(m.x, k0, a);
+          a = fmaf(m.y, k1, a);
+          a = fmaf(m.z, k2, a);
+          a = fmaf(m.w, k3, a);
+          part[jj][blk] = a;
+        }
+      }
+    }
     float acc[JB];
 #pragma unroll
-    for (int jj = 0; jj < JB; ++jj) acc[jj] = 0.f;
-#pragma unroll 4
-    for (int c4 = 0; c4 < D / 4; ++c4) {
-      const uint2 kk = src[c4];
-      const float k0 = bf16lo(kk.x), k1 = bf16hi(kk.x);
-      const float k2 = bf16lo(kk.y), k3 = bf16hi(kk.y);
-#pragma unroll
-      for (int jj = 0; jj < JB; ++jj) {
-        const float4 m = reinterpret_cast<const float4*>(Ms + (size_t)(jb + jj) * D)[c4];
-        float a = acc[jj];
-        a = fmaf(m.x, k0, a);
-        a = fmaf(m.y, k1, a);
-        a = fmaf(m.z, k2, a);
-        a = fmaf(m.w, k3, a);
-        acc[jj] = a;
-      }
+    for (int jj = 0; jj < JB; ++jj) {
+      const float* q = part[jj];
+      acc[jj] = ((q[0] + q[1]) + (q[2] + q[3])) + ((q[4] + q[5]) + (q[6] + q[7]));
     }
 #pragma unroll
     for (int jj = 0; jj < JB; jj += 2) {
@@ -82,49 +93,70 @@ __global__ void __launch_bounds__(kBuildThreads) build_kernel(const ProjParams p
   for (int v = 0; v < R / 8; ++v) dst[v] = make_uint4(outw[4 * v], outw[4 * v + 1], outw[4 * v + 2], outw[4 * v + 3]);
 }
 
-// One warp per (b, h): lane j computes outputs j, j+32.
+// One CTA per (b, h); thread t computes the partial of output j = t / 8 (+32 per pass) over
+// channel block t % 8, and the 8 partials meet in a butterfly.
 template <int D, int R>
 __global__ void __launch_bounds__(256) append_kernel(const ProjParams p) {
-  __shared__ float ks[8][D];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int bh = blockIdx.x * 8 + warp;
-  if (bh >= p.B * p.Hkv) return;
+  const int bh = blockIdx.x;
   const int b = bh / p.Hkv, h = bh % p.Hkv;
   const int n = p.seqlens[b];
   if (n < 0 || n > p.cap) {
-    if (lane == 0 && h == 0) record_error(p.err, kDevBadSeqlen, (uint32_t)b);
+    if (threadIdx.x == 0 && h == 0) record_error(p.err, kDevBadSeqlen, (uint32_t)b);
     return;
   }
   if (n == 0) return;
   const int i = n - 1;
-  const __nv_bfloat16* kn = p.K + (size_t)bh * D;
-  for (int c = lane; c < D; c += 32) ks[warp][c] = __bfloat162float(kn[c]);
-  __syncwarp();
   size_t row;
   if (p.paged) {
     const int pg = p.page_table[(size_t)b * p.max_pages + (i >> 6)];
     if (pg < 0 || pg >= p.num_pages) {
-      if (lane == 0) record_error(p.err, kDevBadPage, (uint32_t)b);
+      if (threadIdx.x == 0) record_error(p.err, kDevBadPage, (uint32_t)b);
       return;
     }
     row = ((size_t)pg * p.Hkv + h) * 64 + (i & 63);
   } else {
     row = (size_t)bh * p.cap + i;
   }
+  constexpr int BLK = D / 8;
+  const int part = threadIdx.x & 7;
+  float kf[BLK];
+  {
+    const uint32_t* kn = reinterpret_cast<const uint32_t*>(p.K + (size_t)bh * D + part * BLK);
 #pragma unroll
-  for (int j = lane; j < R; j += 32) {
-    const float* Mj = p.M + ((size_t)h * R + j) * D;
-    float a = 0.f;
-    for (int c = 0; c < D; ++c) a = fmaf(Mj[c], ks[warp][c], a);
-    p.Kproj[row * R + j] = __float2bfloat16_rn(a);
+    for (int e = 0; e < BLK / 2; ++e) {
+      const uint32_t w = kn[e];
+      kf[2 * e] = bf16lo(w);
+      kf[2 * e + 1] = bf16hi(w);
+    }
+  }
+#pragma unroll
+  for (int pass = 0; pass < (R + 31) / 32; ++pass) {
+    const int j = threadIdx.x / 8 + pass * 32;
+    if (j < R) {
+      const float4* Mj = reinterpret_cast<const float4*>(p.M + ((size_t)h * R + j) * D + part * BLK);
+      float4 m[BLK / 4];
+#pragma unroll
+      for (int e = 0; e < BLK / 4; ++e) m[e] = Mj[e];
+      float a = 0.f;
+#pragma unroll
+      for (int e = 0; e < BLK / 4; ++e) {
+        a = fmaf(m[e].x, kf[4 * e + 0], a);
+        a = fmaf(m[e].y, kf[4 * e + 1], a);
+        a = fmaf(m[e].z, kf[4 * e + 2], a);
+        a = fmaf(m[e].w, kf[4 * e + 3], a);
+      }
+      a += __shfl_xor_sync(0xffffffffu, a, 1);
+      a += __shfl_xor_sync(0xffffffffu, a, 2);
+      a += __shfl_xor_sync(0xffffffffu, a, 4);
+      if (part == 0) p.Kproj[row * R + j] = __float2bfloat16_rn(a);
+    }
   }
 }
 
 template <int D, int R>
 cudaError_t launch_dr(const ProjParams& p, cudaStream_t stream) {
   if (p.append) {
-    const int blocks = (p.B * p.Hkv + 7) / 8;
-    append_kernel<D, R><<<blocks, 256, 0, stream>>>(p);
+    append_kernel<D, R><<<p.B * p.Hkv, 256, 0, stream>>>(p);
     return cudaGetLastError();
   }
   const size_t smem = (size_t)R * D * 4;

@@ -23,8 +23,8 @@ struct ProjParams {
 };
 cudaError_t launch_proj(const ProjParams& p, cudaStream_t stream);
 
-// ---------------------------------------------------------------------------- selection
-struct SelectParams {
+// ---------------------------------------------------------------------------- score scan
+struct ScoreParams {
   const __nv_bfloat16* q;      // [B][Hq][d]
   const float* M;              // [Hkv][r][d]
   const __nv_bfloat16* kproj;  // cache layout, width r
@@ -32,18 +32,32 @@ struct SelectParams {
   const int32_t* seqlens;
   const int32_t* kvec;         // [B]
   const float* log_g;          // [B][Hkv][cap] or null
-  int32_t* idx_out;            // [B][Hkv][k_max]
+  uint32_t* keys;              // workspace: [B][Hkv][cap] order-preserving keys of u_i
+  uint32_t* hist;              // workspace: [B][Hkv][2048] counts of the keys' top 11 bits (zero on entry)
   float* scores_out;           // [B][Hkv][cap] or null
   uint32_t* err;
   int B, Hq, Hkv, G, d, r, cap, max_pages, num_pages, paged, k_max;
   float sigma, lam;
+  int rows_per_cta;
+};
+void plan_score(ScoreParams& p, int num_sms);
+cudaError_t launch_score(const ScoreParams& p, cudaStream_t stream);
+
+// ---------------------------------------------------------------------------- selection
+struct SelectParams {
+  const uint32_t* keys;        // workspace keys written by the score kernel
+  uint32_t* hist;              // workspace histograms (cleared here after use)
+  const int32_t* seqlens;
+  const int32_t* kvec;         // [B]
+  int32_t* idx_out;            // [B][Hkv][k_max]
+  uint32_t* err;
+  int B, Hkv, cap, k_max;
   int cluster;                 // CTAs per (b, h)
   int chunk;                   // max positions per CTA (multiple of 512)
-  int nstages;                 // bulk-copy ring depth
-  int stage_bytes;             // bytes per ring stage
-  int off_ring, off_q, off_bar, off_ctl, smem_bytes;
+  int cand_cap;                // candidate list capacity per CTA
+  int off_hist, off_ctl, smem_bytes;
 };
-// Chooses cluster size, chunk and ring depth for a shape; returns false if unsupported.
+// Chooses cluster size and chunk for a shape; returns false if unsupported.
 bool plan_select(SelectParams& p, int num_sms);
 cudaError_t launch_select(const SelectParams& p, cudaStream_t stream);
 

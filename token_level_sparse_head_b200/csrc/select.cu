@@ -1,26 +1,20 @@
-// Fused score scan + per-KV-head top-k selection (sm_100a).
+// Per-KV-head top-k selection over the score keys (sm_100a).
 //
-// One thread-block cluster per (sequence b, KV head h).  Each CTA of the cluster owns a
-// contiguous chunk of positions:
-//   1. q-bar = mean of the G query heads of h, q-hat = sigma * M[h] q-bar (JSSA page, section
-//      打分误差的定义: selection uses the group-mean query and s-hat = q-bar^T M^T M k).
-//   2. The chunk's projected-cache rows stream through a ring of shared-memory stages filled by
-//      bulk copies on the TMA engine (one copy per contiguous run: the whole stage for the
-//      contiguous layout, one per 64-token page for the paged one).  Each thread scores one
-//      row: u_i = q-hat . Kproj_i (+ lambda log g_i, SAS page section 2.1), with packed fp32
-//      FMAs, and stores the order-preserving uint32 key of u_i in shared memory.  Scoring scans
-//      every candidate (JSSA page, section Triton 内核的三个设计点: scoring is not sparse).
-//   3. Radix select of the k-th largest key over the whole cluster: up to three digit passes
-//      (11, 11, 10 bits).  Each CTA histograms its chunk in shared memory, adds the non-zero
-//      bins into rank 0's histogram through distributed shared memory, rank 0 finds the digit
-//      holding the k-th key and broadcasts it.  A pass that isolates exactly the remaining
-//      count ends the search early.
-//   4. Ordered compaction: positions with a larger key are selected, and of those with the
-//      threshold key the lowest positions fill the remainder (exact ties -> lower position).
-//      A cluster-wide exclusive count gives every position its output slot, so the index list
-//      comes out in ascending order with no sort.
-// Scores never leave the chip.  The per-KV-head top-k shared by the G query heads is the
-// selection rule of the JSSA page, section JSSA 的整体结构 / Figure 1.
+// JSSA page, section JSSA 的整体结构 / Figure 1: every KV head keeps the positions of its k
+// largest projected scores, and its G query heads share them; section 局限与需要留意的地方:
+// no sink or recent window is forced.  The score kernel has left each (b, h)'s order-preserving
+// uint32 keys in the workspace (on chip in L2) together with a histogram of their top 11 bits.
+//
+// One thread-block cluster per (b, h); each CTA copies a contiguous chunk of the keys into
+// shared memory.  The k-th largest key is found digit by digit (11, 11, 10 bits):
+//   digit 1 straight from the global histogram (every CTA computes the same answer);
+//   digits 2 and 3 from histograms of the surviving candidates only, which each CTA adds into
+//   rank 0's shared memory with fire-and-forget cluster reductions, one cluster barrier each.
+// A digit whose bin holds exactly the remaining count ends the search.  Then an ordered
+// compaction: positions with a larger key are selected, and of those equal to the threshold key
+// the lowest positions fill the remainder (exact ties -> lower position).  A cluster-wide
+// exclusive count gives every position its output slot, so the index list comes out ascending
+// with no sort.
 #include <cooperative_groups.h>
 
 #include "sas_device.cuh"
@@ -32,12 +26,11 @@ namespace sas {
 namespace {
 
 constexpr int kThreads = 256;
-constexpr int kStageRows = 256;  // one row per thread per stage
 constexpr int kBins = 2048;      // 11-bit digits
-constexpr int kMaxStages = 8;
+constexpr int kCand2 = 2048;     // survivors of the second digit kept on chip
 
 struct Ctl {
-  uint32_t prefix, mask, k_rem, eq;
+  uint32_t cnt1, cnt2, pad0, pad1;
   uint32_t cta_gt, cta_eq, gt_before, eq_before;
 };
 
@@ -73,250 +66,225 @@ __device__ __forceinline__ void hist_add(uint32_t* hist, uint32_t bin, bool acti
   if ((__ffs(peers) - 1) == lane) atomicAdd(&hist[bin], (uint32_t)__popc(peers));
 }
 
-template <int R>
+// Digit holding the k_rem-th largest key, from a histogram of `nb` bins (2048 or 1024) that may
+// live in another CTA's shared memory.  Every CTA of a cluster runs this on the same histogram
+// and gets the same answer.  Thread t covers digits [nb - (t+1)*per, nb - t*per).
+struct Found {
+  uint32_t digit, above, eq, pad;
+};
+
+template <int PER>
+__device__ __forceinline__ void find_digit(const uint32_t* H, uint32_t k_rem, uint32_t* wsum, Found* out) {
+  const int tid = threadIdx.x;
+  const int lo = PER * kThreads - (tid + 1) * PER;  // first digit of my range (nb = PER * 256)
+  uint32_t c[PER];
+  if constexpr (PER == 8) {
+    const uint4 a = *reinterpret_cast<const uint4*>(H + lo);
+    const uint4 b = *reinterpret_cast<const uint4*>(H + lo + 4);
+    c[0] = a.x; c[1] = a.y; c[2] = a.z; c[3] = a.w; c[4] = b.x; c[5] = b.y; c[6] = b.z; c[7] = b.w;
+  } else {
+    const uint4 a = *reinterpret_cast<const uint4*>(H + lo);
+    c[0] = a.x; c[1] = a.y; c[2] = a.z; c[3] = a.w;
+  }
+  uint32_t tsum = 0u;
+#pragma unroll
+  for (int j = 0; j < PER; ++j) tsum += c[j];
+  uint32_t tot;
+  const uint32_t above = block_excl_scan(tsum, wsum, &tot);
+  if (above < k_rem && k_rem <= above + tsum) {
+    uint32_t a = above;
+#pragma unroll
+    for (int j = PER - 1; j >= 0; --j) {
+      if (a + c[j] >= k_rem) {
+        out->digit = (uint32_t)(lo + j);
+        out->above = a;
+        out->eq = c[j];
+        break;
+      }
+      a += c[j];
+    }
+  }
+  __syncthreads();
+}
+
+// Appends `key` (where take is true) to list[] through a shared counter; warp-aggregated.
+__device__ __forceinline__ void list_append(uint32_t* list, uint32_t* counter, uint32_t cap, uint32_t key, bool take) {
+  const uint32_t m = __ballot_sync(0xffffffffu, take);
+  if (m == 0u) return;
+  const int lane = threadIdx.x & 31;
+  const int leader = __ffs(m) - 1;
+  uint32_t base = 0u;
+  if (lane == leader) base = atomicAdd(counter, (uint32_t)__popc(m));
+  base = __shfl_sync(0xffffffffu, base, leader);
+  if (take) {
+    const uint32_t pos = base + (uint32_t)__popc(m & ((1u << lane) - 1u));
+    if (pos < cap) list[pos] = key;
+  }
+}
+
+// Fire-and-forget add into the same shared-memory word of cluster CTA `rank`.
+__device__ __forceinline__ void red_add_cluster(const uint32_t* local, uint32_t rank, uint32_t v) {
+  uint32_t ra;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"(smem_u32(local)), "r"(rank));
+  asm volatile("red.relaxed.cluster.shared::cluster.add.u32 [%0], %1;" ::"r"(ra), "r"(v) : "memory");
+}
+
 __global__ void __launch_bounds__(kThreads) select_topk_kernel(const SelectParams p) {
   extern __shared__ __align__(128) unsigned char smem[];
   cg::cluster_group cluster = cg::this_cluster();
   const int rank = (int)cluster.block_rank();
   const int C = (int)cluster.num_blocks();
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int tid = threadIdx.x;
   const int bh = blockIdx.y;
-  const int b = bh / p.Hkv, h = bh % p.Hkv;
+  const int b = bh / p.Hkv;
 
   uint32_t* keys = reinterpret_cast<uint32_t*>(smem);
-  unsigned char* ring = smem + p.off_ring;
-  uint32_t* hist_local = reinterpret_cast<uint32_t*>(ring);
-  uint32_t* hist_global = hist_local + kBins;
-  float* qbar = reinterpret_cast<float*>(smem + p.off_q);
-  float* qhat = qbar + 128;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + p.off_bar);
+  uint32_t* hl = reinterpret_cast<uint32_t*>(smem + p.off_hist);  // this CTA's histogram
+  uint32_t* gh1 = hl + kBins;                                       // rank 0: cluster histogram, digit 2
+  uint32_t* gh2 = gh1 + kBins;                                      // rank 0: cluster histogram, digit 3
+  uint32_t* cand2 = gh2 + kBins / 2;
+  uint32_t* cand = cand2 + kCand2;
+  const uint32_t cap1 = (uint32_t)p.cand_cap;
   Ctl* ctl = reinterpret_cast<Ctl*>(smem + p.off_ctl);
-  uint32_t* wsum = reinterpret_cast<uint32_t*>(ctl + 1);
+  Found* found = reinterpret_cast<Found*>(ctl + 1);
+  uint32_t* wsum = reinterpret_cast<uint32_t*>(found + 1);
 
-  // ---- per-sequence values (checked on the device) ----
+  // per-sequence values (range errors were recorded by the score kernel)
   int n = p.seqlens[b];
-  if (n < 0 || n > p.cap) {
-    if (rank == 0 && tid == 0 && h == 0) record_error(p.err, kDevBadSeqlen, (uint32_t)b);
-    n = 0;
-  }
-  int kb = p.kvec[b];
-  if (kb > p.k_max) {
-    if (rank == 0 && tid == 0 && h == 0) record_error(p.err, kDevKOverMax, (uint32_t)b);
-    kb = p.k_max;
-  }
+  if (n < 0 || n > p.cap) n = 0;
+  const int kb = min(p.kvec[b], p.k_max);
   const int k_eff = max(0, min(kb, n));
   int32_t* idx = p.idx_out + (size_t)bh * p.k_max;
 
-  // Nothing to rank: empty selection, or every position selected (scores still computed when
-  // they are requested).  Uniform per cluster.
-  const bool want_scores = (p.scores_out != nullptr) && n > 0;
-  if (!want_scores && (k_eff == 0 || k_eff == n)) {
+  // Nothing to rank: empty selection, or every position selected.  Uniform per cluster.
+  if (k_eff == 0 || k_eff == n) {
     for (int j = rank * kThreads + tid; j < p.k_max; j += C * kThreads) idx[j] = (j < k_eff) ? j : -1;
     return;
   }
 
   // ---- this CTA's positions [c0, c1) ----
   const int chunk_b = ((n + C - 1) / C + 511) & ~511;  // multiple of 512 -> even run
-  const int run = chunk_b / kThreads;                  // positions per thread in the select
+  const int run = chunk_b / kThreads;                  // positions per thread
   const int c0 = min(rank * chunk_b, n);
   const int c1 = min(c0 + chunk_b, n);
   const int len = c1 - c0;
-
-  // ---- 1. q-bar and q-hat ----
-  for (int c = tid; c < p.d; c += kThreads) {
-    const __nv_bfloat16* qg = p.q + ((size_t)b * p.Hq + (size_t)h * p.G) * p.d + c;
-    float s = 0.f;
-    for (int g = 0; g < p.G; ++g) s += __bfloat162float(qg[(size_t)g * p.d]);
-    qbar[c] = s / (float)p.G;
-  }
-  if (tid == 0) {
-    for (int s = 0; s < p.nstages; ++s) mbar_init(&bars[s], 1);
-    fence_barrier_init();
-  }
-  __syncthreads();
-  for (int j = warp; j < R; j += kThreads / 32) {
-    const float* Mj = p.M + ((size_t)h * R + j) * p.d;
-    float s = 0.f;
-    for (int c = lane; c < p.d; c += 32) s = fmaf(Mj[c], qbar[c], s);
-#pragma unroll
-    for (int o = 16; o; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-    if (lane == 0) qhat[j] = s * p.sigma;
-  }
-  __syncthreads();
-
-  // Each thread reads its row's 16-byte chunks in a rotated order so that the 8 lanes of a
-  // shared-memory phase hit distinct banks; q-hat is held in the same rotated order, so the
-  // register index stays static.
-  constexpr int CPR = R / 8;                        // 16-byte chunks per row
-  constexpr int STAG = (64 / R) > 1 ? (64 / R) : 1; // lanes sharing a rotation
-  const int rot = (tid / STAG) % CPR;
-  float2 qr[CPR][4];
-#pragma unroll
-  for (int cc = 0; cc < CPR; ++cc) {
-    const int ch = (cc + rot) % CPR;
-#pragma unroll
-    for (int e = 0; e < 4; ++e) qr[cc][e] = make_float2(qhat[ch * 8 + 2 * e], qhat[ch * 8 + 2 * e + 1]);
-  }
-
-  // ---- 2. stream the chunk's projected rows ----
-  const bool gated = (p.log_g != nullptr);
-  const size_t lg_base = (size_t)bh * p.cap;
-  const int nst = (len + kStageRows - 1) / kStageRows;
-  const int kp_stage_bytes = kStageRows * R * 2;
-
-  auto issue = [&](int s) {
-    const int r0 = s * kStageRows;
-    const int nr = min(kStageRows, len - r0);
-    const int slot = s % p.nstages;
-    unsigned char* dst = ring + (size_t)slot * p.stage_bytes;
-    const int pos0 = c0 + r0;
-    uint32_t bytes = 0;
-    if (!p.paged) {
-      bytes += (uint32_t)nr * R * 2;
-    } else {
-      for (int t = 0; t < nr; t += 64) {
-        const int pg = p.page_table[(size_t)b * p.max_pages + (pos0 + t) / 64];
-        if (pg >= 0 && pg < p.num_pages) bytes += (uint32_t)min(64, nr - t) * R * 2;
-      }
-    }
-    if (gated) bytes += (uint32_t)((nr + 3) & ~3) * 4;
-    mbar_arrive_expect_tx(&bars[slot], bytes);
-    if (!p.paged) {
-      const __nv_bfloat16* src = p.kproj + ((size_t)bh * p.cap + pos0) * R;
-      bulk_g2s(dst, src, (uint32_t)nr * R * 2, &bars[slot]);
-    } else {
-      for (int t = 0; t < nr; t += 64) {
-        const int pos = pos0 + t;
-        const int pg = p.page_table[(size_t)b * p.max_pages + pos / 64];
-        if (pg >= 0 && pg < p.num_pages) {
-          const __nv_bfloat16* src = p.kproj + (((size_t)pg * p.Hkv + h) * 64 + (pos & 63)) * R;
-          bulk_g2s(dst + (size_t)t * R * 2, src, (uint32_t)min(64, nr - t) * R * 2, &bars[slot]);
-        } else {
-          record_error(p.err, kDevBadPage, (uint32_t)b);
-        }
-      }
-    }
-    if (gated) bulk_g2s(dst + kp_stage_bytes, p.log_g + lg_base + pos0, (uint32_t)((nr + 3) & ~3) * 4, &bars[slot]);
-  };
-
-  if (tid == 0)
-    for (int s = 0; s < min(nst, p.nstages); ++s) issue(s);
-
-  bool waited_ok = true;
-  for (int s = 0; s < nst; ++s) {
-    const int slot = s % p.nstages;
-    const uint32_t parity = (uint32_t)(s / p.nstages) & 1u;
-    if (!mbar_wait_bounded(&bars[slot], parity)) waited_ok = false;
-    const int row = s * kStageRows + tid;
-    if (row < len) {
-      const unsigned char* st = ring + (size_t)slot * p.stage_bytes;
-      const uint4* kr = reinterpret_cast<const uint4*>(st + (size_t)tid * (R * 2));
-      // Per-chunk partial sums, combined by a butterfly over the chunk index: the result is
-      // the same for every rotation, so identical rows give bit-identical scores (exact ties).
-      float pc[CPR];
-#pragma unroll
-      for (int cc = 0; cc < CPR; ++cc) {
-        const uint4 w = kr[(cc + rot) % CPR];
-        float2 a = ffma2(qr[cc][0], make_float2(bf16lo(w.x), bf16hi(w.x)), make_float2(0.f, 0.f));
-        a = ffma2(qr[cc][1], make_float2(bf16lo(w.y), bf16hi(w.y)), a);
-        a = ffma2(qr[cc][2], make_float2(bf16lo(w.z), bf16hi(w.z)), a);
-        a = ffma2(qr[cc][3], make_float2(bf16lo(w.w), bf16hi(w.w)), a);
-        pc[cc] = a.x + a.y;
-      }
-#pragma unroll
-      for (int half = CPR / 2; half >= 1; half >>= 1)
-#pragma unroll
-        for (int cc = 0; cc < half; ++cc) pc[cc] = pc[cc] + pc[cc + half];
-      float u = pc[0];
-      if (gated) {
-        const float lg = reinterpret_cast<const float*>(st + kp_stage_bytes)[tid];
-        u = fmaf(p.lam, lg, u);
-      }
-      keys[row + row / run] = float_key(u);
-      if (p.scores_out != nullptr) p.scores_out[lg_base + c0 + row] = u;
-    }
-    __syncthreads();
-    if (tid == 0 && s + p.nstages < nst) issue(s + p.nstages);
-  }
-  if (!waited_ok) record_error(p.err, kDevWaitTimeout, (uint32_t)bh);
-
-  if (k_eff == 0) {  // scores were requested, nothing is selected (uniform per cluster)
-    for (int j = rank * kThreads + tid; j < p.k_max; j += C * kThreads) idx[j] = -1;
-    return;
-  }
-
-  // ---- 3. radix select across the cluster ----
-  for (int i = tid; i < 2 * kBins; i += kThreads) hist_local[i] = 0u;
-  cluster.sync();  // all keys written; every CTA's histograms zeroed
-
-  uint32_t prefix = 0u, mask = 0u, k_rem = (uint32_t)k_eff;
   const int my0 = tid * run;
-  uint32_t* g0 = cluster.map_shared_rank(hist_global, 0);
-  for (int pass = 0; pass < 3; ++pass) {
-    const int shift = pass == 0 ? 21 : (pass == 1 ? 10 : 0);
-    const uint32_t dmask = pass == 2 ? 0x3ffu : 0x7ffu;
-    const int nb = (int)dmask + 1;
-    if (pass > 0) {
-      for (int i = tid; i < kBins; i += kThreads) hist_local[i] = 0u;
-      __syncthreads();
+
+  // ---- keys of the chunk into shared memory (padded: one spare word per run) ----
+  const uint32_t* gk = p.keys + (size_t)bh * p.cap + c0;
+  for (int v = tid; v * 4 < len; v += kThreads) {
+    const int li = v * 4;
+    if (li + 4 <= len) {
+      const uint4 w = *reinterpret_cast<const uint4*>(gk + li);
+      keys[li + li / run] = w.x;
+      keys[li + 1 + (li + 1) / run] = w.y;
+      keys[li + 2 + (li + 2) / run] = w.z;
+      keys[li + 3 + (li + 3) / run] = w.w;
+    } else {
+      for (int e = li; e < len; ++e) keys[e + e / run] = gk[e];
     }
+  }
+  for (int i = tid; i < kBins + kBins + kBins / 2; i += kThreads) hl[i] = 0u;  // hl, gh1, gh2
+  if (tid == 0) {
+    ctl->cnt1 = 0u;
+    ctl->cnt2 = 0u;
+  }
+
+  // ---- digit 1 from the global histogram (identical in every CTA of the cluster) ----
+  const uint32_t* ghist = p.hist + (size_t)bh * kBins;
+  uint32_t k_rem = (uint32_t)k_eff;
+  find_digit<8>(ghist, k_rem, wsum, found);  // ends with __syncthreads: keys, zeros visible
+  uint32_t prefix = found->digit << 21;
+  uint32_t mask = 0x7ffu << 21;
+  k_rem -= found->above;
+  bool done = (found->eq == k_rem);
+  // Every CTA has read the global histogram and zeroed its cluster histograms: after this
+  // barrier, rank 0 clears the global histogram for the next call and the adds can start.
+  cluster.sync();
+  if (rank == 0)
+    for (int i = tid; i < kBins; i += kThreads) const_cast<uint32_t*>(ghist)[i] = 0u;
+
+  bool ovf1 = false;
+  if (!done) {
+    // candidates: the keys in the threshold bin of digit 1
     for (int i = 0; i < run; ++i) {
       const int li = my0 + i;
-      uint32_t key = 0u;
-      bool act = false;
-      if (li < len) {
-        key = keys[li + tid];  // == keys[li + li / run]
-        act = (key & mask) == prefix;
-      }
-      hist_add(hist_local, (key >> shift) & dmask, act);
+      const uint32_t key = li < len ? keys[li + tid] : 0u;
+      list_append(cand, &ctl->cnt1, cap1, key, li < len && (key & mask) == prefix);
     }
     __syncthreads();
-    for (int i = tid; i < nb; i += kThreads) {
-      const uint32_t v = hist_local[i];
-      if (v) atomicAdd(&g0[i], v);
-    }
-    cluster.sync();
-    if (rank == 0) {
-      const int per = nb / kThreads;
-      const int hi = nb - tid * per;  // thread t covers digits [hi - per, hi), highest first
-      uint32_t tsum = 0u;
-      for (int j = 1; j <= per; ++j) tsum += hist_global[hi - j];
-      uint32_t tot;
-      const uint32_t above = block_excl_scan(tsum, wsum, &tot);
-      if (above < k_rem && k_rem <= above + tsum) {
-        uint32_t a = above;
-        for (int j = 1; j <= per; ++j) {
-          const uint32_t c = hist_global[hi - j];
-          if (a + c >= k_rem) {
-            const uint32_t digit = (uint32_t)(hi - j);
-            Ctl v;
-            v.prefix = prefix | (digit << shift);
-            v.mask = mask | (dmask << shift);
-            v.k_rem = k_rem - a;
-            v.eq = c;
-            for (int rr = 0; rr < C; ++rr) {
-              Ctl* dstc = cluster.map_shared_rank(ctl, rr);
-              dstc->prefix = v.prefix;
-              dstc->mask = v.mask;
-              dstc->k_rem = v.k_rem;
-              dstc->eq = v.eq;
-            }
-            break;
-          }
-          a += c;
-        }
+    const uint32_t n1 = ctl->cnt1;
+    ovf1 = n1 > cap1;
+    if (!ovf1) {
+      for (uint32_t e0 = 0; e0 < n1; e0 += kThreads) {
+        const uint32_t e = e0 + tid;
+        const uint32_t key = e < n1 ? cand[e] : 0u;
+        hist_add(hl, (key >> 10) & 0x7ffu, e < n1);
       }
-      __syncthreads();
-      for (int i = tid; i < nb; i += kThreads) hist_global[i] = 0u;
+    } else {
+      for (int i = 0; i < run; ++i) {
+        const int li = my0 + i;
+        const uint32_t key = li < len ? keys[li + tid] : 0u;
+        hist_add(hl, (key >> 10) & 0x7ffu, li < len && (key & mask) == prefix);
+      }
+    }
+    __syncthreads();
+    for (int i = tid; i < kBins; i += kThreads) {
+      const uint32_t v = hl[i];
+      if (v) red_add_cluster(gh1 + i, 0, v);
     }
     cluster.sync();
-    prefix = ctl->prefix;
-    mask = ctl->mask;
-    k_rem = ctl->k_rem;
-    if (ctl->eq == k_rem) break;  // the threshold digit holds exactly the remainder
+    find_digit<8>(cluster.map_shared_rank(gh1, 0), k_rem, wsum, found);
+    prefix |= found->digit << 10;
+    mask |= 0x7ffu << 10;
+    k_rem -= found->above;
+    done = (found->eq == k_rem);
+  }
+  if (!done) {
+    // survivors of digit 2
+    for (int i = tid; i < kBins / 2; i += kThreads) hl[i] = 0u;
+    if (!ovf1) {
+      const uint32_t n1 = ctl->cnt1;
+      for (uint32_t e0 = 0; e0 < n1; e0 += kThreads) {
+        const uint32_t e = e0 + tid;
+        const uint32_t key = e < n1 ? cand[e] : 0u;
+        list_append(cand2, &ctl->cnt2, kCand2, key, e < n1 && (key & mask) == prefix);
+      }
+    } else {
+      for (int i = 0; i < run; ++i) {
+        const int li = my0 + i;
+        const uint32_t key = li < len ? keys[li + tid] : 0u;
+        list_append(cand2, &ctl->cnt2, kCand2, key, li < len && (key & mask) == prefix);
+      }
+    }
+    __syncthreads();
+    const uint32_t n2 = ctl->cnt2;
+    if (n2 <= kCand2) {
+      for (uint32_t e0 = 0; e0 < n2; e0 += kThreads) {
+        const uint32_t e = e0 + tid;
+        const uint32_t key = e < n2 ? cand2[e] : 0u;
+        hist_add(hl, key & 0x3ffu, e < n2);
+      }
+    } else {
+      for (int i = 0; i < run; ++i) {
+        const int li = my0 + i;
+        const uint32_t key = li < len ? keys[li + tid] : 0u;
+        hist_add(hl, key & 0x3ffu, li < len && (key & mask) == prefix);
+      }
+    }
+    __syncthreads();
+    for (int i = tid; i < kBins / 2; i += kThreads) {
+      const uint32_t v = hl[i];
+      if (v) red_add_cluster(gh2 + i, 0, v);
+    }
+    cluster.sync();
+    find_digit<4>(cluster.map_shared_rank(gh2, 0), k_rem, wsum, found);
+    prefix |= found->digit;
+    mask = 0xffffffffu;
+    k_rem -= found->above;
   }
 
-  // ---- 4. ordered compaction ----
+  // ---- ordered compaction ----
   const uint32_t need = k_rem;  // how many of the threshold-key positions to take
   uint32_t n_gt = 0u, n_eq = 0u;
   for (int i = 0; i < run; ++i) {
@@ -334,15 +302,22 @@ __global__ void __launch_bounds__(kThreads) select_topk_kernel(const SelectParam
     ctl->cta_eq = tot & 0xffffu;
   }
   cluster.sync();
-  if (tid == 0) {
+  if (tid < 32) {
     uint32_t gb = 0u, eb = 0u;
-    for (int rr = 0; rr < rank; ++rr) {
-      const Ctl* rc = cluster.map_shared_rank(ctl, rr);
-      gb += rc->cta_gt;
-      eb += rc->cta_eq;
+    if (tid < rank) {
+      const Ctl* rc = cluster.map_shared_rank(ctl, tid);
+      gb = rc->cta_gt;
+      eb = rc->cta_eq;
     }
-    ctl->gt_before = gb;
-    ctl->eq_before = eb;
+#pragma unroll
+    for (int o = 16; o; o >>= 1) {
+      gb += __shfl_xor_sync(0xffffffffu, gb, o);
+      eb += __shfl_xor_sync(0xffffffffu, eb, o);
+    }
+    if (tid == 0) {
+      ctl->gt_before = gb;
+      ctl->eq_before = eb;
+    }
   }
   __syncthreads();
   uint32_t gt_c = ctl->gt_before + (excl >> 16);
@@ -362,12 +337,11 @@ __global__ void __launch_bounds__(kThreads) select_topk_kernel(const SelectParam
     }
   }
   for (int j = k_eff + rank * kThreads + tid; j < p.k_max; j += C * kThreads) idx[j] = -1;
-  cluster.sync();  // peers may still read this CTA's control block
+  cluster.sync();  // peers may still read this CTA's shared memory
 }
 
-template <int R>
-cudaError_t launch_r(const SelectParams& p, cudaStream_t stream) {
-  auto kern = select_topk_kernel<R>;
+cudaError_t launch_sel(const SelectParams& p, cudaStream_t stream) {
+  auto kern = select_topk_kernel;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, p.smem_bytes);
   if (e != cudaSuccess) return e;
   if (p.cluster > 8) {
@@ -392,7 +366,6 @@ cudaError_t launch_r(const SelectParams& p, cudaStream_t stream) {
 }  // namespace
 
 bool plan_select(SelectParams& p, int num_sms) {
-  if (p.r != 16 && p.r != 32 && p.r != 64) return false;
   const int cap = p.cap;
   const int heads = p.B * p.Hkv;
   int C = 1;
@@ -403,31 +376,15 @@ bool plan_select(SelectParams& p, int num_sms) {
   if (chunk > kMaxChunk) return false;
   p.cluster = C;
   p.chunk = chunk;
-  p.stage_bytes = kStageRows * p.r * 2 + kStageRows * 4;
+  p.cand_cap = chunk / 4 > 1024 ? chunk / 4 : 1024;
   const int keys_bytes = ((chunk + kThreads) * 4 + 127) & ~127;
-  // Ring depth: deeper when few CTAs share an SM.
-  const long ctas = (long)heads * C;
-  int ns = ctas <= num_sms ? 6 : (ctas <= 2L * num_sms ? 4 : 2);
-  if (ns > kMaxStages) ns = kMaxStages;
-  p.nstages = ns;
-  int ring = ns * p.stage_bytes;
-  if (ring < 2 * kBins * 4) ring = 2 * kBins * 4;
-  ring = (ring + 127) & ~127;
-  p.off_ring = keys_bytes;
-  p.off_q = p.off_ring + ring;
-  p.off_bar = p.off_q + (128 + 64) * 4;
-  p.off_ctl = p.off_bar + kMaxStages * 8;
-  p.smem_bytes = p.off_ctl + (int)sizeof(Ctl) + (kThreads / 32) * 4;
+  p.off_hist = keys_bytes;
+  const int hist_bytes = (kBins + kBins + kBins / 2 + kCand2 + p.cand_cap) * 4;
+  p.off_ctl = p.off_hist + ((hist_bytes + 15) & ~15);
+  p.smem_bytes = p.off_ctl + (int)sizeof(Ctl) + (int)sizeof(Found) + (kThreads / 32) * 4;
   return p.smem_bytes <= 227 * 1024;
 }
 
-cudaError_t launch_select(const SelectParams& p, cudaStream_t stream) {
-  switch (p.r) {
-    case 16: return launch_r<16>(p, stream);
-    case 32: return launch_r<32>(p, stream);
-    case 64: return launch_r<64>(p, stream);
-    default: return cudaErrorInvalidValue;
-  }
-}
+cudaError_t launch_select(const SelectParams& p, cudaStream_t stream) { return launch_sel(p, stream); }
 
 }  // namespace sas
