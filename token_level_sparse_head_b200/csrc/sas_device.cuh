@@ -43,6 +43,21 @@ __device__ __forceinline__ uint32_t float_key(float f) {
 
 __device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
 
+// Size of the selection, min(k_b, N_b) clamped at 0, and whether it needs ranking (neither
+// empty nor every position).  The ranking test is written on the inputs rather than as
+// (k_eff == 0 || k_eff == n): with nvcc 12.9 for sm_100a, an equality test between
+// max(0, min(k, n)) and n was observed to evaluate true for k = 64, n = 512.
+struct SeqSelection {
+  int k_eff;
+  bool ranked;
+};
+__device__ __forceinline__ SeqSelection seq_selection(int kb, int n) {
+  SeqSelection s;
+  s.k_eff = max(0, min(kb, n));
+  s.ranked = (kb > 0) && (n > 0) && (kb < n);
+  return s;
+}
+
 // ----------------------------------------------------------------------------- PTX
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));

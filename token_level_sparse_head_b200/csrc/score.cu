@@ -75,11 +75,10 @@ __global__ void __launch_bounds__(kThreads) score_kernel(const ScoreParams p) {
     if (blockIdx.x == 0 && tid == 0 && h == 0) record_error(p.err, kDevKOverMax, (uint32_t)b);
     kb = p.k_max;
   }
-  const int k_eff = max(0, min(kb, n));
   // Nothing to rank (empty selection or every position selected): no scores are needed,
   // unless the caller asked for them.  The CTA-uniform exits are expressed as one guard
   // around the body rather than early returns.
-  const bool need_hist = !(k_eff == 0 || k_eff == n);  // the selection ranks this (b, h)
+  const bool need_hist = seq_selection(kb, n).ranked;  // the selection ranks this (b, h)
   const int r0 = blockIdx.x * p.rows_per_cta;
   const int r1 = min(r0 + p.rows_per_cta, n);
   const bool skip = (!need_hist && p.scores_out == nullptr) || r0 >= r1;
