@@ -48,7 +48,8 @@ def roofline_bytes(B, Hq, Hkv, d, r, seqlens, ks, lam):
     lg = sum(int(n) * 4 for n in seqlens) * Hkv if lam != 0.0 else 0
     lg_sel = sum(min(int(k), int(n)) * 4 for n, k in zip(seqlens, ks)) * Hkv if lam != 0.0 else 0
     return {
-        "select": kproj + q + lg,
+        "score": kproj + q + lg,
+        "select": 0,
         "attend": kv + q + out + lg_sel,
         "step": kproj + kv + q + out + lg,
         "kproj": kproj, "kv": kv,
@@ -190,12 +191,14 @@ class Workload:
         ev[0].record()
         L.sas_append_proj(self.shape, self.knew, p.M, self.kproj, p.page_table, p.seqlens)
         ev[1].record()
-        L.sas_select_topk(self.shape, p.q, p.M, self.kproj, p.page_table, p.seqlens, p.k, p.k_max, p.lam,
-                          p.log_g, s.idx, None, s.workspace, s.ws_bytes)
+        L.sas_score_scan(self.shape, p.q, p.M, self.kproj, p.page_table, p.seqlens, p.k, p.k_max, p.lam, p.log_g,
+                         None, s.workspace, s.ws_bytes)
         ev[2].record()
+        L.sas_select_from_scores(self.shape, p.seqlens, p.k, p.k_max, s.idx, s.workspace, s.ws_bytes)
+        ev[3].record()
         L.sas_sparse_attention(self.shape, p.q, p.K, p.V, p.page_table, p.seqlens, s.idx, p.k, p.k_max, p.lam,
                                p.log_g, s.out, s.workspace, s.ws_bytes)
-        ev[3].record()
+        ev[4].record()
 
     def dense(self):
         p = self.p
@@ -277,22 +280,19 @@ def run_ours(args):
 
     # --- per-kernel durations (component entry points, events between the kernels)
     nk = max(3, min(args.steps, 200))
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(nk)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(nk)]
     torch.cuda.synchronize()
     for i in range(nk):
         wl.step_parts(evs[i])
     torch.cuda.synchronize()
-    k_ms = {
-        "append": statistics.mean(e[0].elapsed_time(e[1]) for e in evs),
-        "select": statistics.mean(e[1].elapsed_time(e[2]) for e in evs),
-        "attend": statistics.mean(e[2].elapsed_time(e[3]) for e in evs),
-    }
-    dom = "select" if k_ms["select"] >= k_ms["attend"] else "attend"
+    names = ("append", "score", "select", "attend")
+    k_ms = {nm: statistics.mean(e[i].elapsed_time(e[i + 1]) for e in evs) for i, nm in enumerate(names)}
+    dom = max(("score", "attend"), key=lambda nm: k_ms[nm])  # the kernels with algorithmic HBM bytes
     dom_bytes = wl.bytes[dom]
     head_bytes = dict(wl.bytes)
     head_dense_bytes = wl.dense_bytes
     achieved = dom_bytes / (k_ms[dom] * 1e-3) / 1e9
-    traffic = recorded_traffic("select.cu" if dom == "select" else "attend.cu", args.workload)
+    traffic = recorded_traffic({"score": "score.cu", "select": "select.cu", "attend": "attend.cu"}[dom], args.workload)
 
     # --- dense full-KV baseline on the same workload
     for _ in range(2):
@@ -334,13 +334,13 @@ def run_ours(args):
             w1.step()
         t1 = flushed_steps(torch, w1.step, max(10, min(args.steps, 100)), flush)
         td1 = flushed_steps(torch, w1.dense, 10, flush)
-        kt = {"append": [], "select": [], "attend": []}
+        kt = {"append": [], "score": [], "select": [], "attend": []}
         for _ in range(20):
             flush.zero_()
-            ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+            ev = [torch.cuda.Event(enable_timing=True) for _ in range(5)]
             w1.step_parts(ev)
             torch.cuda.synchronize()
-            for i, kname in enumerate(("append", "select", "attend")):
+            for i, kname in enumerate(("append", "score", "select", "attend")):
                 kt[kname].append(ev[i].elapsed_time(ev[i + 1]))
         secondary = {"workload": SECONDARY_WORKLOAD, "ms_per_step": t1 * 1e3, "steps_per_s": 1.0 / t1,
                      "hbm_gbs": w1.bytes["step"] / t1 / 1e9, "dense_ms_per_step": td1 * 1e3,

@@ -165,6 +165,21 @@ sas_status sas_select_topk(const sas_shape* shape, const void* q, const float* M
                            int32_t k_max, float lambda, const float* log_g, int32_t* idx_out,
                            float* scores_out, void* workspace, size_t ws_bytes, void* stream);
 
+/* The two halves of sas_select_topk, for composing or timing them separately; they share
+ * the workspace (the scan leaves per-position keys and per-(b, h) histograms in it, the
+ * selection consumes and clears the histograms).  Run them in this order on one stream.
+ *   sas_score_scan: every cached token of every (b, h) is scored on the projected cache
+ *     (JSSA page, section Triton 内核的三个设计点: scoring scans every candidate);
+ *     arguments as sas_select_topk.
+ *   sas_select_from_scores: the per-KV-head top-k of the scanned keys into idx_out. */
+sas_status sas_score_scan(const sas_shape* shape, const void* q, const float* M, const void* Kproj,
+                          const int32_t* page_table, const int32_t* seqlens, const int32_t* k,
+                          int32_t k_max, float lambda, const float* log_g, float* scores_out,
+                          void* workspace, size_t ws_bytes, void* stream);
+sas_status sas_select_from_scores(const sas_shape* shape, const int32_t* seqlens, const int32_t* k,
+                                  int32_t k_max, int32_t* idx_out, void* workspace, size_t ws_bytes,
+                                  void* stream);
+
 /* The attention half of sas_decode_step alone: softmax attention of every query head over
  * the first min(k_b, N_b) entries of its KV head's index list idx [B][Hkv][k_max] (any order,
  * entries in [0, N_b)), reading K/V rows in place. */

@@ -124,6 +124,11 @@ def run_small(p_cpu, device="cuda", dense=True, check_build=True):
     scores = torch.full((p.B, p.Hkv, p.cap), float("nan"), dtype=torch.float32, device=device)
     idx_sel = torch.full((p.B, p.Hkv, p.k_max), -7, dtype=torch.int32, device=device)
     sess.select(p.q, p.M, kp_in, p.page_table, p.seqlens, p.k, p.lam, p.log_g, idx=idx_sel, scores=scores)
+    # the two halves of the selection, called separately, give the same index lists
+    idx_split = torch.full((p.B, p.Hkv, p.k_max), -7, dtype=torch.int32, device=device)
+    lib.sas_score_scan(shape, p.q, p.M, kp_in, p.page_table, p.seqlens, p.k, p.k_max, p.lam, p.log_g, None,
+                       sess.workspace, sess.ws_bytes)
+    lib.sas_select_from_scores(shape, p.seqlens, p.k, p.k_max, idx_split, sess.workspace, sess.ws_bytes)
     out = torch.full((p.B, p.Hq, p.d), float("nan"), dtype=torch.float32, device=device)
     idx = torch.full((p.B, p.Hkv, p.k_max), -7, dtype=torch.int32, device=device)
     sess.decode(p.q, p.M, kp_in, p.K, p.V, p.page_table, p.seqlens, p.k, p.lam, p.log_g, out=out, idx=idx)
@@ -131,6 +136,7 @@ def run_small(p_cpu, device="cuda", dense=True, check_build=True):
     st, code, where = sess.check()
     assert code == 0, f"device check error {code} at {where}"
     assert torch.equal(idx, idx_sel), "decode_step and select_topk index lists differ"
+    assert torch.equal(idx, idx_split), "score_scan + select_from_scores differ from decode_step"
     sc, ix, ot = f64(scores), f64(idx), f64(out)
     G = p.Hq // p.Hkv
     ndiff = 0

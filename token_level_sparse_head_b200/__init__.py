@@ -12,6 +12,8 @@ from .lib import (  # noqa: F401
     sas_decode_workspace_bytes,
     sas_dense_decode,
     sas_dense_workspace_bytes,
+    sas_score_scan,
+    sas_select_from_scores,
     sas_select_topk,
     sas_sparse_attention,
     sas_workspace_init,

@@ -117,16 +117,22 @@ sas_status check_cache_ptrs(const sas_shape* s, const int32_t* page_table, const
   return SAS_OK;
 }
 
-sas_status do_select(const sas_shape* s, const void* q, const float* M, const void* Kproj,
-                     const int32_t* page_table, const int32_t* seqlens, const int32_t* k, int32_t k_max,
-                     float lambda, const float* log_g, int32_t* idx_out, float* scores_out, void* ws,
-                     cudaStream_t st) {
+struct SelectPlan {
+  sas::ScoreParams sp;
+  sas::SelectParams sl;
+};
+
+sas_status plan_selection(const sas_shape* s, const void* q, const float* M, const void* Kproj,
+                          const int32_t* page_table, const int32_t* seqlens, const int32_t* k, int32_t k_max,
+                          float lambda, const float* log_g, int32_t* idx_out, float* scores_out, void* ws,
+                          SelectPlan* out) {
   const sas::AttendParams a = attend_plan(s, k_max);
   const WsLayout L = ws_layout(a, true);
   unsigned char* w = static_cast<unsigned char*>(ws);
   const int sms = num_sms();
 
-  sas::ScoreParams sp = {};
+  sas::ScoreParams& sp = out->sp;
+  sp = {};
   sp.q = static_cast<const __nv_bfloat16*>(q);
   sp.M = M;
   sp.kproj = static_cast<const __nv_bfloat16*>(Kproj);
@@ -146,7 +152,8 @@ sas_status do_select(const sas_shape* s, const void* q, const float* M, const vo
   sp.lam = lambda;
   sas::plan_score(sp, sms);
 
-  sas::SelectParams sl = {};
+  sas::SelectParams& sl = out->sl;
+  sl = {};
   sl.keys = sp.keys;
   sl.hist = sp.hist;
   sl.seqlens = seqlens;
@@ -155,12 +162,27 @@ sas_status do_select(const sas_shape* s, const void* q, const float* M, const vo
   sl.err = sp.err;
   sl.B = s->B; sl.Hkv = s->Hkv; sl.cap = sp.cap; sl.k_max = k_max;
   if (!sas::plan_select(sl, sms)) return fail(SAS_ERR_UNSUPPORTED, "no selection plan for this shape");
-
-  cudaError_t e = sas::launch_score(sp, st);
-  if (e != cudaSuccess) return cuda_fail(e, "score kernel launch");
-  e = sas::launch_select(sl, st);
-  if (e != cudaSuccess) return cuda_fail(e, "select kernel launch");
   return SAS_OK;
+}
+
+sas_status run_score(const SelectPlan& pl, cudaStream_t st) {
+  const cudaError_t e = sas::launch_score(pl.sp, st);
+  return e == cudaSuccess ? SAS_OK : cuda_fail(e, "score kernel launch");
+}
+
+sas_status run_select(const SelectPlan& pl, cudaStream_t st) {
+  const cudaError_t e = sas::launch_select(pl.sl, st);
+  return e == cudaSuccess ? SAS_OK : cuda_fail(e, "select kernel launch");
+}
+
+sas_status do_select(const sas_shape* s, const void* q, const float* M, const void* Kproj,
+                     const int32_t* page_table, const int32_t* seqlens, const int32_t* k, int32_t k_max,
+                     float lambda, const float* log_g, int32_t* idx_out, float* scores_out, void* ws,
+                     cudaStream_t st) {
+  SelectPlan pl;
+  SAS_TRY(plan_selection(s, q, M, Kproj, page_table, seqlens, k, k_max, lambda, log_g, idx_out, scores_out, ws, &pl));
+  SAS_TRY(run_score(pl, st));
+  return run_select(pl, st);
 }
 
 sas_status do_attend(const sas_shape* s, const void* q, const void* K, const void* V, const int32_t* page_table,
@@ -297,6 +319,42 @@ sas_status sas_select_topk(const sas_shape* shape, const void* q, const float* M
   if (ws_bytes < sas_decode_workspace_bytes(shape, k_max)) return fail(SAS_ERR_INVALID_ARG, "workspace too small");
   return do_select(shape, q, M, Kproj, page_table, seqlens, k, k_max, lambda, log_g, idx_out, scores_out,
                    workspace, static_cast<cudaStream_t>(stream));
+}
+
+sas_status sas_score_scan(const sas_shape* shape, const void* q, const float* M, const void* Kproj,
+                          const int32_t* page_table, const int32_t* seqlens, const int32_t* k, int32_t k_max,
+                          float lambda, const float* log_g, float* scores_out, void* workspace, size_t ws_bytes,
+                          void* stream) {
+  SAS_TRY(check_shape(shape));
+  if (k_max < 1) return fail(SAS_ERR_INVALID_ARG, "k_max must be >= 1");
+  SAS_TRY(check_ptr(q, "q"));
+  SAS_TRY(check_ptr(M, "M"));
+  SAS_TRY(check_ptr(Kproj, "Kproj"));
+  SAS_TRY(check_ptr(k, "k"));
+  SAS_TRY(check_ptr(scores_out, "scores_out", false));
+  SAS_TRY(check_cache_ptrs(shape, page_table, seqlens));
+  if (lambda != 0.0f) SAS_TRY(check_ptr(log_g, "log_g"));
+  SAS_TRY(check_ptr(workspace, "workspace"));
+  if (ws_bytes < sas_decode_workspace_bytes(shape, k_max)) return fail(SAS_ERR_INVALID_ARG, "workspace too small");
+  SelectPlan pl;
+  SAS_TRY(plan_selection(shape, q, M, Kproj, page_table, seqlens, k, k_max, lambda, log_g, nullptr, scores_out,
+                         workspace, &pl));
+  return run_score(pl, static_cast<cudaStream_t>(stream));
+}
+
+sas_status sas_select_from_scores(const sas_shape* shape, const int32_t* seqlens, const int32_t* k, int32_t k_max,
+                                  int32_t* idx_out, void* workspace, size_t ws_bytes, void* stream) {
+  SAS_TRY(check_shape(shape));
+  if (k_max < 1) return fail(SAS_ERR_INVALID_ARG, "k_max must be >= 1");
+  SAS_TRY(check_ptr(seqlens, "seqlens"));
+  SAS_TRY(check_ptr(k, "k"));
+  SAS_TRY(check_ptr(idx_out, "idx_out"));
+  SAS_TRY(check_ptr(workspace, "workspace"));
+  if (ws_bytes < sas_decode_workspace_bytes(shape, k_max)) return fail(SAS_ERR_INVALID_ARG, "workspace too small");
+  SelectPlan pl;
+  SAS_TRY(plan_selection(shape, nullptr, nullptr, nullptr, nullptr, seqlens, k, k_max, 0.0f, nullptr, idx_out,
+                         nullptr, workspace, &pl));
+  return run_select(pl, static_cast<cudaStream_t>(stream));
 }
 
 sas_status sas_sparse_attention(const sas_shape* shape, const void* q, const void* K, const void* V,

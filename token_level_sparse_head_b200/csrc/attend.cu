@@ -24,7 +24,7 @@ namespace {
 constexpr int kWarps = 4;
 constexpr int kThreads = kWarps * 32;
 constexpr int kTile = 8;     // tokens per warp tile
-constexpr int kStages = 4;   // ring depth per warp
+constexpr int kStages = 3;   // ring depth per warp
 
 template <int D, int GT>
 struct Geo {
@@ -54,10 +54,14 @@ __host__ __device__ inline Smem smem_layout(int split_len, int splits) {
   s.off_rows = o;  o += split_len * 4;
   s.off_lg = o;    o += split_len * 4;
   o = (o + 127) & ~127;
-  s.off_ring = o;  o += kWarps * kStages * Gm::STAGE_BYTES;
+  s.off_ring = o;
+  // After the tile loop the ring is idle: the warp merge (and the split merge) reuse it.
+  const int ring = kWarps * kStages * Gm::STAGE_BYTES;
+  const int merge = kWarps * GT * (D + 2) * 4;
+  s.off_merge = o;
+  o += ring > merge ? ring : merge;
   s.off_pbuf = o;  o += kWarps * kTile * GT * 4;
   s.off_sbuf = o;  o += kWarps * GT * 4;
-  s.off_merge = o; o += kWarps * GT * (D + 2) * 4;
   o = (o + 7) & ~7;
   s.off_bars = o;  o += kWarps * kStages * 8;
   s.off_w = o;     o += splits * GT * 4 + GT * 8;
@@ -336,6 +340,9 @@ __global__ void __launch_bounds__(kThreads) attend_kernel(const AttendParams p) 
     const bool head_bit = (m >= (1 << Gm::SHIFT)) && (m < (1 << (Gm::SHIFT + Gm::LOG_GT)));
     if (!head_bit) l_tot += __shfl_xor_sync(0xffffffffu, l_tot, m);
   }
+  // The merge buffer aliases the ring: every warp must be done with its stages (all issued
+  // copies have been waited for) before any warp writes its totals.
+  __syncthreads();
   // merge[warp][g][0..D-1] = acc, [D] = m, [D+1] = l
   float* mw = merge + (size_t)warp * GT * (D + 2);
 #pragma unroll

@@ -30,7 +30,7 @@ namespace {
 constexpr int kThreads = 512;
 constexpr int kWarps = kThreads / 32;
 constexpr int kBins = 2048;          // 11-bit digits
-constexpr int kPerThread = 8;        // keys per thread per tile (two 16-byte loads)
+constexpr int kPerThread = 16;       // keys per thread per tile (four 16-byte loads)
 constexpr int kTile = kThreads * kPerThread;
 constexpr int kCandCap = 8192;       // candidate keys kept on chip per CTA
 constexpr int kCand2Cap = 2048;      // survivors of the second digit
@@ -152,20 +152,23 @@ __device__ __forceinline__ void red_add_cluster(const uint32_t* local, uint32_t 
   asm volatile("red.relaxed.cluster.shared::cluster.add.u32 [%0], %1;" ::"r"(ra), "r"(v) : "memory");
 }
 
-// Keys [t*kTile + tid*8, +8) of the chunk; positions past len read as 0 (and are masked).
+// Keys [t*kTile + tid*kPerThread, +kPerThread) of the chunk; positions past len read as 0 (and
+// are masked by the callers).
 __device__ __forceinline__ void load_tile(const uint32_t* gk, int len, int t, uint32_t (&k)[kPerThread]) {
   const int li = t * kTile + (int)threadIdx.x * kPerThread;
   if (li + kPerThread <= len) {
-    const uint4 a = __ldcg(reinterpret_cast<const uint4*>(gk + li));
-    const uint4 b = __ldcg(reinterpret_cast<const uint4*>(gk + li + 4));
-    k[0] = a.x; k[1] = a.y; k[2] = a.z; k[3] = a.w; k[4] = b.x; k[5] = b.y; k[6] = b.z; k[7] = b.w;
+#pragma unroll
+    for (int v = 0; v < kPerThread / 4; ++v) {
+      const uint4 a = __ldcg(reinterpret_cast<const uint4*>(gk + li + 4 * v));
+      k[4 * v + 0] = a.x; k[4 * v + 1] = a.y; k[4 * v + 2] = a.z; k[4 * v + 3] = a.w;
+    }
   } else {
 #pragma unroll
     for (int e = 0; e < kPerThread; ++e) k[e] = (li + e < len) ? __ldcg(gk + li + e) : 0u;
   }
 }
 
-__global__ void __launch_bounds__(kThreads) select_topk_kernel(const SelectParams p) {
+__global__ void __launch_bounds__(kThreads, 2) select_topk_kernel(const SelectParams p) {
   extern __shared__ __align__(128) unsigned char smem_raw[];
   SelSmem& S = *reinterpret_cast<SelSmem*>(smem_raw);
   cg::cluster_group cluster = cg::this_cluster();
@@ -186,7 +189,7 @@ __global__ void __launch_bounds__(kThreads) select_topk_kernel(const SelectParam
   const bool trivial = !sel.ranked;
 
   // this CTA's positions [c0, c1): chunks of whole 16-byte groups
-  const int chunk_b = (((n + C - 1) / C) + 7) & ~7;
+  const int chunk_b = (((n + C - 1) / C) + 15) & ~15;
   const int c0 = min(rank * chunk_b, n);
   const int c1 = min(c0 + chunk_b, n);
   const int len = c1 - c0;
@@ -443,11 +446,12 @@ __global__ void __launch_bounds__(kThreads) select_topk_kernel(const SelectParam
 
 bool plan_select(SelectParams& p, int num_sms) {
   const int heads = p.B * p.Hkv;
-  // About one wave (two 512-thread CTAs per SM); never chunks below one tile.
+  // Double the CTAs per head while the grid still fits one wave of two CTAs per SM and each
+  // CTA keeps at least one tile of keys.
   int C = 1;
   while (C < kMaxCluster && (long)heads * C * 2 <= 2L * num_sms && (p.cap + 2 * C - 1) / (2 * C) >= kTile) C *= 2;
   p.cluster = C;
-  p.chunk = (((p.cap + C - 1) / C) + 7) & ~7;
+  p.chunk = (((p.cap + C - 1) / C) + 15) & ~15;
   p.cand_cap = kCandCap;
   p.off_hist = 0;
   p.off_ctl = 0;

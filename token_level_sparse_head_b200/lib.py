@@ -43,6 +43,9 @@ _SIGS = {
                                        _vp, _i32, _f32, _vp, _vp, _vp, _vp, _sz, _vp]),
     "sas_select_topk": (ctypes.c_int, [ctypes.POINTER(sas_shape), _vp, _vp, _vp, _vp, _vp, _vp, _i32,
                                        _f32, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "sas_score_scan": (ctypes.c_int, [ctypes.POINTER(sas_shape), _vp, _vp, _vp, _vp, _vp, _vp, _i32, _f32,
+                                      _vp, _vp, _vp, _sz, _vp]),
+    "sas_select_from_scores": (ctypes.c_int, [ctypes.POINTER(sas_shape), _vp, _vp, _i32, _vp, _vp, _sz, _vp]),
     "sas_sparse_attention": (ctypes.c_int, [ctypes.POINTER(sas_shape), _vp, _vp, _vp, _vp, _vp, _vp,
                                             _vp, _i32, _f32, _vp, _vp, _vp, _sz, _vp]),
     "sas_dense_decode": (ctypes.c_int, [ctypes.POINTER(sas_shape), _vp, _vp, _vp, _vp, _vp, _vp, _vp,
@@ -184,6 +187,19 @@ def sas_select_topk(shape: Shape, q, M, Kproj, page_table, seqlens, k, k_max: in
                                   _p(seqlens), _p(k), int(k_max), float(lam), _p(log_g), _p(idx_out),
                                   _p(scores_out), _p(workspace), int(ws_bytes), _stream(stream)),
            "sas_select_topk")
+
+
+def sas_score_scan(shape: Shape, q, M, Kproj, page_table, seqlens, k, k_max: int, lam: float, log_g,
+                   scores_out, workspace, ws_bytes: int, stream=None):
+    _check(load().sas_score_scan(ctypes.byref(shape.c()), _p(q), _p(M), _p(Kproj), _p(page_table), _p(seqlens),
+                                 _p(k), int(k_max), float(lam), _p(log_g), _p(scores_out), _p(workspace),
+                                 int(ws_bytes), _stream(stream)), "sas_score_scan")
+
+
+def sas_select_from_scores(shape: Shape, seqlens, k, k_max: int, idx_out, workspace, ws_bytes: int,
+                           stream=None):
+    _check(load().sas_select_from_scores(ctypes.byref(shape.c()), _p(seqlens), _p(k), int(k_max), _p(idx_out),
+                                         _p(workspace), int(ws_bytes), _stream(stream)), "sas_select_from_scores")
 
 
 def sas_sparse_attention(shape: Shape, q, K, V, page_table, seqlens, idx, k, k_max: int, lam: float,
