@@ -173,12 +173,6 @@ __global__ void __launch_bounds__(kThreads) score_kernel(const ScoreParams p) {
     // every element of the prefetch buffer is written on every path (no read of an
     // uninitialised value on a warp's last batch)
     uint4 nxt[NI];
-    if (t + 2 < my_batches && lane == 0) {
-      // ask the L2 for the batch after next (its 32 rows are contiguous: one run of 64*R bytes)
-      const int pb = r0 + (warp + (t + 2) * kWarps) * kBatch;
-      const int rows = min(kBatch, r1 - pb);
-      if (rows > 0) bulk_prefetch_l2(row_ptr(pb), (uint32_t)(rows * R * 2 + 15) & ~15u);
-    }
     if (t + 1 < my_batches) {
       load(t + 1, nxt);
     } else {

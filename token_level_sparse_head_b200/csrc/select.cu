@@ -30,10 +30,10 @@ namespace {
 constexpr int kThreads = 512;
 constexpr int kWarps = kThreads / 32;
 constexpr int kBins = 2048;          // 11-bit digits
-constexpr int kPerThread = 16;       // keys per thread per tile (four 16-byte loads)
-constexpr int kTile = kThreads * kPerThread;
-constexpr int kCandCap = 8192;       // candidate keys kept on chip per CTA
-constexpr int kCand2Cap = 2048;      // survivors of the second digit
+constexpr int kStep = 16;            // keys per thread per step (four 16-byte loads)
+constexpr int kMaxRun = 256;         // keys per thread at most (the plan sizes clusters for it)
+constexpr int kWords = kMaxRun / 32; // per-thread position bitmask words
+constexpr int kOwnCand = 16;         // candidate keys kept on chip per thread
 
 struct Ctl {
   uint32_t cnt1, cnt2, gt0, pad;
@@ -48,9 +48,9 @@ struct SelSmem {
   uint32_t hl[kBins];        // this CTA's histogram
   uint32_t gh1[kBins];       // rank 0: cluster histogram of digit 2
   uint32_t gh2[kBins / 2];   // rank 0: cluster histogram of digit 3
-  uint32_t cand[kCandCap];
-  uint32_t cand2[kCand2Cap];
+  uint32_t cand[kOwnCand][kThreads];  // per-thread candidate keys, in position order
   uint32_t wsum[kWarps];
+  unsigned long long wsum64[kWarps];
   Ctl ctl;
   Found found;
 };
@@ -82,6 +82,30 @@ __device__ __forceinline__ uint32_t block_sum(uint32_t v, uint32_t* wsum) {
   uint32_t tot;
   block_excl_scan(v, wsum, &tot);
   return tot;
+}
+
+// Exclusive prefix sum of 64-bit values over the block; *total receives the block sum.
+__device__ __forceinline__ unsigned long long block_excl_scan64(unsigned long long v, unsigned long long* wsum,
+                                                                unsigned long long* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  unsigned long long x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const unsigned long long y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) wsum[warp] = x;
+  __syncthreads();
+  unsigned long long off = 0, tot = 0;
+#pragma unroll
+  for (int w = 0; w < kWarps; ++w) {
+    const unsigned long long s = wsum[w];
+    off += (w < warp) ? s : 0ull;
+    tot += s;
+  }
+  __syncthreads();
+  *total = tot;
+  return off + x - v;
 }
 
 // Warp-aggregated shared-memory histogram increment (many lanes share few bins).
@@ -152,19 +176,39 @@ __device__ __forceinline__ void red_add_cluster(const uint32_t* local, uint32_t 
   asm volatile("red.relaxed.cluster.shared::cluster.add.u32 [%0], %1;" ::"r"(ra), "r"(v) : "memory");
 }
 
-// Keys [t*kTile + tid*kPerThread, +kPerThread) of the chunk; positions past len read as 0 (and
-// are masked by the callers).
-__device__ __forceinline__ void load_tile(const uint32_t* gk, int len, int t, uint32_t (&k)[kPerThread]) {
-  const int li = t * kTile + (int)threadIdx.x * kPerThread;
-  if (li + kPerThread <= len) {
+// Step i of this thread's contiguous run: keys [base + 16 i, +16) of the chunk; positions past
+// the run or the chunk read as 0 (and are masked by the callers).  Cached loads: the four
+// 16-byte loads of a step share 32-byte sectors.
+__device__ __forceinline__ void load_step(const uint32_t* gk, int base, int end, int i, uint32_t (&k)[kStep]) {
+  const int li = base + i * kStep;
+  if (li + kStep <= end) {
 #pragma unroll
-    for (int v = 0; v < kPerThread / 4; ++v) {
-      const uint4 a = __ldcg(reinterpret_cast<const uint4*>(gk + li + 4 * v));
+    for (int v = 0; v < kStep / 4; ++v) {
+      const uint4 a = *reinterpret_cast<const uint4*>(gk + li + 4 * v);
       k[4 * v + 0] = a.x; k[4 * v + 1] = a.y; k[4 * v + 2] = a.z; k[4 * v + 3] = a.w;
     }
   } else {
 #pragma unroll
-    for (int e = 0; e < kPerThread; ++e) k[e] = (li + e < len) ? __ldcg(gk + li + e) : 0u;
+    for (int e = 0; e < kStep; ++e) k[e] = (li + e < end) ? gk[li + e] : 0u;
+  }
+}
+
+// Bit e of the result is set where positions base + e (e < 16) lie before `end`.
+__device__ __forceinline__ uint32_t valid_bits(int base, int end) {
+  const int n = end - base;
+  return n >= kStep ? 0xffffu : (n > 0 ? ((1u << n) - 1u) : 0u);
+}
+
+// Bitmasks of the keys k[e] with (k & mask) above / equal to `prefix`.
+__device__ __forceinline__ void step_masks(const uint32_t (&k)[kStep], uint32_t mask, uint32_t prefix,
+                                           uint32_t& above, uint32_t& equal) {
+  above = 0u;
+  equal = 0u;
+#pragma unroll
+  for (int e = 0; e < kStep; ++e) {
+    const uint32_t m = k[e] & mask;
+    above |= (m > prefix ? 1u : 0u) << e;
+    equal |= (m == prefix ? 1u : 0u) << e;
   }
 }
 
@@ -188,22 +232,29 @@ __global__ void __launch_bounds__(kThreads, 2) select_topk_kernel(const SelectPa
   // The exits are one guard around the body, not early returns.
   const bool trivial = !sel.ranked;
 
-  // this CTA's positions [c0, c1): chunks of whole 16-byte groups
+  // this CTA's positions [c0, c1); each thread owns a contiguous run of K of them
   const int chunk_b = (((n + C - 1) / C) + 15) & ~15;
   const int c0 = min(rank * chunk_b, n);
   const int c1 = min(c0 + chunk_b, n);
   const int len = c1 - c0;
   const uint32_t* gk = p.keys + (size_t)bh * p.cap + c0;
-  const int ntiles = (len + kTile - 1) / kTile;
+  const int K = ((len + kThreads - 1) / kThreads + kStep - 1) / kStep * kStep;
+  const int my0 = min(tid * K, len);
+  const int my1 = min(my0 + K, len);
+  const int nsteps = (my1 - my0 + kStep - 1) / kStep;
+  const int lane = tid & 31, warp = tid >> 5;
 
   if (trivial) {
     for (int j = rank * kThreads + tid; j < p.k_max; j += C * kThreads) idx[j] = (j < k_eff) ? j : -1;
   } else {
-    for (int i = tid; i < kBins + kBins + kBins / 2; i += kThreads) S.hl[i] = 0u;  // hl, gh1, gh2
-    if (tid == 0) {
-      S.ctl.cnt1 = 0u;
-      S.ctl.cnt2 = 0u;
+    // Bring the whole chunk of keys towards the SM early: the L2 fetches them from DRAM in
+    // large runs while the digit search below runs.
+    if (warp == 0) {
+      const int bytes = ((len * 4) + 15) & ~15;
+      for (int o = lane * 8192; o < bytes; o += 32 * 8192)
+        bulk_prefetch_l2(reinterpret_cast<const unsigned char*>(gk) + o, (uint32_t)min(8192, bytes - o));
     }
+    for (int i = tid; i < kBins + kBins + kBins / 2; i += kThreads) S.hl[i] = 0u;  // hl, gh1, gh2
     // ---- digit 1 from the global histogram ----
     const uint32_t* ghist = p.hist + (size_t)bh * kBins;
     uint32_t k_rem = (uint32_t)k_eff;
@@ -213,32 +264,45 @@ __global__ void __launch_bounds__(kThreads, 2) select_topk_kernel(const SelectPa
     uint32_t mask = 0x7ffu << 21;
     k_rem -= S.found.above;
     bool done = (S.found.eq == k_rem);
+    const bool done1 = done;
 
-    // ---- pass 1 over the chunk: keys above digit 1, candidates equal to it ----
-    uint32_t gt0 = 0u, eq0 = 0u;
-    {
-      uint32_t cur[kPerThread];
+    // ---- the one read of my run: bitmasks of the keys above digit 1 (gtm) and equal to it
+    // (cm); the equal ones (candidates) are also kept, in position order, in my slot ----
+    uint32_t gtm[kWords], cm[kWords];
 #pragma unroll
-      for (int e = 0; e < kPerThread; ++e) cur[e] = 0u;
-      if (ntiles > 0) load_tile(gk, len, 0, cur);
-      for (int t = 0; t < ntiles; ++t) {
-        uint32_t nxt[kPerThread];
+    for (int w = 0; w < kWords; ++w) {
+      gtm[w] = 0u;
+      cm[w] = 0u;
+    }
+    uint32_t nc = 0u;  // my candidates (beyond kOwnCand: keys re-read when needed)
+    for (int i = 0; i < nsteps; ++i) {
+      uint32_t k[kStep];
+      load_step(gk, my0, my1, i, k);
+      uint32_t sg, sc;
+      step_masks(k, 0x7ffu << 21, d0 << 21, sg, sc);
+      const uint32_t vb = valid_bits(my0 + i * kStep, my1);
+      sg &= vb;
+      sc &= vb;
+      const int sh = (i & 1) * kStep;
 #pragma unroll
-        for (int e = 0; e < kPerThread; ++e) nxt[e] = 0u;
-        if (t + 1 < ntiles) load_tile(gk, len, t + 1, nxt);
-        const int li = t * kTile + tid * kPerThread;
-#pragma unroll
-        for (int e = 0; e < kPerThread; ++e) {
-          const bool valid = li + e < len;
-          const uint32_t dg = cur[e] >> 21;
-          gt0 += (valid && dg > d0) ? 1u : 0u;
-          eq0 += (valid && dg == d0) ? 1u : 0u;
-          if (!done) list_append(S.cand, &S.ctl.cnt1, kCandCap, cur[e], valid && dg == d0);
+      for (int w = 0; w < kWords; ++w) {
+        if (w == (i >> 1)) {
+          gtm[w] |= sg << sh;
+          cm[w] |= sc << sh;
         }
+      }
+      if (sc != 0u && !done) {
 #pragma unroll
-        for (int e = 0; e < kPerThread; ++e) cur[e] = nxt[e];
+        for (int e = 0; e < kStep; ++e) {
+          if ((sc >> e) & 1u) {
+            if (nc < (uint32_t)kOwnCand) S.cand[nc][tid] = k[e];
+            ++nc;
+          }
+        }
       }
     }
+    const bool own_ovf = nc > (uint32_t)kOwnCand;
+    const uint32_t nown = min(nc, (uint32_t)kOwnCand);
     __syncthreads();
     // Every CTA has read the global histogram and zeroed its cluster histograms: after this
     // barrier rank 0 clears the global histogram for the next call, and the adds may start.
@@ -246,26 +310,30 @@ __global__ void __launch_bounds__(kThreads, 2) select_topk_kernel(const SelectPa
     if (rank == 0)
       for (int i = tid; i < kBins; i += kThreads) const_cast<uint32_t*>(ghist)[i] = 0u;
 
-    const uint32_t n1 = S.ctl.cnt1;
-    const bool ovf1 = n1 > (uint32_t)kCandCap;
-    // ---- digit 2: histogram of the candidates, summed over the cluster in rank 0 ----
-    if (!done) {
-      if (!ovf1) {
-        for (uint32_t e0 = 0; e0 < n1; e0 += kThreads) {
-          const uint32_t e = e0 + tid;
-          const uint32_t key = e < n1 ? S.cand[e] : 0u;
-          hist_add(S.hl, (key >> 10) & 0x7ffu, e < n1);
-        }
-      } else {
-        for (int t = 0; t < ntiles; ++t) {
-          uint32_t k[kPerThread];
-          load_tile(gk, len, t, k);
-          const int li = t * kTile + tid * kPerThread;
+    // Histogram of digit `shift` (11 bits at 10, or 10 bits at 0) of my candidates that match
+    // the current prefix, into hl: from my slot, or by re-reading my run when it overflowed.
+    auto cand_hist = [&](int shift, uint32_t dmask) {
 #pragma unroll
-          for (int e = 0; e < kPerThread; ++e)
-            hist_add(S.hl, (k[e] >> 10) & 0x7ffu, li + e < len && (k[e] & mask) == prefix);
+      for (int j = 0; j < kOwnCand; ++j) {
+        const uint32_t key = S.cand[j][tid];
+        const bool act = !own_ovf && (uint32_t)j < nown && (key & mask) == prefix;
+        hist_add(S.hl, (key >> shift) & dmask, act);
+      }
+      if (own_ovf) {
+        for (int i = 0; i < nsteps; ++i) {
+          uint32_t k[kStep];
+          load_step(gk, my0, my1, i, k);
+          const int li = my0 + i * kStep;
+#pragma unroll
+          for (int e = 0; e < kStep; ++e)
+            if (li + e < my1 && (k[e] & mask) == prefix) atomicAdd(&S.hl[(k[e] >> shift) & dmask], 1u);
         }
       }
+    };
+
+    // ---- digit 2 ----
+    if (!done) {
+      cand_hist(10, 0x7ffu);
       __syncthreads();
       const uint32_t* gh1 = S.hl;
       if (C > 1) {
@@ -285,40 +353,8 @@ __global__ void __launch_bounds__(kThreads, 2) select_topk_kernel(const SelectPa
     // ---- digit 3 ----
     if (!done) {
       for (int i = tid; i < kBins / 2; i += kThreads) S.hl[i] = 0u;
-      if (!ovf1) {
-        for (uint32_t e0 = 0; e0 < n1; e0 += kThreads) {
-          const uint32_t e = e0 + tid;
-          const uint32_t key = e < n1 ? S.cand[e] : 0u;
-          list_append(S.cand2, &S.ctl.cnt2, kCand2Cap, key, e < n1 && (key & mask) == prefix);
-        }
-      } else {
-        for (int t = 0; t < ntiles; ++t) {
-          uint32_t k[kPerThread];
-          load_tile(gk, len, t, k);
-          const int li = t * kTile + tid * kPerThread;
-#pragma unroll
-          for (int e = 0; e < kPerThread; ++e)
-            list_append(S.cand2, &S.ctl.cnt2, kCand2Cap, k[e], li + e < len && (k[e] & mask) == prefix);
-        }
-      }
       __syncthreads();
-      const uint32_t n2 = S.ctl.cnt2;
-      if (n2 <= (uint32_t)kCand2Cap) {
-        for (uint32_t e0 = 0; e0 < n2; e0 += kThreads) {
-          const uint32_t e = e0 + tid;
-          const uint32_t key = e < n2 ? S.cand2[e] : 0u;
-          hist_add(S.hl, key & 0x3ffu, e < n2);
-        }
-      } else {
-        for (int t = 0; t < ntiles; ++t) {
-          uint32_t k[kPerThread];
-          load_tile(gk, len, t, k);
-          const int li = t * kTile + tid * kPerThread;
-#pragma unroll
-          for (int e = 0; e < kPerThread; ++e)
-            hist_add(S.hl, k[e] & 0x3ffu, li + e < len && (k[e] & mask) == prefix);
-        }
-      }
+      cand_hist(0, 0x3ffu);
       __syncthreads();
       const uint32_t* gh2 = S.hl;
       if (C > 1) {
@@ -336,37 +372,42 @@ __global__ void __launch_bounds__(kThreads, 2) select_topk_kernel(const SelectPa
     }
     const uint32_t need = k_rem;  // how many of the threshold-key positions to take
 
-    // ---- CTA totals: above the threshold, equal to it ----
-    uint32_t my_gt = gt0, my_eq = 0u;
-    if (done && mask == (0x7ffu << 21)) {
-      my_eq = eq0;  // the first digit settled the threshold: its whole bin is selected
-    } else if (!ovf1) {
-      // keys above digit 1 are all above the threshold; the rest is among the candidates
-      for (uint32_t e = tid; e < n1; e += kThreads) {
-        const uint32_t m = S.cand[e] & mask;
-        my_gt += (m > prefix) ? 1u : 0u;
-        my_eq += (m == prefix) ? 1u : 0u;
-      }
-    } else {
-      my_gt = 0u;
-      for (int t = 0; t < ntiles; ++t) {
-        uint32_t k[kPerThread];
-        load_tile(gk, len, t, k);
-        const int li = t * kTile + tid * kPerThread;
+    // The key of my j-th candidate (position order), from my slot or from memory.
+    auto own_key = [&](uint32_t j, int pos_in_chunk) -> uint32_t {
+      return own_ovf ? gk[pos_in_chunk] : S.cand[j][tid];
+    };
+
+    // ---- my counts above / equal to the threshold ----
+    uint32_t my_gt = 0u, my_eq = 0u;
 #pragma unroll
-        for (int e = 0; e < kPerThread; ++e) {
-          const uint32_t m = k[e] & mask;
-          const bool valid = li + e < len;
-          my_gt += (valid && m > prefix) ? 1u : 0u;
-          my_eq += (valid && m == prefix) ? 1u : 0u;
+    for (int w = 0; w < kWords; ++w) {
+      my_gt += (uint32_t)__popc(gtm[w]);
+      my_eq += (uint32_t)__popc(cm[w]);
+    }
+    if (!done1) {
+      // the candidates split by their full keys
+      uint32_t cgt = 0u, ceq = 0u, j = 0u;
+#pragma unroll
+      for (int w = 0; w < kWords; ++w) {
+        uint32_t bits = cm[w];
+        while (bits) {
+          const int bpos = __ffs(bits) - 1;
+          bits &= bits - 1u;
+          const uint32_t m = own_key(j, my0 + w * 32 + bpos) & mask;
+          ++j;
+          cgt += (m > prefix) ? 1u : 0u;
+          ceq += (m == prefix) ? 1u : 0u;
         }
       }
+      my_gt += cgt;
+      my_eq = ceq;
     }
-    const uint32_t cta_gt = block_sum(my_gt, S.wsum);
-    const uint32_t cta_eq = block_sum(my_eq, S.wsum);
+    unsigned long long tot;
+    const unsigned long long ex =
+        block_excl_scan64(((unsigned long long)my_gt << 32) | my_eq, S.wsum64, &tot);
     if (tid == 0) {
-      S.ctl.cta_gt = cta_gt;
-      S.ctl.cta_eq = cta_eq;
+      S.ctl.cta_gt = (uint32_t)(tot >> 32);
+      S.ctl.cta_eq = (uint32_t)tot;
     }
     uint32_t gt_base = 0u, eq_base = 0u;
     if (C > 1) {
@@ -393,48 +434,39 @@ __global__ void __launch_bounds__(kThreads, 2) select_topk_kernel(const SelectPa
       eq_base = S.ctl.eq_before;
     }
 
-    // ---- pass 2 over the chunk: ordered compaction, one block scan per tile ----
+    // ---- write my selected positions in order (no further reads unless my slot overflowed) ----
     {
-      uint32_t cur[kPerThread];
+      uint32_t gc = gt_base + (uint32_t)(ex >> 32);
+      uint32_t ec = eq_base + (uint32_t)ex;
+      uint32_t j = 0u;
 #pragma unroll
-      for (int e = 0; e < kPerThread; ++e) cur[e] = 0u;
-      if (ntiles > 0) load_tile(gk, len, 0, cur);
-      for (int t = 0; t < ntiles; ++t) {
-        uint32_t nxt[kPerThread];
-#pragma unroll
-        for (int e = 0; e < kPerThread; ++e) nxt[e] = 0u;
-        if (t + 1 < ntiles) load_tile(gk, len, t + 1, nxt);
-        const int li = t * kTile + tid * kPerThread;
-        uint32_t tg = 0u, te = 0u;
-#pragma unroll
-        for (int e = 0; e < kPerThread; ++e) {
-          const uint32_t m = cur[e] & mask;
-          const bool valid = li + e < len;
-          tg += (valid && m > prefix) ? 1u : 0u;
-          te += (valid && m == prefix) ? 1u : 0u;
-        }
-        uint32_t tot;
-        const uint32_t ex = block_excl_scan((tg << 16) | te, S.wsum, &tot);
-        uint32_t gc = gt_base + (ex >> 16);
-        uint32_t ec = eq_base + (ex & 0xffffu);
-#pragma unroll
-        for (int e = 0; e < kPerThread; ++e) {
-          const uint32_t m = cur[e] & mask;
-          if (li + e < len) {
-            const int pos = c0 + li + e;
-            if (m > prefix) {
-              idx[gc + min(ec, need)] = pos;
-              ++gc;
-            } else if (m == prefix) {
-              if (ec < need) idx[gc + ec] = pos;
-              ++ec;
-            }
+      for (int w = 0; w < kWords; ++w) {
+        uint32_t bits = gtm[w] | cm[w];
+        while (bits) {
+          const int bpos = __ffs(bits) - 1;
+          bits &= bits - 1u;
+          const int pic = my0 + w * 32 + bpos;  // position in the chunk
+          bool above, equal;
+          if ((gtm[w] >> bpos) & 1u) {
+            above = true;
+            equal = false;
+          } else if (done1) {
+            above = false;
+            equal = true;
+          } else {
+            const uint32_t m = own_key(j, pic) & mask;
+            above = m > prefix;
+            equal = m == prefix;
+          }
+          if (!((gtm[w] >> bpos) & 1u)) ++j;
+          if (above) {
+            idx[gc + min(ec, need)] = c0 + pic;
+            ++gc;
+          } else if (equal) {
+            if (ec < need) idx[gc + ec] = c0 + pic;
+            ++ec;
           }
         }
-        gt_base += tot >> 16;
-        eq_base += tot & 0xffffu;
-#pragma unroll
-        for (int e = 0; e < kPerThread; ++e) cur[e] = nxt[e];
       }
     }
     for (int j = k_eff + rank * kThreads + tid; j < p.k_max; j += C * kThreads) idx[j] = -1;
@@ -449,10 +481,12 @@ bool plan_select(SelectParams& p, int num_sms) {
   // Double the CTAs per head while the grid still fits one wave of two CTAs per SM and each
   // CTA keeps at least one tile of keys.
   int C = 1;
-  while (C < kMaxCluster && (long)heads * C * 2 <= 2L * num_sms && (p.cap + 2 * C - 1) / (2 * C) >= kTile) C *= 2;
+  while (C < kMaxCluster && (p.cap + C - 1) / C > kThreads * kMaxRun) C *= 2;
+  while (C < kMaxCluster && (long)heads * C * 2 <= 2L * num_sms && (p.cap + 2 * C - 1) / (2 * C) >= kThreads * kStep) C *= 2;
+  if ((p.cap + C - 1) / C > kThreads * kMaxRun) return false;
   p.cluster = C;
   p.chunk = (((p.cap + C - 1) / C) + 15) & ~15;
-  p.cand_cap = kCandCap;
+  p.cand_cap = kThreads * kOwnCand;
   p.off_hist = 0;
   p.off_ctl = 0;
   p.smem_bytes = (int)sizeof(SelSmem);
