@@ -195,6 +195,50 @@ sas_status sas_dense_decode(const sas_shape* shape, const void* q, const void* K
                             const int32_t* page_table, const int32_t* seqlens, float* out,
                             void* workspace, size_t ws_bytes, void* stream);
 
+/* Bytes of the library's fixed scratch array (16 MiB), used by sas_decode_step_static_scratch. */
+#define SAS_STATIC_SCRATCH_BYTES (16u << 20)
+
+/* sas_decode_step without a caller workspace.  The pages describe no such call: it is an
+ * interface convenience with no counterpart in the method.
+ *
+ * Who needs it: callers that cannot hand the library device memory, e.g. a C or C++ host
+ * that owns no device allocator and must not call cudaMalloc on its decode path (cudaMalloc
+ * can stall the whole device), or a plug-in inside a framework whose caching allocator owns
+ * every byte of device memory and offers extension code no scratch buffer.  This call makes
+ * no allocation of any kind: its scratch is a fixed array of SAS_STATIC_SCRATCH_BYTES in the
+ * library's device image, placed by the CUDA driver when the library's device code is loaded
+ * on a device (at its first use under lazy module loading, CUDA's default).
+ *
+ * Arguments, outputs and results are those of sas_decode_step (same kernels, same launch
+ * configuration); there is no workspace argument.
+ *
+ * Size limit: the shape and k_max must need at most SAS_STATIC_SCRATCH_BYTES of workspace,
+ * i.e. sas_decode_workspace_bytes(shape, k_max) <= SAS_STATIC_SCRATCH_BYTES.  For example
+ * B=1, Hq=32, Hkv=8, d=128, r=32, 131072 tokens, k_max=4096 needs about 4.6 MiB and B=4 at
+ * 65536 tokens about 10.3 MiB; B=16 at 131072 tokens needs 67 MiB and is rejected.  A shape
+ * over the limit returns SAS_ERR_UNSUPPORTED before anything is launched, with the sizes in
+ * sas_last_error_detail(); use sas_decode_step with a workspace for it.
+ *
+ * Setup: the first call on each device looks up the array's device address
+ * (cudaGetSymbolAddress) with that device current, and caches it; make that first call before
+ * any stream capture begins.  The current device selects which device's array is used.
+ *
+ * Sharing: all calls on one device use the same array.  Calls that overlap in time on that
+ * device (different streams, or different host threads, without ordering between them) race
+ * on it and give wrong results; order them on one stream.  Each call first clears, on
+ * `stream`, the part of the array that must start at zero (the device error word, the
+ * per-head histograms and the split counters); the rest is written before it is read.
+ *
+ * Device-side checks still run, but their error word lives in the shared array, is cleared by
+ * the next call and cannot be read with sas_check_workspace: callers that need the device
+ * checks reported use sas_decode_step with their own workspace. */
+sas_status sas_decode_step_static_scratch(const sas_shape* shape, const void* q, const float* M,
+                                          const void* Kproj, const void* K, const void* V,
+                                          const int32_t* page_table, const int32_t* seqlens,
+                                          const int32_t* k, int32_t k_max, float lambda,
+                                          const float* log_g, float* out, int32_t* idx_out,
+                                          void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -4,6 +4,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 
 #include "sas.h"
 #include "sas_kernels.h"
@@ -414,6 +415,83 @@ sas_status sas_dense_decode(const sas_shape* shape, const void* q, const void* K
   if (ws_bytes < sas_dense_workspace_bytes(shape)) return fail(SAS_ERR_INVALID_ARG, "workspace too small");
   return do_attend(shape, q, K, V, page_table, seqlens, nullptr, nullptr, cap_of(shape), 0.0f, nullptr, out,
                    workspace, static_cast<cudaStream_t>(stream));
+}
+
+}  // extern "C"
+
+// ---------------------------------------------------------------------------------------------
+// sas_decode_step_static_scratch: the decode step on a fixed scratch array that belongs to the
+// library, for callers that cannot provide a workspace.  The array is part of this file's
+// device image, so no allocation call is ever made for it: the CUDA driver places it when the
+// image is loaded on a device.  One array per device, shared by every call on that device.
+// ---------------------------------------------------------------------------------------------
+static __device__ __align__(256) unsigned char g_static_scratch[SAS_STATIC_SCRATCH_BYTES];
+
+namespace {
+
+constexpr int kMaxScratchDevices = 64;
+std::mutex g_scratch_mutex;
+void* g_scratch_ptr[kMaxScratchDevices] = {};
+
+// Address of this device's copy of g_static_scratch.  The first call on a device looks it up
+// with that device current; later calls reuse the cached pointer.
+sas_status static_scratch_ptr(void** out) {
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxScratchDevices)
+    return fail(SAS_ERR_UNSUPPORTED, "device ordinal %d: the static scratch supports devices 0..%d", dev,
+                kMaxScratchDevices - 1);
+  std::lock_guard<std::mutex> lock(g_scratch_mutex);
+  if (g_scratch_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_static_scratch);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress of the static scratch");
+    g_scratch_ptr[dev] = p;
+  }
+  *out = g_scratch_ptr[dev];
+  return SAS_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+sas_status sas_decode_step_static_scratch(const sas_shape* shape, const void* q, const float* M,
+                                          const void* Kproj, const void* K, const void* V,
+                                          const int32_t* page_table, const int32_t* seqlens, const int32_t* k,
+                                          int32_t k_max, float lambda, const float* log_g, float* out,
+                                          int32_t* idx_out, void* stream) {
+  SAS_TRY(check_shape(shape));
+  if (k_max < 1) return fail(SAS_ERR_INVALID_ARG, "k_max must be >= 1");
+  const size_t need = sas_decode_workspace_bytes(shape, k_max);
+  if (need > (size_t)SAS_STATIC_SCRATCH_BYTES)
+    return fail(SAS_ERR_UNSUPPORTED,
+                "this shape and k_max need %zu bytes of scratch, more than the %zu-byte static scratch; "
+                "call sas_decode_step with a caller workspace instead",
+                need, (size_t)SAS_STATIC_SCRATCH_BYTES);
+  SAS_TRY(check_ptr(q, "q"));
+  SAS_TRY(check_ptr(M, "M"));
+  SAS_TRY(check_ptr(Kproj, "Kproj"));
+  SAS_TRY(check_ptr(K, "K"));
+  SAS_TRY(check_ptr(V, "V"));
+  SAS_TRY(check_ptr(k, "k"));
+  SAS_TRY(check_ptr(out, "out"));
+  SAS_TRY(check_ptr(idx_out, "idx_out"));
+  SAS_TRY(check_cache_ptrs(shape, page_table, seqlens));
+  if (lambda != 0.0f) SAS_TRY(check_ptr(log_g, "log_g"));
+
+  void* ws = nullptr;
+  SAS_TRY(static_scratch_ptr(&ws));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // The error word, the per-head histograms and the split counters must start at zero; a
+  // previous call may have been cut short, so every call clears them.  The score keys and
+  // the attention partials that follow are written before they are read.
+  const WsLayout L = ws_layout(attend_plan(shape, k_max), true);
+  const cudaError_t e = cudaMemsetAsync(ws, 0, L.partials, st);
+  if (e != cudaSuccess) return cuda_fail(e, "clearing the static scratch");
+  SAS_TRY(do_select(shape, q, M, Kproj, page_table, seqlens, k, k_max, lambda, log_g, idx_out, nullptr, ws, st));
+  return do_attend(shape, q, K, V, page_table, seqlens, idx_out, k, k_max, lambda, log_g, out, ws, st);
 }
 
 }  // extern "C"

@@ -50,7 +50,10 @@ _SIGS = {
                                             _vp, _i32, _f32, _vp, _vp, _vp, _sz, _vp]),
     "sas_dense_decode": (ctypes.c_int, [ctypes.POINTER(sas_shape), _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                                         _sz, _vp]),
+    "sas_decode_step_static_scratch": (ctypes.c_int, [ctypes.POINTER(sas_shape), _vp, _vp, _vp, _vp, _vp, _vp,
+                                                      _vp, _vp, _i32, _f32, _vp, _vp, _vp, _vp]),
 }
+STATIC_SCRATCH_BYTES = 16 << 20  # SAS_STATIC_SCRATCH_BYTES
 EXPORTED = tuple(_SIGS)
 
 
@@ -215,3 +218,12 @@ def sas_dense_decode(shape: Shape, q, K, V, page_table, seqlens, out, workspace,
     _check(load().sas_dense_decode(ctypes.byref(shape.c()), _p(q), _p(K), _p(V), _p(page_table),
                                    _p(seqlens), _p(out), _p(workspace), int(ws_bytes), _stream(stream)),
            "sas_dense_decode")
+
+
+def sas_decode_step_static_scratch(shape: Shape, q, M, Kproj, K, V, page_table, seqlens, k, k_max: int,
+                                   lam: float, log_g, out, idx_out, stream=None):
+    """sas_decode_step on the library's fixed scratch array (no workspace argument)."""
+    _check(load().sas_decode_step_static_scratch(ctypes.byref(shape.c()), _p(q), _p(M), _p(Kproj), _p(K), _p(V),
+                                                 _p(page_table), _p(seqlens), _p(k), int(k_max), float(lam),
+                                                 _p(log_g), _p(out), _p(idx_out), _stream(stream)),
+           "sas_decode_step_static_scratch")
