@@ -214,8 +214,8 @@ sas_status sas_dense_decode(const sas_shape* shape, const void* q, const void* K
  *
  * Size limit: the shape and k_max must need at most SAS_STATIC_SCRATCH_BYTES of workspace,
  * i.e. sas_decode_workspace_bytes(shape, k_max) <= SAS_STATIC_SCRATCH_BYTES.  For example
- * B=1, Hq=32, Hkv=8, d=128, r=32, 131072 tokens, k_max=4096 needs about 4.6 MiB and B=4 at
- * 65536 tokens about 10.3 MiB; B=16 at 131072 tokens needs 67 MiB and is rejected.  A shape
+ * B=1, Hq=32, Hkv=8, d=128, r=32, 131072 tokens, k_max=4096 needs about 4.8 MiB and B=4 at
+ * 65536 tokens about 11 MiB; B=16 at 131072 tokens needs 70 MiB and is rejected.  A shape
  * over the limit returns SAS_ERR_UNSUPPORTED before anything is launched, with the sizes in
  * sas_last_error_detail(); use sas_decode_step with a workspace for it.
  *

@@ -91,7 +91,7 @@ WsLayout ws_layout(const sas::AttendParams& a, bool with_keys) {
   WsLayout w;
   size_t o = kErrBytes;
   w.hist = o;
-  o += (size_t)a.B * a.Hkv * 2048 * 4;
+  o += (size_t)a.B * a.Hkv * sas::kHistBins * 4;
   w.counters = o;
   o += ((size_t)a.B * a.Hkv * a.ngz * 4 + 255) & ~(size_t)255;
   w.partials = o;

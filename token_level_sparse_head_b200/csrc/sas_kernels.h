@@ -8,6 +8,13 @@
 
 namespace sas {
 
+// Radix digits of the 32-bit score keys used by the selection: 13 + 10 + 9 bits.  The score
+// kernel histograms the first digit of every (b, h).
+constexpr int kHistShift = 19;
+constexpr int kHistBins = 1 << (32 - kHistShift);  // 8192
+constexpr int kDigit2Bits = 10;
+constexpr int kDigit3Bits = 9;
+
 // ---------------------------------------------------------------------------- projection
 struct ProjParams {
   const __nv_bfloat16* K;      // build: cache (layout below); append: K_new [B][Hkv][d]
@@ -33,12 +40,12 @@ struct ScoreParams {
   const int32_t* kvec;         // [B]
   const float* log_g;          // [B][Hkv][cap] or null
   uint32_t* keys;              // workspace: [B][Hkv][cap] order-preserving keys of u_i
-  uint32_t* hist;              // workspace: [B][Hkv][2048] counts of the keys' top 11 bits (zero on entry)
+  uint32_t* hist;              // workspace: [B][Hkv][kHistBins] counts of the keys' first digit (zero on entry)
   float* scores_out;           // [B][Hkv][cap] or null
   uint32_t* err;
   int B, Hq, Hkv, G, d, r, cap, max_pages, num_pages, paged, k_max;
   float sigma, lam;
-  int rows_per_cta;
+  int ctas;                    // persistent grid size
 };
 void plan_score(ScoreParams& p, int num_sms);
 cudaError_t launch_score(const ScoreParams& p, cudaStream_t stream);

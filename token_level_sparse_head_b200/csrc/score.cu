@@ -5,243 +5,437 @@
 // h; section Triton 内核的三个设计点: scoring is not sparse, it scans every candidate.  The gate
 // of the SAS page (section 2.1) adds lambda * log g_i.  Each score is kept as the order-preserving
 // uint32 key of u_i = sigma * s-hat_i (+ lambda log g_i); a per-(b, h) histogram of the keys' top
-// 11 bits is accumulated for the selection that follows.
+// 13 bits is accumulated for the selection that follows.
 //
-// The projected cache is streamed with fully coalesced 16-byte loads (a warp reads 32 rows as
-// one 2*r*32-byte run per instruction group, the next batch prefetched into registers), at
-// high occupancy; the keys go to the workspace with an L2 evict-last hint so that the
-// selection kernel finds them on chip, the cache rows with evict-first.
+// Persistent kernel, one CTA per SM.  The work is the list of 4 KB blocks of projected rows
+// (64 rows at r = 32) of every (b, h) that needs scores, in (b, h, position) order; each CTA
+// takes one contiguous, equal share of it, so a CTA walks the rows of one or a few heads front
+// to back.  A producer warp streams the blocks into a shared-memory ring with bulk copies (TMA
+// engine: one copy per block, or per 64-token page piece for the paged layout, plus the block's
+// gate values); each of its lanes owns one ring slot.  Sixteen consumer warps take the blocks in
+// turn, each with its own two ring slots, so every warp's dependent chain (dot products,
+// butterfly reduction, key, histogram) overlaps the others' and about 130 KB of rows stay in
+// flight per SM.  Full blocks take a path without per-row tests.  Keys go to the workspace with
+// an L2 evict-last hint so that the selection kernel finds them on chip.
 #include "sas_device.cuh"
 #include "sas_kernels.h"
 
 namespace sas {
 namespace {
 
-constexpr int kThreads = 256;
-constexpr int kWarps = kThreads / 32;
-constexpr int kBatch = 32;  // rows per warp per batch
-constexpr int kBins = 2048;
-constexpr int kMaxRowsPerCta = 64 * kWarps * kBatch;
+constexpr int kConsumerWarps = 16;
+constexpr int kConsumers = kConsumerWarps * 32;
+constexpr int kThreads = kConsumers + 32;  // + one producer warp
+constexpr int kBlockBytes = 4096;          // projected bytes per block (one ring stage)
+constexpr int kDepth = 2;                  // ring slots per consumer warp
+constexpr int kSlots = kConsumerWarps * kDepth;
 
-__device__ __forceinline__ uint64_t policy_evict_first() {
-  uint64_t pol;
-  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
-  return pol;
-}
+template <int R>
+struct Geo {
+  static constexpr int ROW_BYTES = 2 * R;
+  static constexpr int BLOCK_ROWS = kBlockBytes / ROW_BYTES;  // 128 / 64 / 32 for r = 16 / 32 / 64
+  static constexpr int NB = BLOCK_ROWS / 32;                  // 32-row batches per block
+  static constexpr int LG_BYTES = BLOCK_ROWS * 4;             // gate values of one block
+  static constexpr int SLOT_BYTES = kBlockBytes + LG_BYTES;
+  static constexpr int LPR = R / 8;     // lanes per row, 16 bytes each
+  static constexpr int RPI = 32 / LPR;  // rows per load instruction
+  static constexpr int NI = LPR;        // load instructions per 32-row batch
+  static constexpr int LOG_LPR = LPR == 2 ? 1 : LPR == 4 ? 2 : 3;
+};
+
+// Position of a CTA's share in the block list, computed once by the producer warp.
+struct Plan {
+  int count;  // blocks of this CTA
+  int b0;     // sequence of the first block
+  int h0, c0; // KV head and block index within it
+};
+
+template <int R, int D>
+struct Smem {
+  unsigned char ring[kSlots][Geo<R>::SLOT_BYTES];
+  uint32_t hist[kHistBins];
+  float qbar[D];
+  float qhat[R];
+  uint64_t full[kSlots];
+  uint64_t empty[kSlots];
+  Plan plan;
+};
+static_assert(sizeof(Smem<16, 128>) <= 227 * 1024 && sizeof(Smem<32, 128>) <= 227 * 1024 &&
+                  sizeof(Smem<64, 128>) <= 227 * 1024,
+              "score kernel shared memory");
+
 __device__ __forceinline__ uint64_t policy_evict_last() {
   uint64_t pol;
   asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
   return pol;
 }
-__device__ __forceinline__ uint4 ldg_hint(const void* ptr, uint64_t pol) {
-  uint4 v;
-  asm volatile("ld.global.nc.L1::no_allocate.L2::cache_hint.v4.u32 {%0,%1,%2,%3}, [%4], %5;"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-               : "l"(ptr), "l"(pol));
-  return v;
-}
 __device__ __forceinline__ void stg_hint(uint32_t* ptr, uint32_t v, uint64_t pol) {
   asm volatile("st.global.L2::cache_hint.u32 [%0], %1, %2;" ::"l"(ptr), "r"(v), "l"(pol) : "memory");
 }
-
-// Warp-aggregated shared-memory histogram increment.
-__device__ __forceinline__ void hist_add(uint32_t* hist, uint32_t bin, bool active) {
-  const uint32_t act = __ballot_sync(0xffffffffu, active);
-  if (!active) return;
-  const uint32_t peers = __match_any_sync(act, bin);
-  if ((__ffs(peers) - 1) == (int)(threadIdx.x & 31)) atomicAdd(&hist[bin], (uint32_t)__popc(peers));
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+// Barrier 1 among the consumer warps only (the producer warp never joins it).
+__device__ __forceinline__ void consumers_sync() {
+  asm volatile("bar.sync 1, %0;" ::"n"(kConsumers) : "memory");
 }
 
-template <int R, int D>
-__global__ void __launch_bounds__(kThreads) score_kernel(const ScoreParams p) {
-  constexpr int LPR = R / 8;         // lanes per row (16 bytes each)
-  constexpr int RPI = 32 / LPR;      // rows per load instruction
-  constexpr int NI = kBatch / RPI;   // load instructions per batch
-  __shared__ float qbar[D];
-  __shared__ float qhat[R];
-  __shared__ uint32_t hist[kBins];
-  __shared__ int pages_s[kMaxRowsPerCta / 64];
+// Dot product of 8 bf16 values (one 16-byte chunk of a row) with this lane's 8 channels of q-hat.
+__device__ __forceinline__ float dot8(const float2 (&qv)[4], uint4 w) {
+  float2 a = ffma2(qv[0], make_float2(bf16lo(w.x), bf16hi(w.x)), make_float2(0.f, 0.f));
+  a = ffma2(qv[1], make_float2(bf16lo(w.y), bf16hi(w.y)), a);
+  a = ffma2(qv[2], make_float2(bf16lo(w.z), bf16hi(w.z)), a);
+  a = ffma2(qv[3], make_float2(bf16lo(w.w), bf16hi(w.w)), a);
+  return a.x + a.y;
+}
 
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int bh = blockIdx.y;
-  const int b = bh / p.Hkv, h = bh % p.Hkv;
+// Transposing butterfly over the LPR lanes of a row: v[i] holds this lane's partial dot of row
+// i * RPI + rsub; afterwards the result is the full score of row part * RPI + rsub.
+template <class Gm>
+__device__ __forceinline__ float butterfly(float (&v)[Gm::NI], int lane) {
+#pragma unroll
+  for (int lvl = 0; lvl < Gm::LOG_LPR; ++lvl) {
+    const int m = Gm::LPR >> (lvl + 1);
+    const int half = Gm::NI >> (lvl + 1);
+    const bool upper = (lane & m) != 0;
+#pragma unroll
+    for (int i = 0; i < half; ++i) {
+      const float send = upper ? v[i] : v[i + half];
+      const float keep = upper ? v[i + half] : v[i];
+      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, m);
+    }
+  }
+  return v[0];
+}
+
+// Cached length and scored block count of one sequence.  Both sides of the kernel compute
+// the same values (the producer records bad inputs, once, in CTA 0).
+struct SeqInfo {
+  int n;        // N_b (0 if out of range)
+  int blocks;   // blocks that need scores (0 when nothing is ranked or reported)
+  bool ranked;  // the selection ranks this sequence: histogram needed
+};
+template <int BR>
+__device__ __forceinline__ SeqInfo seq_info(const ScoreParams& p, int b, bool record) {
   int n = p.seqlens[b];
   if (n < 0 || n > p.cap) {
-    if (blockIdx.x == 0 && tid == 0 && h == 0) record_error(p.err, kDevBadSeqlen, (uint32_t)b);
+    if (record) record_error(p.err, kDevBadSeqlen, (uint32_t)b);
     n = 0;
   }
   int kb = p.kvec[b];
   if (kb > p.k_max) {
-    if (blockIdx.x == 0 && tid == 0 && h == 0) record_error(p.err, kDevKOverMax, (uint32_t)b);
+    if (record) record_error(p.err, kDevKOverMax, (uint32_t)b);
     kb = p.k_max;
   }
-  // Nothing to rank (empty selection or every position selected): no scores are needed,
-  // unless the caller asked for them.  The CTA-uniform exits are expressed as one guard
-  // around the body rather than early returns.
-  const bool need_hist = seq_selection(kb, n).ranked;  // the selection ranks this (b, h)
-  const int r0 = blockIdx.x * p.rows_per_cta;
-  const int r1 = min(r0 + p.rows_per_cta, n);
-  const bool skip = (!need_hist && p.scores_out == nullptr) || r0 >= r1;
-  if (!skip) {
-  if (p.paged) {
-    for (int t = tid; t < (r1 - r0 + 63) / 64; t += kThreads) {
-      int pg = p.page_table[(size_t)b * p.max_pages + r0 / 64 + t];
-      if (pg < 0 || pg >= p.num_pages) {
-        record_error(p.err, kDevBadPage, (uint32_t)b);
-        pg = 0;
+  SeqInfo s;
+  s.n = n;
+  s.ranked = seq_selection(kb, n).ranked;
+  s.blocks = (s.ranked || p.scores_out != nullptr) ? (n + BR - 1) / BR : 0;
+  return s;
+}
+
+// The first (b, h) at or after sequence b with blocks to score (b == B when there is none).
+template <int BR>
+__device__ __forceinline__ void next_scored_seq(const ScoreParams& p, int& b, SeqInfo& si) {
+  while (b < p.B && (si = seq_info<BR>(p, b, false)).blocks == 0) ++b;
+}
+
+template <int R, int D, bool GATED>
+__global__ void __launch_bounds__(kThreads, 1) score_kernel(const ScoreParams p) {
+  using Gm = Geo<R>;
+  constexpr int BR = Gm::BLOCK_ROWS;
+  extern __shared__ __align__(128) unsigned char smem_raw[];
+  Smem<R, D>& S = *reinterpret_cast<Smem<R, D>*>(smem_raw);
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+
+  if (tid == 0) {
+    for (int s = 0; s < kSlots; ++s) {
+      mbar_init(&S.full[s], 1);
+      mbar_init(&S.empty[s], 1);
+    }
+    fence_barrier_init();
+  }
+  for (int i = tid; i < kHistBins; i += kThreads) S.hist[i] = 0u;
+
+  // ---- this CTA's share of the block list (producer warp) ----
+  if (warp == kConsumerWarps) {
+    // per-lane block counts of sequences lane, lane + 32, ...; the first 32 are kept
+    long long mine = 0;
+    long long first = 0;
+    for (int b = lane; b < p.B; b += 32) {
+      const long long c = (long long)p.Hkv * seq_info<BR>(p, b, blockIdx.x == 0).blocks;
+      if (b < 32) first = c;
+      mine += c;
+    }
+    long long total = mine;
+#pragma unroll
+    for (int o = 16; o; o >>= 1) total += __shfl_xor_sync(0xffffffffu, total, o);
+    const long long beg = total * blockIdx.x / gridDim.x;
+    const long long end = total * (blockIdx.x + 1) / gridDim.x;
+    // first sequence whose blocks contain `beg`
+    int b0 = p.B;
+    long long before = 0, cum = 0;
+    if (beg < end) {
+      for (int base = 0; base < p.B; base += 32) {
+        const int b = base + lane;
+        long long cnt = first;
+        if (base > 0) cnt = b < p.B ? (long long)p.Hkv * seq_info<BR>(p, b, false).blocks : 0;
+        if (b >= p.B) cnt = 0;
+        long long incl = cnt;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const long long t = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += t;
+        }
+        const long long start = cum + incl - cnt;
+        const uint32_t hit = __ballot_sync(0xffffffffu, cnt > 0 && start <= beg && beg < start + cnt);
+        if (hit) {
+          const int l = __ffs(hit) - 1;
+          b0 = base + l;
+          before = __shfl_sync(0xffffffffu, start, l);
+          break;
+        }
+        cum += __shfl_sync(0xffffffffu, incl, 31);
       }
-      pages_s[t] = pg;
+    }
+    if (lane == 0) {
+      Plan pl = {0, p.B, 0, 0};
+      if (b0 < p.B) {
+        const int nb = seq_info<BR>(p, b0, false).blocks;
+        const long long off = beg - before;
+        pl.count = (int)(end - beg);
+        pl.b0 = b0;
+        pl.h0 = (int)(off / nb);
+        pl.c0 = (int)(off % nb);
+      }
+      S.plan = pl;
     }
   }
-
-  // ---- q-hat = sigma * M[h] q-bar (independent vector loads) ----
-  constexpr int TPR = kThreads / R;
-  constexpr int CH = D / TPR;
-  const int qj = tid / TPR, qpart = tid % TPR;
-  float4 mreg[CH / 4];
-  {
-    const float4* Mrow = reinterpret_cast<const float4*>(p.M + ((size_t)h * R + qj) * D + qpart * CH);
-#pragma unroll
-    for (int i = 0; i < CH / 4; ++i) mreg[i] = Mrow[i];
-  }
-  if (tid < D) {
-    const __nv_bfloat16* qg = p.q + ((size_t)b * p.Hq + (size_t)h * p.G) * D + tid;
-    float sq = 0.f;
-#pragma unroll 4
-    for (int g = 0; g < p.G; ++g) sq += __bfloat162float(qg[(size_t)g * D]);
-    qbar[tid] = sq / (float)p.G;
-  }
-  for (int i = tid; i < kBins; i += kThreads) hist[i] = 0u;
   __syncthreads();
-  {
-    float sp = 0.f;
-#pragma unroll
-    for (int i = 0; i < CH / 4; ++i) {
-      const float* qb = qbar + qpart * CH + 4 * i;
-      sp = fmaf(mreg[i].x, qb[0], sp);
-      sp = fmaf(mreg[i].y, qb[1], sp);
-      sp = fmaf(mreg[i].z, qb[2], sp);
-      sp = fmaf(mreg[i].w, qb[3], sp);
+  const Plan pl = S.plan;
+  const bool gated = GATED;
+  const bool scores = p.scores_out != nullptr;
+  bool waited_ok = true;
+
+  if (warp == kConsumerWarps) {
+    // ---------------------------------------------------------------- producer
+    // Lane l owns ring slot l (kSlots == 32) and issues the CTA's blocks l, l + 32, l + 64, ...
+    // into it, each once consumer warp l % 16 has released the slot.
+    static_assert(kSlots == 32, "one producer lane per ring slot");
+    if (pl.count > lane) {
+      const unsigned char* kp = reinterpret_cast<const unsigned char*>(p.kproj);
+      int b = pl.b0, h = pl.h0, c = pl.c0;
+      SeqInfo si = seq_info<BR>(p, b, false);
+      // advance the walk by k blocks
+      auto advance = [&](int k) {
+        while (k > 0 && b < p.B) {
+          const int take = min(k, si.blocks - c);
+          c += take;
+          k -= take;
+          if (c == si.blocks) {
+            c = 0;
+            if (++h == p.Hkv) {
+              h = 0;
+              ++b;
+              next_scored_seq<BR>(p, b, si);
+            }
+          }
+        }
+      };
+      advance(lane);
+      const int slot = lane;
+      uint32_t phase = 0u;
+      for (int t = lane; t < pl.count; t += kSlots) {
+        if (t >= kSlots) {
+          if (!mbar_wait_bounded(&S.empty[slot], phase)) waited_ok = false;
+          phase ^= 1u;
+        }
+        const int row0 = c * BR;
+        const int rows = min(BR, si.n - row0);
+        const int bh = b * p.Hkv + h;
+        // gate values: a whole number of 16-byte units, inside the [cap] row (cap % 4 == 0)
+        const uint32_t lg_bytes = gated ? (uint32_t)((rows + 3) & ~3) * 4u : 0u;
+        unsigned char* dst = S.ring[slot];
+        mbar_arrive_expect_tx(&S.full[slot], (uint32_t)rows * Gm::ROW_BYTES + lg_bytes);
+        if (!p.paged) {
+          bulk_g2s(dst, kp + ((size_t)bh * p.cap + row0) * Gm::ROW_BYTES, (uint32_t)rows * Gm::ROW_BYTES,
+                   &S.full[slot]);
+        } else {
+          const int32_t* pt = p.page_table + (size_t)b * p.max_pages;
+          for (int g = row0; g < row0 + rows;) {
+            const int pr = min(64 - (g & 63), row0 + rows - g);  // rows in this page piece
+            int pg = pt[g >> 6];
+            if (pg < 0 || pg >= p.num_pages) {
+              record_error(p.err, kDevBadPage, (uint32_t)b);
+              pg = 0;
+            }
+            bulk_g2s(dst + (size_t)(g - row0) * Gm::ROW_BYTES,
+                     kp + (((size_t)pg * p.Hkv + h) * 64 + (g & 63)) * Gm::ROW_BYTES, (uint32_t)pr * Gm::ROW_BYTES,
+                     &S.full[slot]);
+            g += pr;
+          }
+        }
+        if (gated) bulk_g2s(dst + kBlockBytes, p.log_g + (size_t)bh * p.cap + row0, lg_bytes, &S.full[slot]);
+        advance(kSlots);
+      }
+      if (!waited_ok) record_error(p.err, kDevWaitTimeout, blockIdx.x);
     }
-#pragma unroll
-    for (int o = TPR / 2; o; o >>= 1) sp += __shfl_xor_sync(0xffffffffu, sp, o);
-    if (qpart == 0) qhat[qj] = sp * p.sigma;
+    return;
   }
-  __syncthreads();
 
-  // This lane's 8 channels of every row it loads: chunk `part` of the row.
-  const int part = lane % LPR;
-  const int rsub = lane / LPR;
-  float2 qv[4];
-#pragma unroll
-  for (int e = 0; e < 4; ++e) qv[e] = make_float2(qhat[part * 8 + 2 * e], qhat[part * 8 + 2 * e + 1]);
-
-  const uint64_t pol_stream = policy_evict_first();
+  // ------------------------------------------------------------------ consumers
   const uint64_t pol_keep = policy_evict_last();
-  const bool gated = p.log_g != nullptr;
-  const size_t key_base = (size_t)bh * p.cap;
+  const int part = lane % Gm::LPR;  // this lane's 16-byte chunk of each row it loads
+  const int rsub = lane / Gm::LPR;  // its row within each load instruction
+  float2 qv[4];
+  int cur_bh = -1;
+  bool cur_ranked = false;
 
-  // Address of row `pos` of this (b, h) in the projected cache.
-  auto row_ptr = [&](int pos) -> const unsigned char* {
-    size_t row;
-    if (p.paged) {
-      row = ((size_t)pages_s[(pos - r0) >> 6] * p.Hkv + h) * 64 + (pos & 63);
-    } else {
-      row = (size_t)bh * p.cap + pos;
+  int b = pl.b0, h = pl.h0, c = pl.c0;
+  SeqInfo si = seq_info<BR>(p, b < p.B ? b : 0, false);
+  int t = 0;  // blocks of the CTA before the current head segment
+  while (t < pl.count) {
+    const int seg = min(si.blocks - c, pl.count - t);  // blocks of this head in the share
+    const int bh = b * p.Hkv + h;
+    // ---- new head (every consumer warp, whether or not it gets blocks of it) ----
+    {
+      constexpr int TPR = kConsumers / R;
+      constexpr int CH = D / TPR;
+      const int qj = tid / TPR, qpart = tid % TPR;
+      float mreg[CH];
+      const float* Mrow = p.M + ((size_t)h * R + qj) * D + qpart * CH;
+#pragma unroll
+      for (int i = 0; i < CH; ++i) mreg[i] = Mrow[i];
+      consumers_sync();  // every warp is done with the previous head's rows
+      if (cur_bh >= 0) {
+        uint32_t* gh = p.hist + (size_t)cur_bh * kHistBins;
+        for (int i = tid; i < kHistBins; i += kConsumers) {
+          const uint32_t v = S.hist[i];
+          if (v) {
+            if (cur_ranked) atomicAdd(&gh[i], v);
+            S.hist[i] = 0u;
+          }
+        }
+      }
+      if (tid < D) {
+        const __nv_bfloat16* qg = p.q + ((size_t)b * p.Hq + (size_t)h * p.G) * D + tid;
+        float sq = 0.f;
+        for (int g = 0; g < p.G; ++g) sq += __bfloat162float(qg[(size_t)g * D]);
+        S.qbar[tid] = sq / (float)p.G;
+      }
+      consumers_sync();
+      float sp = 0.f;
+#pragma unroll
+      for (int i = 0; i < CH; ++i) sp = fmaf(mreg[i], S.qbar[qpart * CH + i], sp);
+#pragma unroll
+      for (int o = TPR / 2; o; o >>= 1) sp += __shfl_xor_sync(0xffffffffu, sp, o);
+      if (qpart == 0) S.qhat[qj] = sp * p.sigma;
+      consumers_sync();
+#pragma unroll
+      for (int e = 0; e < 4; ++e) qv[e] = make_float2(S.qhat[part * 8 + 2 * e], S.qhat[part * 8 + 2 * e + 1]);
+      cur_bh = bh;
+      cur_ranked = si.ranked;
     }
-    return reinterpret_cast<const unsigned char*>(p.kproj + row * R);
-  };
 
-  const int nbatch = (r1 - r0 + kBatch - 1) / kBatch;
-  // Batch t of this warp covers rows r0 + (warp + t*kWarps) * 32 .. +31.
-  auto load = [&](int t, uint4* buf) {
-    const int base = r0 + (warp + t * kWarps) * kBatch;
+    // ---- this warp's blocks of the segment: CTA block indices j = t.. with j % 16 == warp ----
+    for (int j = t + ((warp - t) % kConsumerWarps + kConsumerWarps) % kConsumerWarps; j < t + seg;
+         j += kConsumerWarps) {
+      const int slot = j % kSlots;
+      if (!mbar_wait_bounded(&S.full[slot], (uint32_t)(j / kSlots) & 1u)) waited_ok = false;
+      const int row0 = (c + (j - t)) * BR;
+      const int rows = min(BR, si.n - row0);
+      const unsigned char* st = S.ring[slot];
+      const float* lgs = reinterpret_cast<const float*>(st + kBlockBytes);
+      if (rows == BR) {
+        // full block: every row valid, no per-row tests
 #pragma unroll
-    for (int i = 0; i < NI; ++i) {
-      const int pos = base + i * RPI + rsub;
-      if (pos < r1) buf[i] = ldg_hint(row_ptr(pos) + part * 16, pol_stream);
-      else buf[i] = make_uint4(0u, 0u, 0u, 0u);
+        for (int bt = 0; bt < Gm::NB; ++bt) {
+          const unsigned char* sb = st + (size_t)bt * 32 * Gm::ROW_BYTES;
+          float v[Gm::NI];
+#pragma unroll
+          for (int i = 0; i < Gm::NI; ++i) {
+            const uint4 w = *reinterpret_cast<const uint4*>(sb + (size_t)(i * Gm::RPI + rsub) * Gm::ROW_BYTES + part * 16);
+            v[i] = dot8(qv, w);
+          }
+          const float u0 = butterfly<Gm>(v, lane);
+          const int lr = part * Gm::RPI + rsub;
+          const float u = GATED ? fmaf(p.lam, lgs[bt * 32 + lr], u0) : u0;
+          const uint32_t key = float_key(u);
+          const size_t kidx = (size_t)bh * p.cap + row0 + bt * 32 + lr;
+          stg_hint(p.keys + kidx, key, pol_keep);
+          if (scores) p.scores_out[kidx] = u;
+          if (cur_ranked) atomicAdd(&S.hist[key >> kHistShift], 1u);
+        }
+      } else {
+#pragma unroll
+        for (int bt = 0; bt < Gm::NB; ++bt) {
+          const int wrows = rows - bt * 32;  // rows of this 32-row batch
+          if (wrows > 0) {
+            const unsigned char* sb = st + (size_t)bt * 32 * Gm::ROW_BYTES;
+            float v[Gm::NI];
+#pragma unroll
+            for (int i = 0; i < Gm::NI; ++i) {
+              const int lr = i * Gm::RPI + rsub;
+              uint4 w = make_uint4(0u, 0u, 0u, 0u);
+              if (lr < wrows) w = *reinterpret_cast<const uint4*>(sb + (size_t)lr * Gm::ROW_BYTES + part * 16);
+              v[i] = dot8(qv, w);
+            }
+            const float u0 = butterfly<Gm>(v, lane);
+            const int lr = part * Gm::RPI + rsub;
+            if (lr < wrows) {
+              const float u = GATED ? fmaf(p.lam, lgs[bt * 32 + lr], u0) : u0;
+              const uint32_t key = float_key(u);
+              const size_t kidx = (size_t)bh * p.cap + row0 + bt * 32 + lr;
+              stg_hint(p.keys + kidx, key, pol_keep);
+              if (scores) p.scores_out[kidx] = u;
+              if (cur_ranked) atomicAdd(&S.hist[key >> kHistShift], 1u);
+            }
+          }
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&S.empty[slot]);
     }
-  };
 
-  const int my_batches = nbatch > warp ? (nbatch - warp + kWarps - 1) / kWarps : 0;
-  uint4 cur[NI];
-#pragma unroll
-  for (int i = 0; i < NI; ++i) cur[i] = make_uint4(0u, 0u, 0u, 0u);
-  if (my_batches > 0) load(0, cur);
-  for (int t = 0; t < my_batches; ++t) {
-    // every element of the prefetch buffer is written on every path (no read of an
-    // uninitialised value on a warp's last batch)
-    uint4 nxt[NI];
-    if (t + 1 < my_batches) {
-      load(t + 1, nxt);
-    } else {
-#pragma unroll
-      for (int i = 0; i < NI; ++i) nxt[i] = make_uint4(0u, 0u, 0u, 0u);
+    // ---- next head ----
+    t += seg;
+    c = 0;
+    if (++h == p.Hkv) {
+      h = 0;
+      ++b;
+      next_scored_seq<BR>(p, b, si);
     }
-    const int base = r0 + (warp + t * kWarps) * kBatch;
-    // scores of rows base + i*RPI + rsub, reduced over the LPR lanes of each row
-    float sc[NI];
-#pragma unroll
-    for (int i = 0; i < NI; ++i) {
-      const uint4 w = cur[i];
-      float2 a = ffma2(qv[0], make_float2(bf16lo(w.x), bf16hi(w.x)), make_float2(0.f, 0.f));
-      a = ffma2(qv[1], make_float2(bf16lo(w.y), bf16hi(w.y)), a);
-      a = ffma2(qv[2], make_float2(bf16lo(w.z), bf16hi(w.z)), a);
-      a = ffma2(qv[3], make_float2(bf16lo(w.w), bf16hi(w.w)), a);
-      float s = a.x + a.y;
-#pragma unroll
-      for (int o = 1; o < LPR; o <<= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-      sc[i] = s;
-    }
-    // lane j takes row base + j: instruction j / RPI, row slot j % RPI (held by lane slot*LPR)
-    float u = 0.f;
-#pragma unroll
-    for (int i = 0; i < NI; ++i) {
-      const float v = __shfl_sync(0xffffffffu, sc[i], (lane % RPI) * LPR);
-      if (lane / RPI == i) u = v;
-    }
-    const int pos = base + lane;
-    const bool valid = pos < r1;
-    if (valid && gated) u = fmaf(p.lam, p.log_g[key_base + pos], u);
-    const uint32_t key = float_key(u);
-    if (valid) {
-      stg_hint(p.keys + key_base + pos, key, pol_keep);
-      if (p.scores_out != nullptr) p.scores_out[key_base + pos] = u;
-    }
-    hist_add(hist, key >> 21, valid);
-#pragma unroll
-    for (int i = 0; i < NI; ++i) cur[i] = nxt[i];
   }
-  __syncthreads();
-  if (need_hist) {
-    uint32_t* gh = p.hist + (size_t)bh * kBins;
-    for (int i = tid; i < kBins; i += kThreads) {
-      const uint32_t v = hist[i];
-      if (v) atomicAdd(&gh[i], v);
+  if (cur_bh >= 0) {
+    consumers_sync();
+    uint32_t* gh = p.hist + (size_t)cur_bh * kHistBins;
+    for (int i = tid; i < kHistBins; i += kConsumers) {
+      const uint32_t v = S.hist[i];
+      if (v && cur_ranked) atomicAdd(&gh[i], v);
     }
   }
-  }  // !skip
+  if (!waited_ok) record_error(p.err, kDevWaitTimeout, blockIdx.x);
 }
 
 template <int R, int D>
 cudaError_t launch_rd(const ScoreParams& p, cudaStream_t stream) {
-  dim3 grid((unsigned)((p.cap + p.rows_per_cta - 1) / p.rows_per_cta), (unsigned)(p.B * p.Hkv), 1);
-  score_kernel<R, D><<<grid, kThreads, 0, stream>>>(p);
+  const int smem = (int)sizeof(Smem<R, D>);
+  auto kern = p.log_g != nullptr ? score_kernel<R, D, true> : score_kernel<R, D, false>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  kern<<<p.ctas, kThreads, smem, stream>>>(p);
   return cudaGetLastError();
 }
 
 }  // namespace
 
 void plan_score(ScoreParams& p, int num_sms) {
-  // About four waves of four CTAs per SM; a whole number of warp batches per CTA.
-  const long rows = (long)p.B * p.Hkv * p.cap;
-  long per = rows / (16L * num_sms);
-  const long unit = (long)kWarps * kBatch;
-  per = (per + unit - 1) / unit * unit;
-  if (per < 4 * unit) per = 4 * unit;
-  if (per > kMaxRowsPerCta) per = kMaxRowsPerCta;
-  p.rows_per_cta = (int)per;
+  // Persistent: one CTA per SM, never more CTAs than there can be blocks.
+  const int br = kBlockBytes / (2 * p.r);
+  const long long blocks = (long long)p.B * p.Hkv * ((p.cap + br - 1) / br);
+  long long ctas = num_sms;
+  if (ctas > blocks) ctas = blocks;
+  p.ctas = (int)(ctas < 1 ? 1 : ctas);
 }
 
 cudaError_t launch_score(const ScoreParams& p, cudaStream_t stream) {

@@ -3,20 +3,21 @@
 // JSSA page, section JSSA 的整体结构 / Figure 1: every KV head keeps the positions of its k
 // largest projected scores, and its G query heads share them; section 局限与需要留意的地方:
 // no sink or recent window is forced.  The score kernel has left each (b, h)'s order-preserving
-// uint32 keys in the workspace (in L2) with a histogram of their top 11 bits.
+// uint32 keys in the workspace (in L2) with a histogram of their first 13 bits.
 //
 // A cluster of C CTAs serves one (b, h) (C = 1 when there are enough heads to fill the GPU);
-// each CTA owns a contiguous chunk of positions and reads its keys from L2 twice:
-//   1. the histogram gives the first 11-bit digit of the k-th largest key; the chunk is read
-//      once, counting keys above that digit and keeping the keys equal to it (candidates) in
-//      shared memory;
-//   2. the remaining 11- and 10-bit digits come from histograms of the candidates only,
-//      combined over the cluster through distributed shared memory (one cluster barrier per
-//      digit); a digit whose bin holds exactly the remaining count ends the search;
-//   3. the chunk is read again in tiles: positions with a larger key are selected, and of those
-//      equal to the threshold key the lowest positions fill the remainder (exact ties -> lower
-//      position); block-wide prefix sums per tile and a cluster-wide prefix of the CTA totals
-//      give every position its output slot, so the index list comes out ascending, unsorted.
+// each CTA owns a contiguous chunk of positions.  The k-th largest key T is found as three radix
+// digits (13, 10 and 9 bits); ties on T go to the lower positions.
+//   1. The global histogram gives digit 1.  Each CTA streams its chunk of keys once through a
+//      shared-memory ring (bulk copies), setting a position bitmap of the keys whose digit 1 is
+//      larger (they are selected) and appending the keys whose digit 1 equals it (the
+//      candidates, a few percent of the positions) to a list.
+//   2. The candidate lists are gathered into CTA 0 of the cluster through distributed shared
+//      memory; CTA 0 finds digits 2 and 3 among them, resolves the ties, marks the chosen
+//      candidates in the owners' bitmaps and hands every CTA its first output slot.
+//   3. Each CTA writes the set bits of its bitmap, in order, as ascending positions.
+// When the candidates do not fit the list, or many keys tie on T, every CTA re-reads its keys
+// instead (a slower path with the same result).
 #include <cooperative_groups.h>
 
 #include "sas_device.cuh"
@@ -29,28 +30,45 @@ namespace {
 
 constexpr int kThreads = 512;
 constexpr int kWarps = kThreads / 32;
-constexpr int kBins = 2048;          // 11-bit digits
-constexpr int kStep = 16;            // keys per thread per step (four 16-byte loads)
-constexpr int kMaxRun = 256;         // keys per thread at most (the plan sizes clusters for it)
-constexpr int kWords = kMaxRun / 32; // per-thread position bitmask words
-constexpr int kOwnCand = 16;         // candidate keys kept on chip per thread
-
-struct Ctl {
-  uint32_t cnt1, cnt2, gt0, pad;
-  uint32_t cta_gt, cta_eq, gt_before, eq_before;
-};
+constexpr int kBins2 = 1 << kDigit2Bits;      // 1024
+constexpr int kBins3 = 1 << kDigit3Bits;      // 512
+constexpr int kStageKeys = kWarps * 256;      // keys per ring stage: 8 per lane
+constexpr int kStages = 4;
+constexpr int kChunkMax = 131072;             // positions per CTA at most
+constexpr int kMaxWords = kChunkMax / 32;     // bitmap words per CTA
+constexpr int kCap = 4096;                    // candidate list entries (CTA 0: the whole head's)
+constexpr int kMaxTies = 256;                 // ties on T resolved by CTA 0; more take the slow path
+constexpr uint32_t kFast = 1u, kSlow = 2u;
 
 struct Found {
   uint32_t digit, above, eq, pad;
 };
 
+struct Ctl {
+  uint32_t ccount;   // candidates appended to this CTA's list (CTA 0: gathered from the cluster)
+  uint32_t above;    // keys of this CTA above digit 1
+  uint32_t flag;     // written by CTA 0: kFast (base valid) or kSlow
+  uint32_t base;     // written by CTA 0: first output slot of this CTA
+  uint32_t ntie;
+  int32_t tie_cut;   // ties at positions <= tie_cut are taken
+  uint32_t pad[2];
+  uint32_t above_of[kMaxCluster];  // CTA 0: per-CTA counts
+  uint32_t sel_of[kMaxCluster];
+  uint32_t tie_of[kMaxCluster];
+};
+
 struct SelSmem {
-  uint32_t hl[kBins];        // this CTA's histogram
-  uint32_t gh1[kBins];       // rank 0: cluster histogram of digit 2
-  uint32_t gh2[kBins / 2];   // rank 0: cluster histogram of digit 3
-  uint32_t cand[kOwnCand][kThreads];  // per-thread candidate keys, in position order
+  uint32_t ring[kStages][kStageKeys];
+  uint32_t bm[kMaxWords];     // selected positions of the chunk
+  uint32_t ckey[kCap];        // candidate keys (slow path: tie bits per bitmap word)
+  int32_t cpos[kCap];         // candidate positions in the head
+  uint32_t hloc[kBins2];
+  uint32_t hacc2[kBins2];     // CTA 0, slow path: cluster histogram of digit 2
+  uint32_t hacc3[kBins3];     // CTA 0: histogram of digit 3
+  int32_t tpos[kMaxTies];
+  uint64_t full[kStages];
+  uint64_t empty[kStages];
   uint32_t wsum[kWarps];
-  unsigned long long wsum64[kWarps];
   Ctl ctl;
   Found found;
 };
@@ -78,75 +96,25 @@ __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t* wsum, 
   return off + x - v;
 }
 
-__device__ __forceinline__ uint32_t block_sum(uint32_t v, uint32_t* wsum) {
-  uint32_t tot;
-  block_excl_scan(v, wsum, &tot);
-  return tot;
-}
-
-// Exclusive prefix sum of 64-bit values over the block; *total receives the block sum.
-__device__ __forceinline__ unsigned long long block_excl_scan64(unsigned long long v, unsigned long long* wsum,
-                                                                unsigned long long* total) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  unsigned long long x = v;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const unsigned long long y = __shfl_up_sync(0xffffffffu, x, o);
-    if (lane >= o) x += y;
-  }
-  if (lane == 31) wsum[warp] = x;
-  __syncthreads();
-  unsigned long long off = 0, tot = 0;
-#pragma unroll
-  for (int w = 0; w < kWarps; ++w) {
-    const unsigned long long s = wsum[w];
-    off += (w < warp) ? s : 0ull;
-    tot += s;
-  }
-  __syncthreads();
-  *total = tot;
-  return off + x - v;
-}
-
-// Warp-aggregated shared-memory histogram increment (many lanes share few bins).
-__device__ __forceinline__ void hist_add(uint32_t* hist, uint32_t bin, bool active) {
-  const uint32_t act = __ballot_sync(0xffffffffu, active);
-  if (act == 0u) return;
-  if (active) {
-    const uint32_t peers = __match_any_sync(act, bin);
-    if ((__ffs(peers) - 1) == (int)(threadIdx.x & 31)) atomicAdd(&hist[bin], (uint32_t)__popc(peers));
-  }
-}
-
-// Appends `key` (where take is true) to list[] through a shared counter; warp-aggregated.
-__device__ __forceinline__ void list_append(uint32_t* list, uint32_t* counter, uint32_t cap, uint32_t key, bool take) {
-  const uint32_t m = __ballot_sync(0xffffffffu, take);
-  if (m == 0u) return;
-  const int lane = threadIdx.x & 31;
-  const int leader = __ffs(m) - 1;
-  uint32_t base = 0u;
-  if (lane == leader) base = atomicAdd(counter, (uint32_t)__popc(m));
-  base = __shfl_sync(0xffffffffu, base, leader);
-  if (take) {
-    const uint32_t pos = base + (uint32_t)__popc(m & ((1u << lane) - 1u));
-    if (pos < cap) list[pos] = key;
-  }
-}
-
-// Digit holding the k_rem-th largest key, from a histogram of `nb` = PER * kThreads bins, read
-// through a generic pointer (global memory or a cluster peer's shared memory).  Thread t covers
-// digits [nb - (t+1)*PER, nb - t*PER), highest first.  Every CTA of a cluster that runs this on
-// the same histogram gets the same answer.
+// Digit holding the k_rem-th largest key, from a histogram of PER * kThreads bins read through
+// a generic pointer (this CTA's shared memory, CTA 0's through the cluster, or global memory).
+// Thread t covers digits [nb - (t+1)*PER, nb - t*PER), highest first.  Writes *out (digit,
+// count above it, count in it); out is left unchanged if the histogram holds fewer keys.
 template <int PER>
 __device__ __forceinline__ void find_digit(const uint32_t* H, uint32_t k_rem, uint32_t* wsum, Found* out) {
   const int lo = PER * kThreads - ((int)threadIdx.x + 1) * PER;
   uint32_t c[PER];
-  if constexpr (PER == 4) {
-    const uint4 a = *reinterpret_cast<const uint4*>(H + lo);
-    c[0] = a.x; c[1] = a.y; c[2] = a.z; c[3] = a.w;
-  } else {
+  if constexpr (PER % 4 == 0) {
+#pragma unroll
+    for (int q = 0; q < PER / 4; ++q) {
+      const uint4 a = reinterpret_cast<const uint4*>(H + lo)[q];
+      c[4 * q] = a.x; c[4 * q + 1] = a.y; c[4 * q + 2] = a.z; c[4 * q + 3] = a.w;
+    }
+  } else if constexpr (PER == 2) {
     const uint2 a = *reinterpret_cast<const uint2*>(H + lo);
     c[0] = a.x; c[1] = a.y;
+  } else {
+    c[0] = H[lo];
   }
   uint32_t tsum = 0u;
 #pragma unroll
@@ -169,56 +137,48 @@ __device__ __forceinline__ void find_digit(const uint32_t* H, uint32_t k_rem, ui
   __syncthreads();
 }
 
-// Fire-and-forget add into the same shared-memory word of cluster CTA `rank`.
-__device__ __forceinline__ void red_add_cluster(const uint32_t* local, uint32_t rank, uint32_t v) {
+// ---- distributed shared memory (cluster) primitives ----
+__device__ __forceinline__ uint32_t dsmem_addr(const void* local, uint32_t rank) {
   uint32_t ra;
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"(smem_u32(local)), "r"(rank));
-  asm volatile("red.relaxed.cluster.shared::cluster.add.u32 [%0], %1;" ::"r"(ra), "r"(v) : "memory");
+  return ra;
+}
+__device__ __forceinline__ void dsmem_st(uint32_t addr, uint32_t v) {
+  asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+__device__ __forceinline__ uint32_t dsmem_ld(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+  return v;
+}
+__device__ __forceinline__ uint32_t dsmem_atomic_add(uint32_t addr, uint32_t v) {
+  uint32_t old;
+  asm volatile("atom.relaxed.cluster.shared::cluster.add.u32 %0, [%1], %2;" : "=r"(old) : "r"(addr), "r"(v) : "memory");
+  return old;
+}
+__device__ __forceinline__ void dsmem_red_add(uint32_t addr, uint32_t v) {
+  asm volatile("red.relaxed.cluster.shared::cluster.add.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+__device__ __forceinline__ void dsmem_red_or(uint32_t addr, uint32_t v) {
+  asm volatile("red.relaxed.cluster.shared::cluster.or.b32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+// Split cluster barrier: arrive (release) now, wait (acquire) later.
+__device__ __forceinline__ void cluster_arrive() { asm volatile("barrier.cluster.arrive.aligned;" ::: "memory"); }
+__device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.aligned;" ::: "memory"); }
+__device__ __forceinline__ void cluster_sync() {
+  cluster_arrive();
+  cluster_wait();
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
-// Step i of this thread's contiguous run: keys [base + 16 i, +16) of the chunk; positions past
-// the run or the chunk read as 0 (and are masked by the callers).  Cached loads: the four
-// 16-byte loads of a step share 32-byte sectors.
-__device__ __forceinline__ void load_step(const uint32_t* gk, int base, int end, int i, uint32_t (&k)[kStep]) {
-  const int li = base + i * kStep;
-  if (li + kStep <= end) {
-#pragma unroll
-    for (int v = 0; v < kStep / 4; ++v) {
-      const uint4 a = *reinterpret_cast<const uint4*>(gk + li + 4 * v);
-      k[4 * v + 0] = a.x; k[4 * v + 1] = a.y; k[4 * v + 2] = a.z; k[4 * v + 3] = a.w;
-    }
-  } else {
-#pragma unroll
-    for (int e = 0; e < kStep; ++e) k[e] = (li + e < end) ? gk[li + e] : 0u;
-  }
-}
-
-// Bit e of the result is set where positions base + e (e < 16) lie before `end`.
-__device__ __forceinline__ uint32_t valid_bits(int base, int end) {
-  const int n = end - base;
-  return n >= kStep ? 0xffffu : (n > 0 ? ((1u << n) - 1u) : 0u);
-}
-
-// Bitmasks of the keys k[e] with (k & mask) above / equal to `prefix`.
-__device__ __forceinline__ void step_masks(const uint32_t (&k)[kStep], uint32_t mask, uint32_t prefix,
-                                           uint32_t& above, uint32_t& equal) {
-  above = 0u;
-  equal = 0u;
-#pragma unroll
-  for (int e = 0; e < kStep; ++e) {
-    const uint32_t m = k[e] & mask;
-    above |= (m > prefix ? 1u : 0u) << e;
-    equal |= (m == prefix ? 1u : 0u) << e;
-  }
-}
-
-__global__ void __launch_bounds__(kThreads, 2) select_topk_kernel(const SelectParams p) {
+__global__ void __launch_bounds__(kThreads, 1) select_topk_kernel(const SelectParams p) {
   extern __shared__ __align__(128) unsigned char smem_raw[];
   SelSmem& S = *reinterpret_cast<SelSmem*>(smem_raw);
-  cg::cluster_group cluster = cg::this_cluster();
-  const int rank = (int)cluster.block_rank();
-  const int C = (int)cluster.num_blocks();
-  const int tid = threadIdx.x;
+  const uint32_t rank = cg::this_cluster().block_rank();
+  const int C = (int)cg::this_cluster().num_blocks();
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int bh = blockIdx.y;
   const int b = bh / p.Hkv;
 
@@ -228,265 +188,337 @@ __global__ void __launch_bounds__(kThreads, 2) select_topk_kernel(const SelectPa
   const SeqSelection sel = seq_selection(min(p.kvec[b], p.k_max), n);
   const int k_eff = sel.k_eff;
   int32_t* idx = p.idx_out + (size_t)bh * p.k_max;
-  // Nothing to rank: empty selection, or every position selected (uniform per cluster).
-  // The exits are one guard around the body, not early returns.
-  const bool trivial = !sel.ranked;
 
-  // this CTA's positions [c0, c1); each thread owns a contiguous run of K of them
-  const int chunk_b = (((n + C - 1) / C) + 15) & ~15;
-  const int c0 = min(rank * chunk_b, n);
-  const int c1 = min(c0 + chunk_b, n);
+  // this CTA's positions [c0, c1); chunks are whole bitmap words
+  const int chunk = (((n + C - 1) / C) + 31) & ~31;
+  const int c0 = min((int)rank * chunk, n);
+  const int c1 = min(c0 + chunk, n);
   const int len = c1 - c0;
   const uint32_t* gk = p.keys + (size_t)bh * p.cap + c0;
-  const int K = ((len + kThreads - 1) / kThreads + kStep - 1) / kStep * kStep;
-  const int my0 = min(tid * K, len);
-  const int my1 = min(my0 + K, len);
-  const int nsteps = (my1 - my0 + kStep - 1) / kStep;
-  const int lane = tid & 31, warp = tid >> 5;
+  const int nwords = (len + 31) >> 5;
+  const int wpt = (nwords + kThreads - 1) / kThreads;  // bitmap words per thread (<= 8)
+  const int w0 = min(tid * wpt, nwords), w1 = min(w0 + wpt, nwords);
 
-  if (trivial) {
-    for (int j = rank * kThreads + tid; j < p.k_max; j += C * kThreads) idx[j] = (j < k_eff) ? j : -1;
-  } else {
-    // Bring the whole chunk of keys towards the SM early: the L2 fetches them from DRAM in
-    // large runs while the digit search below runs.
-    if (warp == 0) {
-      const int bytes = ((len * 4) + 15) & ~15;
-      for (int o = lane * 8192; o < bytes; o += 32 * 8192)
-        bulk_prefetch_l2(reinterpret_cast<const unsigned char*>(gk) + o, (uint32_t)min(8192, bytes - o));
-    }
-    for (int i = tid; i < kBins + kBins + kBins / 2; i += kThreads) S.hl[i] = 0u;  // hl, gh1, gh2
-    // ---- digit 1 from the global histogram ----
-    const uint32_t* ghist = p.hist + (size_t)bh * kBins;
-    uint32_t k_rem = (uint32_t)k_eff;
-    find_digit<4>(ghist, k_rem, S.wsum, &S.found);
-    const uint32_t d0 = S.found.digit;
-    uint32_t prefix = d0 << 21;
-    uint32_t mask = 0x7ffu << 21;
-    k_rem -= S.found.above;
-    bool done = (S.found.eq == k_rem);
-    const bool done1 = done;
-
-    // ---- the one read of my run: bitmasks of the keys above digit 1 (gtm) and equal to it
-    // (cm); the equal ones (candidates) are also kept, in position order, in my slot ----
-    uint32_t gtm[kWords], cm[kWords];
-#pragma unroll
-    for (int w = 0; w < kWords; ++w) {
-      gtm[w] = 0u;
-      cm[w] = 0u;
-    }
-    uint32_t nc = 0u;  // my candidates (beyond kOwnCand: keys re-read when needed)
-    for (int i = 0; i < nsteps; ++i) {
-      uint32_t k[kStep];
-      load_step(gk, my0, my1, i, k);
-      uint32_t sg, sc;
-      step_masks(k, 0x7ffu << 21, d0 << 21, sg, sc);
-      const uint32_t vb = valid_bits(my0 + i * kStep, my1);
-      sg &= vb;
-      sc &= vb;
-      const int sh = (i & 1) * kStep;
-#pragma unroll
-      for (int w = 0; w < kWords; ++w) {
-        if (w == (i >> 1)) {
-          gtm[w] |= sg << sh;
-          cm[w] |= sc << sh;
-        }
-      }
-      if (sc != 0u && !done) {
-#pragma unroll
-        for (int e = 0; e < kStep; ++e) {
-          if ((sc >> e) & 1u) {
-            if (nc < (uint32_t)kOwnCand) S.cand[nc][tid] = k[e];
-            ++nc;
-          }
-        }
-      }
-    }
-    const bool own_ovf = nc > (uint32_t)kOwnCand;
-    const uint32_t nown = min(nc, (uint32_t)kOwnCand);
-    __syncthreads();
-    // Every CTA has read the global histogram and zeroed its cluster histograms: after this
-    // barrier rank 0 clears the global histogram for the next call, and the adds may start.
-    if (C > 1) cluster.sync();
-    if (rank == 0)
-      for (int i = tid; i < kBins; i += kThreads) const_cast<uint32_t*>(ghist)[i] = 0u;
-
-    // Histogram of digit `shift` (11 bits at 10, or 10 bits at 0) of my candidates that match
-    // the current prefix, into hl: from my slot, or by re-reading my run when it overflowed.
-    auto cand_hist = [&](int shift, uint32_t dmask) {
-#pragma unroll
-      for (int j = 0; j < kOwnCand; ++j) {
-        const uint32_t key = S.cand[j][tid];
-        const bool act = !own_ovf && (uint32_t)j < nown && (key & mask) == prefix;
-        hist_add(S.hl, (key >> shift) & dmask, act);
-      }
-      if (own_ovf) {
-        for (int i = 0; i < nsteps; ++i) {
-          uint32_t k[kStep];
-          load_step(gk, my0, my1, i, k);
-          const int li = my0 + i * kStep;
-#pragma unroll
-          for (int e = 0; e < kStep; ++e)
-            if (li + e < my1 && (k[e] & mask) == prefix) atomicAdd(&S.hl[(k[e] >> shift) & dmask], 1u);
-        }
-      }
-    };
-
-    // ---- digit 2 ----
-    if (!done) {
-      cand_hist(10, 0x7ffu);
-      __syncthreads();
-      const uint32_t* gh1 = S.hl;
-      if (C > 1) {
-        for (int i = tid; i < kBins; i += kThreads) {
-          const uint32_t v = S.hl[i];
-          if (v) red_add_cluster(S.gh1 + i, 0, v);
-        }
-        cluster.sync();
-        gh1 = cluster.map_shared_rank(S.gh1, 0);
-      }
-      find_digit<4>(gh1, k_rem, S.wsum, &S.found);
-      prefix |= S.found.digit << 10;
-      mask |= 0x7ffu << 10;
-      k_rem -= S.found.above;
-      done = (S.found.eq == k_rem);
-    }
-    // ---- digit 3 ----
-    if (!done) {
-      for (int i = tid; i < kBins / 2; i += kThreads) S.hl[i] = 0u;
-      __syncthreads();
-      cand_hist(0, 0x3ffu);
-      __syncthreads();
-      const uint32_t* gh2 = S.hl;
-      if (C > 1) {
-        for (int i = tid; i < kBins / 2; i += kThreads) {
-          const uint32_t v = S.hl[i];
-          if (v) red_add_cluster(S.gh2 + i, 0, v);
-        }
-        cluster.sync();
-        gh2 = cluster.map_shared_rank(S.gh2, 0);
-      }
-      find_digit<2>(gh2, k_rem, S.wsum, &S.found);
-      prefix |= S.found.digit;
-      mask = 0xffffffffu;
-      k_rem -= S.found.above;
-    }
-    const uint32_t need = k_rem;  // how many of the threshold-key positions to take
-
-    // The key of my j-th candidate (position order), from my slot or from memory.
-    auto own_key = [&](uint32_t j, int pos_in_chunk) -> uint32_t {
-      return own_ovf ? gk[pos_in_chunk] : S.cand[j][tid];
-    };
-
-    // ---- my counts above / equal to the threshold ----
-    uint32_t my_gt = 0u, my_eq = 0u;
-#pragma unroll
-    for (int w = 0; w < kWords; ++w) {
-      my_gt += (uint32_t)__popc(gtm[w]);
-      my_eq += (uint32_t)__popc(cm[w]);
-    }
-    if (!done1) {
-      // the candidates split by their full keys
-      uint32_t cgt = 0u, ceq = 0u, j = 0u;
-#pragma unroll
-      for (int w = 0; w < kWords; ++w) {
-        uint32_t bits = cm[w];
-        while (bits) {
-          const int bpos = __ffs(bits) - 1;
-          bits &= bits - 1u;
-          const uint32_t m = own_key(j, my0 + w * 32 + bpos) & mask;
-          ++j;
-          cgt += (m > prefix) ? 1u : 0u;
-          ceq += (m == prefix) ? 1u : 0u;
-        }
-      }
-      my_gt += cgt;
-      my_eq = ceq;
-    }
-    unsigned long long tot;
-    const unsigned long long ex =
-        block_excl_scan64(((unsigned long long)my_gt << 32) | my_eq, S.wsum64, &tot);
-    if (tid == 0) {
-      S.ctl.cta_gt = (uint32_t)(tot >> 32);
-      S.ctl.cta_eq = (uint32_t)tot;
-    }
-    uint32_t gt_base = 0u, eq_base = 0u;
-    if (C > 1) {
-      cluster.sync();
-      if (tid < 32) {
-        uint32_t gb = 0u, eb = 0u;
-        if (tid < rank) {
-          const Ctl* rc = cluster.map_shared_rank(&S.ctl, tid);
-          gb = rc->cta_gt;
-          eb = rc->cta_eq;
-        }
-#pragma unroll
-        for (int o = 16; o; o >>= 1) {
-          gb += __shfl_xor_sync(0xffffffffu, gb, o);
-          eb += __shfl_xor_sync(0xffffffffu, eb, o);
-        }
-        if (tid == 0) {
-          S.ctl.gt_before = gb;
-          S.ctl.eq_before = eb;
-        }
-      }
-      __syncthreads();
-      gt_base = S.ctl.gt_before;
-      eq_base = S.ctl.eq_before;
-    }
-
-    // ---- write my selected positions in order (no further reads unless my slot overflowed) ----
-    {
-      uint32_t gc = gt_base + (uint32_t)(ex >> 32);
-      uint32_t ec = eq_base + (uint32_t)ex;
-      uint32_t j = 0u;
-#pragma unroll
-      for (int w = 0; w < kWords; ++w) {
-        uint32_t bits = gtm[w] | cm[w];
-        while (bits) {
-          const int bpos = __ffs(bits) - 1;
-          bits &= bits - 1u;
-          const int pic = my0 + w * 32 + bpos;  // position in the chunk
-          bool above, equal;
-          if ((gtm[w] >> bpos) & 1u) {
-            above = true;
-            equal = false;
-          } else if (done1) {
-            above = false;
-            equal = true;
-          } else {
-            const uint32_t m = own_key(j, pic) & mask;
-            above = m > prefix;
-            equal = m == prefix;
-          }
-          if (!((gtm[w] >> bpos) & 1u)) ++j;
-          if (above) {
-            idx[gc + min(ec, need)] = c0 + pic;
-            ++gc;
-          } else if (equal) {
-            if (ec < need) idx[gc + ec] = c0 + pic;
-            ++ec;
-          }
-        }
-      }
-    }
-    for (int j = k_eff + rank * kThreads + tid; j < p.k_max; j += C * kThreads) idx[j] = -1;
-    if (C > 1) cluster.sync();  // peers may still read this CTA's shared memory
+  if (!sel.ranked) {
+    // Nothing to rank (uniform over the cluster): the first k_eff positions, or none.
+    for (int j = (int)rank * kThreads + tid; j < p.k_max; j += C * kThreads) idx[j] = (j < k_eff) ? j : -1;
+    return;
   }
+
+  // ---------------------------------------------------------------- set-up
+  const int nst = (len + kStageKeys - 1) / kStageKeys;
+  if (tid == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&S.full[s], 1);
+      mbar_init(&S.empty[s], kWarps);
+    }
+    fence_barrier_init();
+  }
+  for (int i = tid; i < kMaxWords; i += kThreads) S.bm[i] = 0u;
+  for (int i = tid; i < kBins2; i += kThreads) {
+    S.hloc[i] = 0u;
+    S.hacc2[i] = 0u;
+  }
+  for (int i = tid; i < kBins3; i += kThreads) S.hacc3[i] = 0u;
+  if (tid == 0) {
+    Ctl z = {};
+    z.tie_cut = 0x7fffffff;
+    S.ctl = z;
+    Found f = {};
+    S.found = f;
+  }
+  __syncthreads();
+
+  // Stage s of the chunk: keys [s * kStageKeys, +kStageKeys) as whole 16-byte units (the key
+  // rows have a multiple of 4 entries, so the rounding stays inside this (b, h)'s row).
+  auto issue = [&](int s) {
+    const int slot = s % kStages;
+    const int keys = min(kStageKeys, len - s * kStageKeys);
+    const uint32_t bytes = (uint32_t)((keys + 3) & ~3) * 4u;
+    mbar_arrive_expect_tx(&S.full[slot], bytes);
+    bulk_g2s(S.ring[slot], gk + (size_t)s * kStageKeys, bytes, &S.full[slot]);
+  };
+  if (tid == 0)
+    for (int s = 0; s < min(kStages, nst); ++s) issue(s);
+
+  // ---- digit 1 from the global histogram ----
+  const uint32_t* ghist = p.hist + (size_t)bh * kHistBins;
+  find_digit<kHistBins / kThreads>(ghist, (uint32_t)k_eff, S.wsum, &S.found);
+  const uint32_t d1 = S.found.digit;
+  const uint32_t above1 = S.found.above;  // keys of the head with a larger digit 1
+  const uint32_t eq1 = S.found.eq;        // keys of the head with this digit 1: the candidates
+  const bool fast = eq1 <= (uint32_t)kCap;
+  cluster_arrive();  // this CTA's set-up is done and it has read the global histogram
+
+  bool waited_ok = true;
+  if (fast) {
+    // ------------------------------------------------------------ streaming pass
+    uint32_t my_above = 0u;
+    for (int s = 0; s < nst; ++s) {
+      const int slot = s % kStages;
+      if (!mbar_wait_bounded(&S.full[slot], (uint32_t)(s / kStages) & 1u)) waited_ok = false;
+      const uint32_t* st = S.ring[slot] + warp * 256;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const int lp = s * kStageKeys + warp * 256 + e * 32 + lane;  // position in the chunk
+        const bool valid = lp < len;
+        const uint32_t key = st[e * 32 + lane];
+        const uint32_t dg = key >> kHistShift;
+        const uint32_t ab = __ballot_sync(0xffffffffu, valid && dg > d1);
+        const uint32_t cb = __ballot_sync(0xffffffffu, valid && dg == d1);
+        if (lane == 0) {
+          S.bm[s * (kStageKeys / 32) + warp * 8 + e] = ab;
+          my_above += (uint32_t)__popc(ab);
+        }
+        if (cb) {
+          const int leader = __ffs(cb) - 1;
+          uint32_t base = 0u;
+          if (lane == leader) base = atomicAdd(&S.ctl.ccount, (uint32_t)__popc(cb));
+          base = __shfl_sync(0xffffffffu, base, leader);
+          if ((cb >> lane) & 1u) {
+            const uint32_t j = base + (uint32_t)__popc(cb & ((1u << lane) - 1u));
+            if (j < (uint32_t)kCap) {
+              S.ckey[j] = key;
+              S.cpos[j] = c0 + lp;
+            }
+          }
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&S.empty[slot]);
+      if (tid == 0 && s + kStages < nst) {
+        if (!mbar_wait_bounded(&S.empty[slot], (uint32_t)(s / kStages) & 1u)) waited_ok = false;
+        issue(s + kStages);
+      }
+    }
+    if (lane == 0 && my_above) atomicAdd(&S.ctl.above, my_above);
+    __syncthreads();
+    cluster_wait();  // every CTA of the cluster is set up: CTA 0's list may now be appended to
+
+    // ------------------------------------------------------------ gather into CTA 0
+    const uint32_t mine = min(S.ctl.ccount, (uint32_t)kCap);
+    if (rank != 0) {
+      if (tid == 0) {
+        const uint32_t base = dsmem_atomic_add(dsmem_addr(&S.ctl.ccount, 0), mine);
+        S.ctl.ntie = base;  // this CTA's first slot in CTA 0's list (ntie is free here)
+        dsmem_st(dsmem_addr(&S.ctl.above_of[rank], 0), S.ctl.above);
+      }
+      __syncthreads();
+      const uint32_t base = S.ctl.ntie;
+      for (uint32_t i = tid; i < mine; i += kThreads) {
+        if (base + i < (uint32_t)kCap) {
+          dsmem_st(dsmem_addr(&S.ckey[base + i], 0), S.ckey[i]);
+          dsmem_st(dsmem_addr(&S.cpos[base + i], 0), (uint32_t)S.cpos[i]);
+        }
+      }
+    } else if (tid == 0) {
+      S.ctl.above_of[0] = S.ctl.above;
+    }
+    cluster_sync();  // B: CTA 0 holds every candidate
+    if (rank == 0) {
+      for (int i = tid; i < kHistBins; i += kThreads) const_cast<uint32_t*>(ghist)[i] = 0u;  // for the next call
+      if (tid == 0) S.ctl.ntie = 0u;
+      __syncthreads();
+      // ---- CTA 0: digits 2 and 3 among the candidates, then the ties ----
+      const uint32_t total = S.ctl.ccount;
+      bool ok = total == eq1;  // every candidate arrived (else: slow path)
+      uint32_t k_rem = (uint32_t)k_eff - above1;
+      uint32_t T = 0u, need = 0u;
+      if (ok) {
+        for (uint32_t i = tid; i < total; i += kThreads)
+          atomicAdd(&S.hloc[(S.ckey[i] >> kDigit3Bits) & (kBins2 - 1)], 1u);
+        __syncthreads();
+        find_digit<kBins2 / kThreads>(S.hloc, k_rem, S.wsum, &S.found);
+        const uint32_t d2 = S.found.digit;
+        k_rem -= S.found.above;
+        const uint32_t pre = (d1 << kDigit2Bits) | d2;
+        for (uint32_t i = tid; i < total; i += kThreads)
+          if ((S.ckey[i] >> kDigit3Bits) == pre) atomicAdd(&S.hacc3[S.ckey[i] & (kBins3 - 1)], 1u);
+        __syncthreads();
+        find_digit<kBins3 / kThreads>(S.hacc3, k_rem, S.wsum, &S.found);
+        T = (pre << kDigit3Bits) | S.found.digit;
+        k_rem -= S.found.above;
+        need = k_rem;  // ties on T to take, 1 <= need <= eq
+        const uint32_t eq = S.found.eq;
+        if (need < eq) {
+          if (eq > (uint32_t)kMaxTies) {
+            ok = false;
+          } else {
+            // the need-th lowest position among the ties
+            for (uint32_t i = tid; i < total; i += kThreads)
+              if (S.ckey[i] == T) S.tpos[atomicAdd(&S.ctl.ntie, 1u)] = S.cpos[i];
+            __syncthreads();
+            for (uint32_t j = tid; j < eq; j += kThreads) {
+              const int pj = S.tpos[j];
+              uint32_t r = 0u;
+              for (uint32_t x = 0; x < eq; ++x) r += (S.tpos[x] < pj) ? 1u : 0u;
+              if (r == need - 1u) S.ctl.tie_cut = pj;
+            }
+          }
+        }
+        __syncthreads();
+      }
+      if (ok) {
+        // ---- mark the chosen candidates in their owners' bitmaps; count them per CTA ----
+        const int cut = S.ctl.tie_cut;
+        for (uint32_t i = tid; i < total; i += kThreads) {
+          const uint32_t key = S.ckey[i];
+          const int pos = S.cpos[i];
+          if (key > T || (key == T && pos <= cut)) {
+            const int owner = pos / chunk;
+            const int lp = pos - owner * chunk;
+            atomicAdd(&S.ctl.sel_of[owner], 1u);
+            dsmem_red_or(dsmem_addr(&S.bm[lp >> 5], (uint32_t)owner), 1u << (lp & 31));
+          }
+        }
+        __syncthreads();
+        if (tid < C) {
+          uint32_t base = 0u;
+          for (int c = 0; c < tid; ++c) base += S.ctl.above_of[c] + S.ctl.sel_of[c];
+          dsmem_st(dsmem_addr(&S.ctl.base, (uint32_t)tid), base);
+          dsmem_st(dsmem_addr(&S.ctl.flag, (uint32_t)tid), kFast);
+        }
+      } else if (tid < C) {
+        dsmem_st(dsmem_addr(&S.ctl.flag, (uint32_t)tid), kSlow);
+      }
+    }
+    cluster_sync();  // C: results are in every CTA
+  } else {
+    // Too many candidates for the list: drain the copies issued above, then take the slow path.
+    if (tid == 0)
+      for (int s = 0; s < min(kStages, nst); ++s)
+        if (!mbar_wait_bounded(&S.full[s], 0u)) waited_ok = false;
+    __syncthreads();
+    cluster_wait();
+    if (rank == 0)
+      for (int i = tid; i < kHistBins; i += kThreads) const_cast<uint32_t*>(ghist)[i] = 0u;
+    if (tid == 0) S.ctl.flag = kSlow;
+    __syncthreads();
+  }
+
+  uint32_t out_base;
+  if (S.ctl.flag == kFast) {
+    out_base = S.ctl.base;
+  } else {
+    // ------------------------------------------------------------ slow path: re-read the keys
+    for (int i = tid; i < kBins2; i += kThreads) {
+      S.hloc[i] = 0u;
+      S.hacc2[i] = 0u;
+    }
+    for (int i = tid; i < kBins3; i += kThreads) S.hacc3[i] = 0u;
+    if (tid == 0) S.found = Found{};
+    cluster_sync();  // every CTA's accumulators are clear before the adds
+    uint32_t k_rem = (uint32_t)k_eff - above1;
+    // digit 2
+    for (int i = tid; i < len; i += kThreads) {
+      const uint32_t key = gk[i];
+      if ((key >> kHistShift) == d1) atomicAdd(&S.hloc[(key >> kDigit3Bits) & (kBins2 - 1)], 1u);
+    }
+    __syncthreads();
+    for (int i = tid; i < kBins2; i += kThreads)
+      if (S.hloc[i]) dsmem_red_add(dsmem_addr(&S.hacc2[i], 0), S.hloc[i]);
+    cluster_sync();
+    find_digit<kBins2 / kThreads>(cg::this_cluster().map_shared_rank(S.hacc2, 0), k_rem, S.wsum, &S.found);
+    const uint32_t pre = (d1 << kDigit2Bits) | S.found.digit;
+    k_rem -= S.found.above;
+    // digit 3
+    for (int i = tid; i < kBins3; i += kThreads) S.hloc[i] = 0u;
+    __syncthreads();
+    for (int i = tid; i < len; i += kThreads) {
+      const uint32_t key = gk[i];
+      if ((key >> kDigit3Bits) == pre) atomicAdd(&S.hloc[key & (kBins3 - 1)], 1u);
+    }
+    __syncthreads();
+    for (int i = tid; i < kBins3; i += kThreads)
+      if (S.hloc[i]) dsmem_red_add(dsmem_addr(&S.hacc3[i], 0), S.hloc[i]);
+    cluster_sync();
+    find_digit<kBins3 / kThreads>(cg::this_cluster().map_shared_rank(S.hacc3, 0), k_rem, S.wsum, &S.found);
+    const uint32_t T = (pre << kDigit3Bits) | S.found.digit;
+    const uint32_t need = k_rem - S.found.above;
+    // bits above T and ties on T, word by word; counts per CTA
+    uint32_t n_above = 0u, n_tie = 0u;
+    for (int w = w0; w < w1; ++w) {
+      uint32_t ab = 0u, tb = 0u;
+      for (int e = 0; e < 32 && w * 32 + e < len; ++e) {
+        const uint32_t key = gk[w * 32 + e];
+        ab |= (key > T ? 1u : 0u) << e;
+        tb |= (key == T ? 1u : 0u) << e;
+      }
+      S.bm[w] = ab;
+      S.ckey[w] = tb;
+      n_above += (uint32_t)__popc(ab);
+      n_tie += (uint32_t)__popc(tb);
+    }
+    uint32_t tot_above, tot_tie;
+    const uint32_t tie_pre = block_excl_scan(n_tie, S.wsum, &tot_tie);
+    block_excl_scan(n_above, S.wsum, &tot_above);
+    if (tid == 0) {
+      dsmem_st(dsmem_addr(&S.ctl.above_of[rank], 0), tot_above);
+      dsmem_st(dsmem_addr(&S.ctl.tie_of[rank], 0), tot_tie);
+    }
+    cluster_sync();
+    if (tid == 0) {
+      uint32_t ties_before = 0u, base = 0u;
+      for (int c = 0; c < (int)rank; ++c) {
+        const uint32_t a = dsmem_ld(dsmem_addr(&S.ctl.above_of[c], 0));
+        const uint32_t t = dsmem_ld(dsmem_addr(&S.ctl.tie_of[c], 0));
+        const uint32_t taken = need > ties_before ? min(t, need - ties_before) : 0u;
+        base += a + taken;
+        ties_before += t;
+      }
+      S.ctl.base = base;
+      S.ctl.ntie = ties_before;
+    }
+    cluster_sync();  // every CTA has read CTA 0's counts
+    // take the ties in position order while the running tie rank is below need
+    uint32_t r = S.ctl.ntie + tie_pre;
+    for (int w = w0; w < w1; ++w) {
+      uint32_t tb = S.ckey[w], take = 0u;
+      while (tb) {
+        const int e = __ffs(tb) - 1;
+        tb &= tb - 1u;
+        if (r < need) take |= 1u << e;
+        ++r;
+      }
+      S.bm[w] |= take;
+    }
+    __syncthreads();
+    out_base = S.ctl.base;
+  }
+
+  // ---------------------------------------------------------------- ordered output
+  {
+    uint32_t cnt = 0u;
+    for (int w = w0; w < w1; ++w) cnt += (uint32_t)__popc(S.bm[w]);
+    uint32_t tot;
+    uint32_t o = out_base + block_excl_scan(cnt, S.wsum, &tot);
+    for (int w = w0; w < w1; ++w) {
+      uint32_t bits = S.bm[w];
+      while (bits) {
+        const int e = __ffs(bits) - 1;
+        bits &= bits - 1u;
+        if (o < (uint32_t)k_eff) idx[o] = c0 + w * 32 + e;
+        ++o;
+      }
+    }
+  }
+  for (int j = k_eff + (int)rank * kThreads + tid; j < p.k_max; j += C * kThreads) idx[j] = -1;
+  if (!waited_ok) record_error(p.err, kDevWaitTimeout, (uint32_t)bh);
 }
 
 }  // namespace
 
 bool plan_select(SelectParams& p, int num_sms) {
   const int heads = p.B * p.Hkv;
-  // Double the CTAs per head while the grid still fits one wave of two CTAs per SM and each
-  // CTA keeps at least one tile of keys.
+  // One CTA per SM.  Split a head over a cluster while its chunk is too long, and while the
+  // grid still leaves SMs idle (up to the portable cluster size).
   int C = 1;
-  while (C < kMaxCluster && (p.cap + C - 1) / C > kThreads * kMaxRun) C *= 2;
-  while (C < kMaxCluster && (long)heads * C * 2 <= 2L * num_sms && (p.cap + 2 * C - 1) / (2 * C) >= kThreads * kStep) C *= 2;
-  if ((p.cap + C - 1) / C > kThreads * kMaxRun) return false;
+  while (C < kMaxCluster && (p.cap + C - 1) / C > kChunkMax) C *= 2;
+  while (C < 8 && (long)heads * C * 2 <= (long)num_sms) C *= 2;
+  if ((p.cap + C - 1) / C > kChunkMax) return false;
   p.cluster = C;
-  p.chunk = (((p.cap + C - 1) / C) + 15) & ~15;
-  p.cand_cap = kThreads * kOwnCand;
+  p.chunk = (((p.cap + C - 1) / C) + 31) & ~31;
+  p.cand_cap = kCap;
   p.off_hist = 0;
   p.off_ctl = 0;
   p.smem_bytes = (int)sizeof(SelSmem);
