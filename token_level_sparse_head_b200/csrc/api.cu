@@ -4,10 +4,42 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <array>
 #include <mutex>
+#include <unordered_map>
 
 #include "sas.h"
 #include "sas_kernels.h"
+
+namespace sas {
+
+cudaError_t prepare_kernel(const void* kern, int smem_bytes, bool nonportable_cluster) {
+  constexpr int kDevices = 64;
+  static std::mutex mu;
+  static std::unordered_map<const void*, std::array<int, kDevices>> allowed;  // bytes allowed, per device
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lock(mu);
+  int* lim = nullptr;
+  if (dev >= 0 && dev < kDevices) {
+    auto it = allowed.find(kern);
+    if (it == allowed.end()) {
+      std::array<int, kDevices> none;
+      none.fill(-1);
+      it = allowed.emplace(kern, none).first;
+    }
+    lim = &it->second[dev];
+    if (*lim >= smem_bytes) return cudaSuccess;
+  }
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes);
+  if (e == cudaSuccess && nonportable_cluster)
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+  if (e == cudaSuccess && lim != nullptr) *lim = smem_bytes;
+  return e;
+}
+
+}  // namespace sas
 
 namespace {
 

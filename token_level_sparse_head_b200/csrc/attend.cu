@@ -459,7 +459,7 @@ __global__ void __launch_bounds__(kThreads) attend_kernel(const AttendParams p) 
 template <int D, int GT, bool GATED, bool PAGED, bool DENSE>
 cudaError_t launch_t(const AttendParams& p, cudaStream_t stream) {
   auto kern = attend_kernel<D, GT, GATED, PAGED, DENSE>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, p.smem_bytes);
+  cudaError_t e = prepare_kernel((const void*)kern, p.smem_bytes);
   if (e != cudaSuccess) return e;
   dim3 grid((unsigned)p.splits, (unsigned)(p.B * p.Hkv), (unsigned)p.ngz);
   kern<<<grid, kThreads, (size_t)p.smem_bytes, stream>>>(p);

@@ -161,7 +161,7 @@ cudaError_t launch_dr(const ProjParams& p, cudaStream_t stream) {
   }
   const size_t smem = (size_t)R * D * 4;
   auto kern = build_kernel<D, R>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  cudaError_t e = prepare_kernel((const void*)kern, (int)smem);
   if (e != cudaSuccess) return e;
   dim3 grid((unsigned)((p.cap + p.rows_per_cta - 1) / p.rows_per_cta), (unsigned)(p.B * p.Hkv), 1);
   kern<<<grid, kBuildThreads, smem, stream>>>(p);

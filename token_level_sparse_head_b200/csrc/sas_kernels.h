@@ -96,6 +96,10 @@ void plan_attend(AttendParams& p, int count_max);
 size_t attend_workspace_floats(const AttendParams& p);
 cudaError_t launch_attend(const AttendParams& p, cudaStream_t stream);
 
+// Raises a kernel's dynamic shared-memory limit (and allows non-portable cluster sizes) on the
+// current device once, not on every launch; thread-safe.
+cudaError_t prepare_kernel(const void* kern, int smem_bytes, bool nonportable_cluster = false);
+
 constexpr int kTargetCtas = 1024;   // attention split planning target (device independent)
 constexpr int kMaxSplitLen = 2048;  // index entries per attention CTA at most
 constexpr int kMaxChunk = 16384;    // positions per selection CTA at most

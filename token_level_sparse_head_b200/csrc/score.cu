@@ -421,7 +421,7 @@ template <int R, int D>
 cudaError_t launch_rd(const ScoreParams& p, cudaStream_t stream) {
   const int smem = (int)sizeof(Smem<R, D>);
   auto kern = p.log_g != nullptr ? score_kernel<R, D, true> : score_kernel<R, D, false>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  cudaError_t e = prepare_kernel((const void*)kern, smem);
   if (e != cudaSuccess) return e;
   kern<<<p.ctas, kThreads, smem, stream>>>(p);
   return cudaGetLastError();

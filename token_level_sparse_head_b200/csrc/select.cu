@@ -527,12 +527,8 @@ bool plan_select(SelectParams& p, int num_sms) {
 
 cudaError_t launch_select(const SelectParams& p, cudaStream_t stream) {
   auto kern = select_topk_kernel;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, p.smem_bytes);
+  const cudaError_t e = prepare_kernel((const void*)kern, p.smem_bytes, p.cluster > 8);
   if (e != cudaSuccess) return e;
-  if (p.cluster > 8) {
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-    if (e != cudaSuccess) return e;
-  }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)p.cluster, (unsigned)(p.B * p.Hkv), 1);
   cfg.blockDim = dim3(kThreads, 1, 1);
