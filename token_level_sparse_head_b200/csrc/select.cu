@@ -9,7 +9,7 @@
 // each CTA owns a contiguous chunk of positions.  The k-th largest key T is found as three radix
 // digits (13, 10 and 9 bits); ties on T go to the lower positions.
 //   1. The global histogram gives digit 1.  Each CTA streams its chunk of keys once through a
-//      shared-memory ring (bulk copies), setting a position bitmap of the keys whose digit 1 is
+//      shared-memory ring (bulk copies; one ballot per 32 keys is a bitmap word), setting a position bitmap of the keys whose digit 1 is
 //      larger (they are selected) and appending the keys whose digit 1 equals it (the
 //      candidates, a few percent of the positions) to a list.
 //   2. The candidate lists are gathered into CTA 0 of the cluster through distributed shared
@@ -28,12 +28,12 @@ namespace cg = cooperative_groups;
 namespace sas {
 namespace {
 
-constexpr int kThreads = 512;
+constexpr int kThreads = 1024;
 constexpr int kWarps = kThreads / 32;
 constexpr int kBins2 = 1 << kDigit2Bits;      // 1024
 constexpr int kBins3 = 1 << kDigit3Bits;      // 512
-constexpr int kStageKeys = kWarps * 256;      // keys per ring stage: 8 per lane
-constexpr int kStages = 4;
+constexpr int kStageKeys = kWarps * 128;      // keys per ring stage: 4 per lane
+constexpr int kStages = 8;
 constexpr int kChunkMax = 131072;             // positions per CTA at most
 constexpr int kMaxWords = kChunkMax / 32;     // bitmap words per CTA
 constexpr int kCap = 4096;                    // candidate list entries (CTA 0: the whole head's)
@@ -96,25 +96,32 @@ __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t* wsum, 
   return off + x - v;
 }
 
-// Digit holding the k_rem-th largest key, from a histogram of PER * kThreads bins read through
-// a generic pointer (this CTA's shared memory, CTA 0's through the cluster, or global memory).
-// Thread t covers digits [nb - (t+1)*PER, nb - t*PER), highest first.  Writes *out (digit,
-// count above it, count in it); out is left unchanged if the histogram holds fewer keys.
-template <int PER>
+// Digit holding the k_rem-th largest key, from a histogram of NB bins read through a generic
+// pointer (this CTA's shared memory, CTA 0's through the cluster, or global memory).  Thread t
+// covers digits [NB - (t+1)*PER, NB - t*PER), highest first (threads past NB / PER hold none).
+// Writes *out (digit, count above it, count in it); out is left unchanged if the histogram
+// holds fewer keys.
+template <int NB>
 __device__ __forceinline__ void find_digit(const uint32_t* H, uint32_t k_rem, uint32_t* wsum, Found* out) {
-  const int lo = PER * kThreads - ((int)threadIdx.x + 1) * PER;
+  constexpr int PER = NB >= kThreads ? NB / kThreads : 1;
+  constexpr int ACT = NB / PER;
+  const int lo = NB - ((int)threadIdx.x + 1) * PER;
   uint32_t c[PER];
-  if constexpr (PER % 4 == 0) {
 #pragma unroll
-    for (int q = 0; q < PER / 4; ++q) {
-      const uint4 a = reinterpret_cast<const uint4*>(H + lo)[q];
-      c[4 * q] = a.x; c[4 * q + 1] = a.y; c[4 * q + 2] = a.z; c[4 * q + 3] = a.w;
+  for (int j = 0; j < PER; ++j) c[j] = 0u;
+  if ((int)threadIdx.x < ACT) {
+    if constexpr (PER % 4 == 0) {
+#pragma unroll
+      for (int q = 0; q < PER / 4; ++q) {
+        const uint4 a = reinterpret_cast<const uint4*>(H + lo)[q];
+        c[4 * q] = a.x; c[4 * q + 1] = a.y; c[4 * q + 2] = a.z; c[4 * q + 3] = a.w;
+      }
+    } else if constexpr (PER == 2) {
+      const uint2 a = *reinterpret_cast<const uint2*>(H + lo);
+      c[0] = a.x; c[1] = a.y;
+    } else {
+      c[0] = H[lo];
     }
-  } else if constexpr (PER == 2) {
-    const uint2 a = *reinterpret_cast<const uint2*>(H + lo);
-    c[0] = a.x; c[1] = a.y;
-  } else {
-    c[0] = H[lo];
   }
   uint32_t tsum = 0u;
 #pragma unroll
@@ -196,7 +203,7 @@ __global__ void __launch_bounds__(kThreads, 1) select_topk_kernel(const SelectPa
   const int len = c1 - c0;
   const uint32_t* gk = p.keys + (size_t)bh * p.cap + c0;
   const int nwords = (len + 31) >> 5;
-  const int wpt = (nwords + kThreads - 1) / kThreads;  // bitmap words per thread (<= 8)
+  const int wpt = (nwords + kThreads - 1) / kThreads;  // bitmap words per thread (<= 4)
   const int w0 = min(tid * wpt, nwords), w1 = min(w0 + wpt, nwords);
 
   if (!sel.ranked) {
@@ -243,7 +250,7 @@ __global__ void __launch_bounds__(kThreads, 1) select_topk_kernel(const SelectPa
 
   // ---- digit 1 from the global histogram ----
   const uint32_t* ghist = p.hist + (size_t)bh * kHistBins;
-  find_digit<kHistBins / kThreads>(ghist, (uint32_t)k_eff, S.wsum, &S.found);
+  find_digit<kHistBins>(ghist, (uint32_t)k_eff, S.wsum, &S.found);
   const uint32_t d1 = S.found.digit;
   const uint32_t above1 = S.found.above;  // keys of the head with a larger digit 1
   const uint32_t eq1 = S.found.eq;        // keys of the head with this digit 1: the candidates
@@ -254,33 +261,33 @@ __global__ void __launch_bounds__(kThreads, 1) select_topk_kernel(const SelectPa
   if (fast) {
     // ------------------------------------------------------------ streaming pass
     uint32_t my_above = 0u;
+    // keys of digit d1 are [lo, hi]; above: key > hi (never true when d1 is the top digit)
+    const uint32_t lo = d1 << kHistShift, hi = lo | ((1u << kHistShift) - 1u);
     for (int s = 0; s < nst; ++s) {
       const int slot = s % kStages;
       if (!mbar_wait_bounded(&S.full[slot], (uint32_t)(s / kStages) & 1u)) waited_ok = false;
-      const uint32_t* st = S.ring[slot] + warp * 256;
+      // the warp's 128 keys as 4 words of 32: lane l holds key 32 e + l of word e, so a ballot
+      // is a bitmap word
+      const uint32_t* st = S.ring[slot] + warp * 128;
+      const int lp = s * kStageKeys + warp * 128 + lane;  // chunk position of key e = 0
+      const int wbase = s * (kStageKeys / 32) + warp * 4;
+      const bool full_stage = (s + 1) * kStageKeys <= len;
 #pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const int lp = s * kStageKeys + warp * 256 + e * 32 + lane;  // position in the chunk
-        const bool valid = lp < len;
+      for (int e = 0; e < 4; ++e) {
         const uint32_t key = st[e * 32 + lane];
-        const uint32_t dg = key >> kHistShift;
-        const uint32_t ab = __ballot_sync(0xffffffffu, valid && dg > d1);
-        const uint32_t cb = __ballot_sync(0xffffffffu, valid && dg == d1);
-        if (lane == 0) {
-          S.bm[s * (kStageKeys / 32) + warp * 8 + e] = ab;
-          my_above += (uint32_t)__popc(ab);
-        }
+        const bool valid = full_stage || lp + e * 32 < len;
+        const uint32_t ab = __ballot_sync(0xffffffffu, valid && key > hi);
+        const uint32_t cb = __ballot_sync(0xffffffffu, valid && key - lo <= hi - lo);
+        if (lane == e) S.bm[wbase + e] = ab;
+        my_above += (lane == e) ? (uint32_t)__popc(ab) : 0u;
         if (cb) {
-          const int leader = __ffs(cb) - 1;
           uint32_t base = 0u;
-          if (lane == leader) base = atomicAdd(&S.ctl.ccount, (uint32_t)__popc(cb));
-          base = __shfl_sync(0xffffffffu, base, leader);
-          if ((cb >> lane) & 1u) {
-            const uint32_t j = base + (uint32_t)__popc(cb & ((1u << lane) - 1u));
-            if (j < (uint32_t)kCap) {
-              S.ckey[j] = key;
-              S.cpos[j] = c0 + lp;
-            }
+          if (lane == 0) base = atomicAdd(&S.ctl.ccount, (uint32_t)__popc(cb));
+          base = __shfl_sync(0xffffffffu, base, 0);
+          const uint32_t j = base + (uint32_t)__popc(cb & ((1u << lane) - 1u));
+          if (((cb >> lane) & 1u) && j < (uint32_t)kCap) {
+            S.ckey[j] = key;
+            S.cpos[j] = c0 + lp + e * 32;
           }
         }
       }
@@ -291,6 +298,8 @@ __global__ void __launch_bounds__(kThreads, 1) select_topk_kernel(const SelectPa
         issue(s + kStages);
       }
     }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) my_above += __shfl_xor_sync(0xffffffffu, my_above, o);
     if (lane == 0 && my_above) atomicAdd(&S.ctl.above, my_above);
     __syncthreads();
     cluster_wait();  // every CTA of the cluster is set up: CTA 0's list may now be appended to
@@ -316,7 +325,6 @@ __global__ void __launch_bounds__(kThreads, 1) select_topk_kernel(const SelectPa
     }
     cluster_sync();  // B: CTA 0 holds every candidate
     if (rank == 0) {
-      for (int i = tid; i < kHistBins; i += kThreads) const_cast<uint32_t*>(ghist)[i] = 0u;  // for the next call
       if (tid == 0) S.ctl.ntie = 0u;
       __syncthreads();
       // ---- CTA 0: digits 2 and 3 among the candidates, then the ties ----
@@ -328,14 +336,14 @@ __global__ void __launch_bounds__(kThreads, 1) select_topk_kernel(const SelectPa
         for (uint32_t i = tid; i < total; i += kThreads)
           atomicAdd(&S.hloc[(S.ckey[i] >> kDigit3Bits) & (kBins2 - 1)], 1u);
         __syncthreads();
-        find_digit<kBins2 / kThreads>(S.hloc, k_rem, S.wsum, &S.found);
+        find_digit<kBins2>(S.hloc, k_rem, S.wsum, &S.found);
         const uint32_t d2 = S.found.digit;
         k_rem -= S.found.above;
         const uint32_t pre = (d1 << kDigit2Bits) | d2;
         for (uint32_t i = tid; i < total; i += kThreads)
           if ((S.ckey[i] >> kDigit3Bits) == pre) atomicAdd(&S.hacc3[S.ckey[i] & (kBins3 - 1)], 1u);
         __syncthreads();
-        find_digit<kBins3 / kThreads>(S.hacc3, k_rem, S.wsum, &S.found);
+        find_digit<kBins3>(S.hacc3, k_rem, S.wsum, &S.found);
         T = (pre << kDigit3Bits) | S.found.digit;
         k_rem -= S.found.above;
         need = k_rem;  // ties on T to take, 1 <= need <= eq
@@ -383,6 +391,8 @@ __global__ void __launch_bounds__(kThreads, 1) select_topk_kernel(const SelectPa
       }
     }
     cluster_sync();  // C: results are in every CTA
+    if (rank == 0)
+      for (int i = tid; i < kHistBins; i += kThreads) const_cast<uint32_t*>(ghist)[i] = 0u;  // for the next call
   } else {
     // Too many candidates for the list: drain the copies issued above, then take the slow path.
     if (tid == 0)
@@ -418,7 +428,7 @@ __global__ void __launch_bounds__(kThreads, 1) select_topk_kernel(const SelectPa
     for (int i = tid; i < kBins2; i += kThreads)
       if (S.hloc[i]) dsmem_red_add(dsmem_addr(&S.hacc2[i], 0), S.hloc[i]);
     cluster_sync();
-    find_digit<kBins2 / kThreads>(cg::this_cluster().map_shared_rank(S.hacc2, 0), k_rem, S.wsum, &S.found);
+    find_digit<kBins2>(cg::this_cluster().map_shared_rank(S.hacc2, 0), k_rem, S.wsum, &S.found);
     const uint32_t pre = (d1 << kDigit2Bits) | S.found.digit;
     k_rem -= S.found.above;
     // digit 3
@@ -432,7 +442,7 @@ __global__ void __launch_bounds__(kThreads, 1) select_topk_kernel(const SelectPa
     for (int i = tid; i < kBins3; i += kThreads)
       if (S.hloc[i]) dsmem_red_add(dsmem_addr(&S.hacc3[i], 0), S.hloc[i]);
     cluster_sync();
-    find_digit<kBins3 / kThreads>(cg::this_cluster().map_shared_rank(S.hacc3, 0), k_rem, S.wsum, &S.found);
+    find_digit<kBins3>(cg::this_cluster().map_shared_rank(S.hacc3, 0), k_rem, S.wsum, &S.found);
     const uint32_t T = (pre << kDigit3Bits) | S.found.digit;
     const uint32_t need = k_rem - S.found.above;
     // bits above T and ties on T, word by word; counts per CTA
