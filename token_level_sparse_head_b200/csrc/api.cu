@@ -39,6 +39,31 @@ cudaError_t prepare_kernel(const void* kern, int smem_bytes, bool nonportable_cl
   return e;
 }
 
+int ctas_per_sm(const void* kern, int threads, int smem_bytes) {
+  struct Key {
+    const void* k;
+    int dev, threads, smem;
+    bool operator==(const Key& o) const { return k == o.k && dev == o.dev && threads == o.threads && smem == o.smem; }
+  };
+  struct Hash {
+    size_t operator()(const Key& x) const {
+      return std::hash<const void*>()(x.k) ^ ((size_t)x.dev << 48) ^ ((size_t)x.threads << 32) ^ (size_t)x.smem;
+    }
+  };
+  static std::mutex mu;
+  static std::unordered_map<Key, int, Hash> cache;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 1;
+  const Key key{kern, dev, threads, smem_bytes};
+  std::lock_guard<std::mutex> lock(mu);
+  auto it = cache.find(key);
+  if (it != cache.end()) return it->second;
+  int n = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, threads, (size_t)smem_bytes) != cudaSuccess || n < 1) n = 1;
+  cache.emplace(key, n);
+  return n;
+}
+
 }  // namespace sas
 
 namespace {
@@ -103,11 +128,11 @@ int num_sms() {
 
 constexpr size_t kErrBytes = 256;
 
-sas::AttendParams attend_plan(const sas_shape* s, int count_max) {
+sas::AttendParams attend_plan(const sas_shape* s, int count_max, bool dense) {
   sas::AttendParams a = {};
   a.B = s->B; a.Hq = s->Hq; a.Hkv = s->Hkv; a.G = s->Hq / s->Hkv; a.d = s->d;
   a.cap = cap_of(s);
-  sas::plan_attend(a, count_max);
+  sas::plan_attend(a, count_max, dense);
   return a;
 }
 
@@ -159,7 +184,7 @@ sas_status plan_selection(const sas_shape* s, const void* q, const float* M, con
                           const int32_t* page_table, const int32_t* seqlens, const int32_t* k, int32_t k_max,
                           float lambda, const float* log_g, int32_t* idx_out, float* scores_out, void* ws,
                           SelectPlan* out) {
-  const sas::AttendParams a = attend_plan(s, k_max);
+  const sas::AttendParams a = attend_plan(s, k_max, false);
   const WsLayout L = ws_layout(a, true);
   unsigned char* w = static_cast<unsigned char*>(ws);
   const int sms = num_sms();
@@ -221,7 +246,7 @@ sas_status do_select(const sas_shape* s, const void* q, const float* M, const vo
 sas_status do_attend(const sas_shape* s, const void* q, const void* K, const void* V, const int32_t* page_table,
                      const int32_t* seqlens, const int32_t* idx, const int32_t* k, int32_t count_max,
                      float lambda, const float* log_g, float* out, void* ws, cudaStream_t st) {
-  sas::AttendParams a = attend_plan(s, count_max);
+  sas::AttendParams a = attend_plan(s, count_max, idx == nullptr);
   bind_workspace(a, ws);
   a.q = static_cast<const __nv_bfloat16*>(q);
   a.K = static_cast<const __nv_bfloat16*>(K);
@@ -232,6 +257,7 @@ sas_status do_attend(const sas_shape* s, const void* q, const void* K, const voi
   a.kvec = k;
   a.log_g = (idx != nullptr && lambda != 0.0f) ? log_g : nullptr;
   a.out = out;
+  a.sms = num_sms();
   a.max_pages = s->max_pages; a.num_pages = s->num_pages; a.paged = s->page_size ? 1 : 0;
   a.k_max = count_max;
   a.sigma = 1.0f / sqrtf((float)s->d);
@@ -262,12 +288,12 @@ const char* sas_last_error_detail(void) { return g_detail; }
 
 size_t sas_decode_workspace_bytes(const sas_shape* shape, int32_t k_max) {
   if (check_shape(shape) != SAS_OK || k_max < 1) return 0;
-  return ws_bytes_for(attend_plan(shape, k_max), true);
+  return ws_bytes_for(attend_plan(shape, k_max, false), true);
 }
 
 size_t sas_dense_workspace_bytes(const sas_shape* shape) {
   if (check_shape(shape) != SAS_OK) return 0;
-  return ws_bytes_for(attend_plan(shape, cap_of(shape)), false);
+  return ws_bytes_for(attend_plan(shape, cap_of(shape), true), false);
 }
 
 sas_status sas_workspace_init(void* workspace, size_t ws_bytes, void* stream) {
@@ -519,7 +545,7 @@ sas_status sas_decode_step_static_scratch(const sas_shape* shape, const void* q,
   // The error word, the per-head histograms and the split counters must start at zero; a
   // previous call may have been cut short, so every call clears them.  The score keys and
   // the attention partials that follow are written before they are read.
-  const WsLayout L = ws_layout(attend_plan(shape, k_max), true);
+  const WsLayout L = ws_layout(attend_plan(shape, k_max, false), true);
   const cudaError_t e = cudaMemsetAsync(ws, 0, L.partials, st);
   if (e != cudaSuccess) return cuda_fail(e, "clearing the static scratch");
   SAS_TRY(do_select(shape, q, M, Kproj, page_table, seqlens, k, k_max, lambda, log_g, idx_out, nullptr, ws, st));

@@ -3,9 +3,10 @@
 // JSSA page, section 原理详解(二) / Triton 内核的三个设计点: one launch per layer serves
 // every KV head, each query head is mapped to the index set its KV head selected, and the K/V
 // rows are read where they live, with no staging copy of the selected cache.  One token's K
-// (or V) head slice is contiguous (section 不规则索引本身不是障碍), so each selected row is
-// fetched as one bulk copy of d*2 bytes on the TMA engine straight into this warp's shared
-// memory ring; the page holding it is resolved per index for the paged layout.
+// (or V) head slice is contiguous (section 不规则索引本身不是障碍): the lanes of a warp copy
+// the selected rows in 16-byte pieces (cp.async) straight into the warp's shared-memory ring;
+// the page holding each row is resolved per index for the paged layout.  The dense variant
+// fetches whole 8-row tiles with one bulk copy (TMA engine) each for K and V.
 //
 // Grid: (splits, B*Hkv, G/gt).  A CTA takes a contiguous slice of one (b, h) index list and
 // gt query heads of h; its 4 warps take 8-token tiles of the slice in turn, each warp with its
@@ -24,7 +25,15 @@ namespace {
 constexpr int kWarps = 4;
 constexpr int kThreads = kWarps * 32;
 constexpr int kTile = 8;     // tokens per warp tile
-constexpr int kStages = 3;   // ring depth per warp
+constexpr int kStages = 2;   // ring depth per warp
+
+// 16-byte global -> shared copy by this thread (completes at the next wait on its group).
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
 template <int D, int GT>
 struct Geo {
@@ -188,34 +197,47 @@ __global__ void __launch_bounds__(kThreads) attend_kernel(const AttendParams p) 
   const int ntiles = (cnt + kTile - 1) / kTile;
   const int nt_w = ntiles > warp ? (ntiles - warp + kWarps - 1) / kWarps : 0;
 
+  // Tile `it` of this warp into its ring slot.  Dense: a tile is 8 consecutive positions
+  // starting at a multiple of 8, i.e. consecutive rows of the cache (within one 64-token page
+  // for the paged layout), fetched as one bulk copy each for K and V.  Sparse: the selected
+  // rows are scattered, so every lane copies 16-byte pieces of them (cp.async, one group per
+  // tile; an empty group past the last tile keeps the group count uniform).
+  constexpr int kPieces = kTile * D / 8;          // 16-byte pieces of the tile's K rows
+  constexpr int kPiecesPerLane = kPieces / 32;
   auto issue = [&](int it) {
-    const int tile = warp + it * kWarps;
-    const int tb = tile * kTile;
-    const int ntok = min(kTile, cnt - tb);
     const int slot = it % kStages;
     unsigned char* st = wring + (size_t)slot * Gm::STAGE_BYTES;
-    if (lane == 0) mbar_arrive_expect_tx(&bars[slot], (uint32_t)(ntok * 2 * Gm::ROW_BYTES));
-    __syncwarp();
     if (DENSE) {
-      // A tile is 8 consecutive positions starting at a multiple of 8: consecutive rows of the
-      // cache (within one 64-token page for the paged layout), fetched as one copy each.
+      const int tile = warp + it * kWarps;
+      const int tb = tile * kTile;
+      const int ntok = min(kTile, cnt - tb);
+      if (lane == 0) mbar_arrive_expect_tx(&bars[slot], (uint32_t)(ntok * 2 * Gm::ROW_BYTES));
+      __syncwarp();
       if (lane < 2) {
         const uint32_t row = rows_s[tb];
         const __nv_bfloat16* src = (lane ? p.V : p.K) + (size_t)row * D;
         bulk_g2s(st + (size_t)(lane ? kTile : 0) * Gm::ROW_BYTES, src, (uint32_t)(ntok * Gm::ROW_BYTES), &bars[slot]);
       }
-    } else if (lane < 2 * kTile) {
-      const int t = lane & (kTile - 1);
-      if (t < ntok) {
-        const uint32_t row = rows_s[tb + t];
-        const bool isv = lane >= kTile;
-        const __nv_bfloat16* src = (isv ? p.V : p.K) + (size_t)row * D;
-        bulk_g2s(st + (size_t)(isv ? kTile + t : t) * Gm::ROW_BYTES, src, Gm::ROW_BYTES, &bars[slot]);
+    } else {
+      if (it < nt_w) {
+        const int tb = (warp + it * kWarps) * kTile;
+        const int ntok = min(kTile, cnt - tb);
+#pragma unroll
+        for (int i = 0; i < kPiecesPerLane; ++i) {
+          const int c = lane + 32 * i;         // piece c: row c / (D/8), part c % (D/8)
+          const int t = c / (D / 8), part = c % (D / 8);
+          if (t < ntok) {
+            const size_t row = rows_s[tb + t];
+            cp_async16(st + (size_t)t * Gm::ROW_BYTES + part * 16, p.K + row * D + part * 8);
+            cp_async16(st + (size_t)(kTile + t) * Gm::ROW_BYTES + part * 16, p.V + row * D + part * 8);
+          }
+        }
       }
+      cp_async_commit();
     }
   };
 
-  for (int it = 0; it < min(kStages, nt_w); ++it) issue(it);
+  for (int it = 0; it < (DENSE ? min(kStages, nt_w) : kStages); ++it) issue(it);
 
   float m_run = -INFINITY;  // running max of this lane's head
   float l_part = 0.f;       // this lane's share of the running sum (owner lanes)
@@ -230,7 +252,12 @@ __global__ void __launch_bounds__(kThreads) attend_kernel(const AttendParams p) 
     const int slot = it % kStages;
     const int tb = (warp + it * kWarps) * kTile;
     const int ntok = min(kTile, cnt - tb);
-    if (!mbar_wait_bounded(&bars[slot], (uint32_t)(it / kStages) & 1u)) waited_ok = false;
+    if (DENSE) {
+      if (!mbar_wait_bounded(&bars[slot], (uint32_t)(it / kStages) & 1u)) waited_ok = false;
+    } else {
+      cp_async_wait<kStages - 1>();  // this lane's pieces of tile `it` have landed
+      __syncwarp();                  // ... and every other lane's
+    }
     const unsigned char* st = wring + (size_t)slot * Gm::STAGE_BYTES;
 
     // QK: partial dots of this lane's 8 channels, for NP rows x GT heads.
@@ -329,8 +356,13 @@ __global__ void __launch_bounds__(kThreads) attend_kernel(const AttendParams p) 
       }
     }
     __syncwarp();
-    if (it + kStages < nt_w) issue(it + kStages);
+    if (DENSE) {
+      if (it + kStages < nt_w) issue(it + kStages);
+    } else {
+      issue(it + kStages);
+    }
   }
+  if (!DENSE) cp_async_wait<0>();
   if (!waited_ok) record_error(p.err, kDevWaitTimeout, (uint32_t)bh);
 
   // ---- per-warp totals: l over the owner lanes of each head ----
@@ -456,9 +488,46 @@ __global__ void __launch_bounds__(kThreads) attend_kernel(const AttendParams p) 
   if (tid == 0) p.counters[bhz] = 0u;
 }
 
+// Shared-memory bytes of a plan.
+template <int D, int GT>
+int plan_smem(int split_len, int splits) {
+  return smem_layout<D, GT>(split_len, splits).total;
+}
+
 template <int D, int GT, bool GATED, bool PAGED, bool DENSE>
-cudaError_t launch_t(const AttendParams& p, cudaStream_t stream) {
+cudaError_t launch_t(const AttendParams& p0, cudaStream_t stream) {
   auto kern = attend_kernel<D, GT, GATED, PAGED, DENSE>;
+  AttendParams p = p0;
+  if (!DENSE && p.sms > 0) {
+    // Re-split for whole waves: CTAs resident per SM at the largest slice, then the split count
+    // in [s_lo, max_splits] whose grid fills its last wave best (the most splits when even
+    // max_splits does not fill one wave).
+    const int count_max = p.k_max;
+    const int occ = ctas_per_sm((const void*)kern, kThreads, plan_smem<D, GT>(kMaxSplitLen, p.max_splits));
+    const long heads = (long)p.B * p.Hkv * p.ngz;
+    const long slots = (long)p.sms * occ;
+    const int s_lo = (count_max + kMaxSplitLen - 1) / kMaxSplitLen;
+    int best = p.max_splits;
+    if (heads * p.max_splits > slots) {
+      double best_eff = -1.0;
+      for (int s = s_lo < 1 ? 1 : s_lo; s <= p.max_splits; ++s) {
+        const long ctas = heads * s;
+        const long waves = (ctas + slots - 1) / slots;
+        const double eff = (double)ctas / (double)(waves * slots);
+        if (eff > best_eff + 1e-9) {
+          best_eff = eff;
+          best = s;
+        }
+        if (eff >= 0.9) break;
+      }
+    }
+    int len = (count_max + best - 1) / best;
+    len = (len + 31) & ~31;
+    if (len < 32) len = 32;
+    p.split_len = len;
+    p.splits = (count_max + len - 1) / len;
+    p.smem_bytes = plan_smem<D, GT>(p.split_len, p.splits);
+  }
   cudaError_t e = prepare_kernel((const void*)kern, p.smem_bytes);
   if (e != cudaSuccess) return e;
   dim3 grid((unsigned)p.splits, (unsigned)(p.B * p.Hkv), (unsigned)p.ngz);
@@ -488,35 +557,41 @@ cudaError_t launch_d(const AttendParams& p, cudaStream_t stream) {
 
 }  // namespace
 
-void plan_attend(AttendParams& p, int count_max) {
+void plan_attend(AttendParams& p, int count_max, bool dense) {
   p.gt = (p.G % 4 == 0) ? 4 : ((p.G % 2 == 0) ? 2 : 1);
   p.ngz = p.G / p.gt;
   const long heads = (long)p.B * p.Hkv * p.ngz;
   if (count_max < 1) count_max = 1;
+  const long maxlen = dense ? kMaxSplitLenDense : kMaxSplitLen;
   long s = (kTargetCtas + heads - 1) / heads;
   if (s < 1) s = 1;
   long len = (count_max + s - 1) / s;
   len = (len + 31) & ~31L;
-  if (len < 128) len = 128;
+  if (len < kMinSplitLen) len = kMinSplitLen;
   const long cm32 = ((long)count_max + 31) & ~31L;
   if (len > cm32) len = cm32;
-  if (len > kMaxSplitLen) len = kMaxSplitLen;
+  if (len > maxlen) len = maxlen;
   p.split_len = (int)len;
   p.splits = (int)((count_max + len - 1) / len);
-  p.nstages = kStages;
-  Smem L;
-  if (p.d == 128) {
-    L = (p.gt == 4) ? smem_layout<128, 4>(p.split_len, p.splits)
-                    : (p.gt == 2 ? smem_layout<128, 2>(p.split_len, p.splits) : smem_layout<128, 1>(p.split_len, p.splits));
-  } else {
-    L = (p.gt == 4) ? smem_layout<64, 4>(p.split_len, p.splits)
-                    : (p.gt == 2 ? smem_layout<64, 2>(p.split_len, p.splits) : smem_layout<64, 1>(p.split_len, p.splits));
+  p.max_splits = p.splits;
+  if (!dense) {
+    int more = (count_max + kMinSplitLen - 1) / kMinSplitLen;
+    if (more > kMaxSplitsPerHead) more = kMaxSplitsPerHead;
+    if (more > p.max_splits) p.max_splits = more;
   }
-  p.smem_bytes = L.total;
+  int smem;
+  if (p.d == 128) {
+    smem = (p.gt == 4) ? plan_smem<128, 4>(p.split_len, p.splits)
+                       : (p.gt == 2 ? plan_smem<128, 2>(p.split_len, p.splits) : plan_smem<128, 1>(p.split_len, p.splits));
+  } else {
+    smem = (p.gt == 4) ? plan_smem<64, 4>(p.split_len, p.splits)
+                       : (p.gt == 2 ? plan_smem<64, 2>(p.split_len, p.splits) : plan_smem<64, 1>(p.split_len, p.splits));
+  }
+  p.smem_bytes = smem;
 }
 
 size_t attend_workspace_floats(const AttendParams& p) {
-  return (size_t)p.B * p.Hkv * p.ngz * p.splits * p.gt * (p.d + 2);
+  return (size_t)p.B * p.Hkv * p.ngz * p.max_splits * p.gt * (p.d + 2);
 }
 
 cudaError_t launch_attend(const AttendParams& p, cudaStream_t stream) {

@@ -88,20 +88,28 @@ struct AttendParams {
   int ngz;                     // G / gt
   int splits;                  // CTAs per (b, h, head group)
   int split_len;               // index-list entries per CTA (multiple of 32)
-  int nstages;
+  int max_splits;              // splits the workspace holds partials for (>= splits)
   int smem_bytes;
+  int sms;                     // SMs of the device (launch-time re-split)
 };
-// Split plan for `count_max` index entries per head; pure function of the arguments.
-void plan_attend(AttendParams& p, int count_max);
+// Split plan for `count_max` index entries per head (dense: every cached row); a pure function
+// of the arguments, which sizes the workspace.  launch_attend may re-split the work (up to
+// max_splits) to fill whole waves of the device it runs on.
+void plan_attend(AttendParams& p, int count_max, bool dense);
 size_t attend_workspace_floats(const AttendParams& p);
 cudaError_t launch_attend(const AttendParams& p, cudaStream_t stream);
 
 // Raises a kernel's dynamic shared-memory limit (and allows non-portable cluster sizes) on the
 // current device once, not on every launch; thread-safe.
 cudaError_t prepare_kernel(const void* kern, int smem_bytes, bool nonportable_cluster = false);
+// Resident CTAs per SM of a kernel at a block size and dynamic shared memory (cached per device).
+int ctas_per_sm(const void* kern, int threads, int smem_bytes);
 
-constexpr int kTargetCtas = 1024;   // attention split planning target (device independent)
-constexpr int kMaxSplitLen = 2048;  // index entries per attention CTA at most
+constexpr int kTargetCtas = 1024;       // attention split planning target (device independent)
+constexpr int kMaxSplitLen = 512;       // sparse: index entries per attention CTA at most
+constexpr int kMaxSplitLenDense = 2048; // dense: rows per attention CTA at most
+constexpr int kMinSplitLen = 128;
+constexpr int kMaxSplitsPerHead = 64;   // re-split bound (workspace partials)
 constexpr int kMaxChunk = 16384;    // positions per selection CTA at most
 constexpr int kMaxCluster = 16;
 
