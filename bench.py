@@ -223,6 +223,23 @@ class Workload:
         self.torch.cuda.empty_cache()
 
 
+def max_over_ranks(t, dist=None):
+    """The slowest rank's time (every rank gets it); t itself without a process group."""
+    if dist is None:
+        return t
+    import torch
+
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    tt = torch.tensor([t], dtype=torch.float64, device=dev)
+    dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+    return float(tt.item())
+
+
+def job_throughput(steps, world, t_max):
+    """Whole-job steps/s: every rank ran `steps` steps of its own replica in at most t_max s."""
+    return steps * world / t_max
+
+
 def timed_block(torch, fn, steps, dist=None):
     """Time `steps` calls of fn as one block: barrier + sync on both sides, CUDA events on the
     current stream; returns the max over ranks of the elapsed seconds."""
@@ -237,12 +254,7 @@ def timed_block(torch, fn, steps, dist=None):
     torch.cuda.synchronize()
     if dist is not None:
         dist.barrier()
-    t = e0.elapsed_time(e1) / 1e3
-    if dist is not None:
-        tt = torch.tensor([t], dtype=torch.float64, device="cuda")
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        t = float(tt.item())
-    return t
+    return max_over_ranks(e0.elapsed_time(e1) / 1e3, dist)
 
 
 def flush_l2(flush_buf):
@@ -320,7 +332,7 @@ def run_ours(args):
     t = timed_block(torch, graph.replay if graph is not None else wl.step, args.steps, dist)
     clocks = sampler.stop()
     ms = t / args.steps * 1e3
-    value = args.steps * world / t
+    value = job_throughput(args.steps, world, t)
 
     # --- per-kernel durations (component entry points, events between the kernels)
     nk = max(3, min(args.steps, 200))
@@ -363,7 +375,7 @@ def run_ours(args):
         e2e_step()
     ne = max(3, min(args.steps, 200))
     te = timed_block(torch, e2e_step, ne, dist)
-    e2e = {"value": ne * world / te, "unit": UNIT,
+    e2e = {"value": job_throughput(ne, world, te), "unit": UNIT,
            "h2d_bytes_per_step": q_host.numel() * 2 + knew_host.numel() * 2,
            "d2h_bytes_per_step": out_host.numel() * 4}
 
