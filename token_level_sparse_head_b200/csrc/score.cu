@@ -10,12 +10,12 @@
 // Persistent kernel, one CTA per SM.  The work is the list of 4 KB blocks of projected rows
 // (64 rows at r = 32) of every (b, h) that needs scores, in (b, h, position) order; each CTA
 // takes one contiguous, equal share of it, so a CTA walks the rows of one or a few heads front
-// to back.  A producer warp streams the blocks into a shared-memory ring with bulk copies (TMA
+// to back.  Two producer warps stream the blocks into a shared-memory ring with bulk copies (TMA
 // engine: one copy per block, or per 64-token page piece for the paged layout, plus the block's
-// gate values); each of its lanes owns one ring slot.  Sixteen consumer warps take the blocks in
-// turn, each with its own two ring slots, so every warp's dependent chain (dot products,
-// butterfly reduction, key, histogram) overlaps the others' and about 130 KB of rows stay in
-// flight per SM.  Full blocks take a path without per-row tests.  Keys go to the workspace with
+// gate values); each producer lane owns one ring slot.  Twelve consumer warps take the blocks in
+// turn, each with its own three ring slots, so a warp's processing of one block (dot products,
+// butterfly reduction, key, histogram) overlaps the copies of its next two and about 144 KB of
+// rows stay in flight per SM.  Full blocks take a path without per-row tests.  Keys go to the workspace with
 // an L2 evict-last hint so that the selection kernel finds them on chip.
 #include "sas_device.cuh"
 #include "sas_kernels.h"
@@ -23,12 +23,14 @@
 namespace sas {
 namespace {
 
-constexpr int kConsumerWarps = 16;
+constexpr int kConsumerWarps = 12;
 constexpr int kConsumers = kConsumerWarps * 32;
-constexpr int kThreads = kConsumers + 32;  // + one producer warp
+constexpr int kProducerWarps = 2;          // one lane per ring slot
+constexpr int kThreads = kConsumers + kProducerWarps * 32;
 constexpr int kBlockBytes = 4096;          // projected bytes per block (one ring stage)
-constexpr int kDepth = 2;                  // ring slots per consumer warp
+constexpr int kDepth = 3;                  // ring slots per consumer warp
 constexpr int kSlots = kConsumerWarps * kDepth;
+static_assert(kSlots <= kProducerWarps * 32, "one producer lane per ring slot");
 
 template <int R>
 struct Geo {
@@ -64,11 +66,6 @@ static_assert(sizeof(Smem<16, 128>) <= 227 * 1024 && sizeof(Smem<32, 128>) <= 22
                   sizeof(Smem<64, 128>) <= 227 * 1024,
               "score kernel shared memory");
 
-__device__ __forceinline__ uint64_t policy_evict_last() {
-  uint64_t pol;
-  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
-  return pol;
-}
 __device__ __forceinline__ void stg_hint(uint32_t* ptr, uint32_t v, uint64_t pol) {
   asm volatile("st.global.L2::cache_hint.u32 [%0], %1, %2;" ::"l"(ptr), "r"(v), "l"(pol) : "memory");
 }
@@ -217,12 +214,12 @@ __global__ void __launch_bounds__(kThreads, 1) score_kernel(const ScoreParams p)
   const bool scores = p.scores_out != nullptr;
   bool waited_ok = true;
 
-  if (warp == kConsumerWarps) {
-    // ---------------------------------------------------------------- producer
-    // Lane l owns ring slot l (kSlots == 32) and issues the CTA's blocks l, l + 32, l + 64, ...
-    // into it, each once consumer warp l % 16 has released the slot.
-    static_assert(kSlots == 32, "one producer lane per ring slot");
-    if (pl.count > lane) {
+  if (warp >= kConsumerWarps) {
+    // ---------------------------------------------------------------- producers
+    // Producer lane L owns ring slot L and issues the CTA's blocks L, L + kSlots, ... into it,
+    // each once consumer warp L % kConsumerWarps has released the slot.
+    const int L = (warp - kConsumerWarps) * 32 + lane;
+    if (L < kSlots && pl.count > L) {
       const unsigned char* kp = reinterpret_cast<const unsigned char*>(p.kproj);
       int b = pl.b0, h = pl.h0, c = pl.c0;
       SeqInfo si = seq_info<BR>(p, b, false);
@@ -242,10 +239,10 @@ __global__ void __launch_bounds__(kThreads, 1) score_kernel(const ScoreParams p)
           }
         }
       };
-      advance(lane);
-      const int slot = lane;
+      advance(L);
+      const int slot = L;
       uint32_t phase = 0u;
-      for (int t = lane; t < pl.count; t += kSlots) {
+      for (int t = L; t < pl.count; t += kSlots) {
         if (t >= kSlots) {
           if (!mbar_wait_bounded(&S.empty[slot], phase)) waited_ok = false;
           phase ^= 1u;
@@ -284,7 +281,7 @@ __global__ void __launch_bounds__(kThreads, 1) score_kernel(const ScoreParams p)
   }
 
   // ------------------------------------------------------------------ consumers
-  const uint64_t pol_keep = policy_evict_last();
+  const uint64_t pol_keep = l2_evict_last();
   const int part = lane % Gm::LPR;  // this lane's 16-byte chunk of each row it loads
   const int rsub = lane / Gm::LPR;  // its row within each load instruction
   float2 qv[4];
@@ -299,11 +296,13 @@ __global__ void __launch_bounds__(kThreads, 1) score_kernel(const ScoreParams p)
     const int bh = b * p.Hkv + h;
     // ---- new head (every consumer warp, whether or not it gets blocks of it) ----
     {
-      constexpr int TPR = kConsumers / R;
+      // TPR threads per output of q-hat: a power of two with R * TPR <= kConsumers
+      constexpr int TPR = (kConsumers / R) >= 32 ? 32 : (kConsumers / R) >= 16 ? 16 : (kConsumers / R) >= 8 ? 8 : 4;
       constexpr int CH = D / TPR;
       const int qj = tid / TPR, qpart = tid % TPR;
+      const bool qrow = qj < R;
       float mreg[CH];
-      const float* Mrow = p.M + ((size_t)h * R + qj) * D + qpart * CH;
+      const float* Mrow = p.M + ((size_t)h * R + (qrow ? qj : 0)) * D + qpart * CH;
 #pragma unroll
       for (int i = 0; i < CH; ++i) mreg[i] = Mrow[i];
       consumers_sync();  // every warp is done with the previous head's rows
@@ -329,7 +328,7 @@ __global__ void __launch_bounds__(kThreads, 1) score_kernel(const ScoreParams p)
       for (int i = 0; i < CH; ++i) sp = fmaf(mreg[i], S.qbar[qpart * CH + i], sp);
 #pragma unroll
       for (int o = TPR / 2; o; o >>= 1) sp += __shfl_xor_sync(0xffffffffu, sp, o);
-      if (qpart == 0) S.qhat[qj] = sp * p.sigma;
+      if (qpart == 0 && qrow) S.qhat[qj] = sp * p.sigma;
       consumers_sync();
 #pragma unroll
       for (int e = 0; e < 4; ++e) qv[e] = make_float2(S.qhat[part * 8 + 2 * e], S.qhat[part * 8 + 2 * e + 1]);
