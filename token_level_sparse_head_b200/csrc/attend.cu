@@ -116,6 +116,29 @@ __global__ void __launch_bounds__(kThreads) attend_kernel(const AttendParams p) 
   const int j1 = min(j0 + p.split_len, count);
   const int cnt = max(0, j1 - j0);
 
+  if (lane == 0) {
+    for (int s = 0; s < kStages; ++s) mbar_init(&bars_all[warp * kStages + s], 1);
+    fence_barrier_init();
+  }
+
+  // ---- query slice in registers: lane holds channels c0..c0+7 of each of its gt heads ----
+  const int rl = lane % Gm::LPR;   // lane within its row
+  const int rs = lane / Gm::LPR;   // row slot within a warp instruction
+  const int c0 = rl * 8;
+  float2 qv[GT][4];
+#pragma unroll
+  for (int g = 0; g < GT; ++g) {
+    const int hq = h * p.G + gz * GT + g;
+    const uint4 w = *reinterpret_cast<const uint4*>(p.q + ((size_t)b * p.Hq + hq) * D + c0);
+    qv[g][0] = make_float2(bf16lo(w.x) * p.sigma, bf16hi(w.x) * p.sigma);
+    qv[g][1] = make_float2(bf16lo(w.y) * p.sigma, bf16hi(w.y) * p.sigma);
+    qv[g][2] = make_float2(bf16lo(w.z) * p.sigma, bf16hi(w.z) * p.sigma);
+    qv[g][3] = make_float2(bf16lo(w.w) * p.sigma, bf16hi(w.w) * p.sigma);
+  }
+  // The index list (written by the selection) and the workspace are read only from here on.
+  pdl_wait();
+  pdl_trigger();
+
   // ---- resolve the slice's rows (and gate terms) once; loads batched 4 per thread ----
   for (int jb = 0; jb < cnt; jb += 4 * kThreads) {
     int iv[4];
@@ -160,25 +183,6 @@ __global__ void __launch_bounds__(kThreads) attend_kernel(const AttendParams p) 
         if (GATED) lg_s[j] = p.lam * lgv[u];
       }
     }
-  }
-  if (lane == 0) {
-    for (int s = 0; s < kStages; ++s) mbar_init(&bars_all[warp * kStages + s], 1);
-    fence_barrier_init();
-  }
-
-  // ---- query slice in registers: lane holds channels c0..c0+7 of each of its gt heads ----
-  const int rl = lane % Gm::LPR;   // lane within its row
-  const int rs = lane / Gm::LPR;   // row slot within a warp instruction
-  const int c0 = rl * 8;
-  float2 qv[GT][4];
-#pragma unroll
-  for (int g = 0; g < GT; ++g) {
-    const int hq = h * p.G + gz * GT + g;
-    const uint4 w = *reinterpret_cast<const uint4*>(p.q + ((size_t)b * p.Hq + hq) * D + c0);
-    qv[g][0] = make_float2(bf16lo(w.x) * p.sigma, bf16hi(w.x) * p.sigma);
-    qv[g][1] = make_float2(bf16lo(w.y) * p.sigma, bf16hi(w.y) * p.sigma);
-    qv[g][2] = make_float2(bf16lo(w.z) * p.sigma, bf16hi(w.z) * p.sigma);
-    qv[g][3] = make_float2(bf16lo(w.w) * p.sigma, bf16hi(w.w) * p.sigma);
   }
   __syncthreads();
 
@@ -531,8 +535,7 @@ cudaError_t launch_t(const AttendParams& p0, cudaStream_t stream) {
   cudaError_t e = prepare_kernel((const void*)kern, p.smem_bytes);
   if (e != cudaSuccess) return e;
   dim3 grid((unsigned)p.splits, (unsigned)(p.B * p.Hkv), (unsigned)p.ngz);
-  kern<<<grid, kThreads, (size_t)p.smem_bytes, stream>>>(p);
-  return cudaGetLastError();
+  return launch_pdl(kern, grid, dim3(kThreads), (size_t)p.smem_bytes, stream, p);
 }
 
 template <int D, int GT>

@@ -21,6 +21,8 @@ constexpr int kBuildThreads = 256;
 
 template <int D, int R>
 __global__ void __launch_bounds__(kBuildThreads) build_kernel(const ProjParams p) {
+  pdl_wait();
+  pdl_trigger();
   extern __shared__ __align__(16) unsigned char smem_raw[];
   float* Ms = reinterpret_cast<float*>(smem_raw);
   const int bh = blockIdx.y;
@@ -97,6 +99,8 @@ __global__ void __launch_bounds__(kBuildThreads) build_kernel(const ProjParams p
 // channel block t % 8, and the 8 partials meet in a butterfly.
 template <int D, int R>
 __global__ void __launch_bounds__(256) append_kernel(const ProjParams p) {
+  pdl_wait();
+  pdl_trigger();
   const int bh = blockIdx.x;
   const int b = bh / p.Hkv, h = bh % p.Hkv;
   const int n = p.seqlens[b];
@@ -156,16 +160,14 @@ __global__ void __launch_bounds__(256) append_kernel(const ProjParams p) {
 template <int D, int R>
 cudaError_t launch_dr(const ProjParams& p, cudaStream_t stream) {
   if (p.append) {
-    append_kernel<D, R><<<p.B * p.Hkv, 256, 0, stream>>>(p);
-    return cudaGetLastError();
+    return launch_pdl(append_kernel<D, R>, dim3((unsigned)(p.B * p.Hkv)), dim3(256), 0, stream, p);
   }
   const size_t smem = (size_t)R * D * 4;
   auto kern = build_kernel<D, R>;
   cudaError_t e = prepare_kernel((const void*)kern, (int)smem);
   if (e != cudaSuccess) return e;
   dim3 grid((unsigned)((p.cap + p.rows_per_cta - 1) / p.rows_per_cta), (unsigned)(p.B * p.Hkv), 1);
-  kern<<<grid, kBuildThreads, smem, stream>>>(p);
-  return cudaGetLastError();
+  return launch_pdl(kern, grid, dim3(kBuildThreads), smem, stream, p);
 }
 
 template <int D>

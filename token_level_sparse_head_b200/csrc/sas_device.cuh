@@ -59,6 +59,14 @@ __device__ __forceinline__ SeqSelection seq_selection(int kb, int n) {
 }
 
 // ----------------------------------------------------------------------------- PTX
+// Programmatic dependent launch.  Every kernel of the library calls pdl_wait() before it touches
+// any buffer an earlier kernel on the stream reads or writes, and pdl_trigger() right after, so
+// the next kernel may start its independent prologue while this one runs.  Once a kernel has
+// passed pdl_wait() every earlier kernel on the stream has completed (each of them waited for
+// its own predecessor before triggering).  Both are no-ops for a launch without the attribute.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }

@@ -105,6 +105,32 @@ cudaError_t prepare_kernel(const void* kern, int smem_bytes, bool nonportable_cl
 // Resident CTAs per SM of a kernel at a block size and dynamic shared memory (cached per device).
 int ctas_per_sm(const void* kern, int threads, int smem_bytes);
 
+// Launches kern(p) with programmatic dependent launch allowed (the kernel's pdl_wait() orders
+// it after the previous kernel on the stream) and, if cluster > 0, that cluster size along x.
+template <typename P>
+inline cudaError_t launch_pdl(void (*kern)(P), dim3 grid, dim3 block, size_t smem, cudaStream_t stream, const P& p,
+                              unsigned cluster = 0) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  unsigned n = 1;
+  if (cluster > 0) {
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = cluster;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    n = 2;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = n;
+  return cudaLaunchKernelEx(&cfg, kern, p);
+}
+
 constexpr int kTargetCtas = 1024;       // attention split planning target (device independent)
 constexpr int kMaxSplitLen = 512;       // sparse: index entries per attention CTA at most
 constexpr int kMaxSplitLenDense = 2048; // dense: rows per attention CTA at most

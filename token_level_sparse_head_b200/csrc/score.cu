@@ -209,6 +209,10 @@ __global__ void __launch_bounds__(kThreads, 1) score_kernel(const ScoreParams p)
     }
   }
   __syncthreads();
+  // The projected cache (appended to by the previous kernel), the keys, the histograms and the
+  // error word are touched only from here on.
+  pdl_wait();
+  pdl_trigger();
   const Plan pl = S.plan;
   const bool gated = GATED;
   const bool scores = p.scores_out != nullptr;
@@ -422,8 +426,7 @@ cudaError_t launch_rd(const ScoreParams& p, cudaStream_t stream) {
   auto kern = p.log_g != nullptr ? score_kernel<R, D, true> : score_kernel<R, D, false>;
   cudaError_t e = prepare_kernel((const void*)kern, smem);
   if (e != cudaSuccess) return e;
-  kern<<<p.ctas, kThreads, smem, stream>>>(p);
-  return cudaGetLastError();
+  return launch_pdl(kern, dim3((unsigned)p.ctas), dim3(kThreads), (size_t)smem, stream, p);
 }
 
 }  // namespace

@@ -208,6 +208,8 @@ __global__ void __launch_bounds__(kThreads, 1) select_topk_kernel(const SelectPa
 
   if (!sel.ranked) {
     // Nothing to rank (uniform over the cluster): the first k_eff positions, or none.
+    pdl_wait();
+    pdl_trigger();
     for (int j = (int)rank * kThreads + tid; j < p.k_max; j += C * kThreads) idx[j] = (j < k_eff) ? j : -1;
     return;
   }
@@ -235,6 +237,9 @@ __global__ void __launch_bounds__(kThreads, 1) select_topk_kernel(const SelectPa
     S.found = f;
   }
   __syncthreads();
+  // The keys and histograms of the score pass are read only from here on.
+  pdl_wait();
+  pdl_trigger();
 
   // Stage s of the chunk: keys [s * kStageKeys, +kStageKeys) as whole 16-byte units (the key
   // rows have a multiple of 4 entries, so the rounding stays inside this (b, h)'s row).
@@ -539,19 +544,8 @@ cudaError_t launch_select(const SelectParams& p, cudaStream_t stream) {
   auto kern = select_topk_kernel;
   const cudaError_t e = prepare_kernel((const void*)kern, p.smem_bytes, p.cluster > 8);
   if (e != cudaSuccess) return e;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)p.cluster, (unsigned)(p.B * p.Hkv), 1);
-  cfg.blockDim = dim3(kThreads, 1, 1);
-  cfg.dynamicSmemBytes = (size_t)p.smem_bytes;
-  cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = (unsigned)p.cluster;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, p);
+  return launch_pdl(kern, dim3((unsigned)p.cluster, (unsigned)(p.B * p.Hkv), 1), dim3(kThreads), (size_t)p.smem_bytes,
+                    stream, p, (unsigned)p.cluster);
 }
 
 }  // namespace sas
