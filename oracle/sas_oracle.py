@@ -56,6 +56,26 @@ def bf16_round(x) -> np.ndarray:
 
 
 # ----------------------------------------------------------------------------------------
+# FP8 E4M3 rounding (the storage format of the FP8 projected cache)
+# ----------------------------------------------------------------------------------------
+E4M3_MAX = 448.0  # largest finite E4M3 value
+
+
+def e4m3_round(x) -> np.ndarray:
+    """Round float64 values to the nearest FP8 E4M3 value, ties to even, saturating at +-448.
+
+    E4M3 keeps 4 significant bits with exponent bias 7: a value x = m * 2**e (0.5 <= |m| < 1)
+    has quantum 2**(e-4); below the normal range the quantum stays 2**-9 (subnormals).  The
+    format has no infinity; magnitudes past 448 saturate (the finite-saturating conversion).
+    """
+    x = np.asarray(x, np.float64)
+    _, e = np.frexp(x)
+    qe = np.maximum(e.astype(np.int64) - 4, -9)
+    y = np.ldexp(np.rint(np.ldexp(x, -qe)), qe)  # scaling by powers of two is exact
+    return np.clip(y, -E4M3_MAX, E4M3_MAX)
+
+
+# ----------------------------------------------------------------------------------------
 # Cache layout: logical rows of one (sequence, KV head)
 # ----------------------------------------------------------------------------------------
 def logical_rows(cache, b, h, n, page_table=None, page_size=64):
@@ -80,6 +100,14 @@ def project_keys(K_rows, M):
     K_rows: [n, d] (bf16 values as float64); M: [r, d] with orthonormal rows.
     """
     return bf16_round(np.asarray(K_rows, np.float64) @ np.asarray(M, np.float64).T)
+
+
+def project_keys_fp8(K_rows, M, scale):
+    """FP8 projected rows: codes = e4m3( (K_rows @ M^T) / scale ); the value scored is
+    scale * code.  ([JSSA] FP8 打分缓存的影响可以忽略: the projected cache is stored in FP8;
+    the per-KV-head scale is this implementation's reading, the pages leave it open.)"""
+    y = np.asarray(K_rows, np.float64) @ np.asarray(M, np.float64).T
+    return e4m3_round(y / float(scale))
 
 
 # ----------------------------------------------------------------------------------------
@@ -184,12 +212,14 @@ def decode_head(q_heads, M_h, kproj_rows, K_rows, V_rows, k, lam=0.0, log_g_rows
 
 
 def decode_step(q, Kproj, K, V, M, seqlens, k, lam=0.0, log_g=None, page_table=None,
-                page_size=64, heads=None):
+                page_size=64, heads=None, kproj_scale=None):
     """Decode step over all (or the listed) (sequence, KV head) pairs.
 
     Arrays are numpy (bf16 values as float64, fp32 as float64, ints as int64):
       q [B][Hq][d]; Kproj/K/V in the contiguous or paged layout (see logical_rows);
       M [Hkv][r][d]; seqlens, k [B]; log_g [B][Hkv][cap] when lam != 0.
+    kproj_scale: [Hkv] for an FP8 cache (Kproj holds the codes; the scored rows are
+      kproj_scale[h] * codes), None for a bf16 cache.
     heads: optional list of (b, h) pairs to evaluate (default all).
     Returns dict (b, h) -> (idx, out [G, d], u, keys).
     """
@@ -201,6 +231,8 @@ def decode_step(q, Kproj, K, V, M, seqlens, k, lam=0.0, log_g=None, page_table=N
     for b, h in pairs:
         n = int(seqlens[b])
         kp = logical_rows(Kproj, b, h, n, page_table, page_size)
+        if kproj_scale is not None:
+            kp = float(kproj_scale[h]) * np.asarray(kp, np.float64)
         kr = logical_rows(K, b, h, n, page_table, page_size)
         vr = logical_rows(V, b, h, n, page_table, page_size)
         lg = None if lam == 0.0 else np.asarray(log_g)[b, h, :n]
@@ -223,8 +255,9 @@ def dense_step(q, K, V, seqlens, Hkv, page_table=None, page_size=64, heads=None)
     return res
 
 
-def build_proj_cache(K, M, seqlens, page_table=None, page_size=64, heads=None):
-    """O1 over whole caches: returns a Kproj array in the layout of K (rows past N_b are 0)."""
+def build_proj_cache(K, M, seqlens, page_table=None, page_size=64, heads=None, kproj_scale=None):
+    """O1 over whole caches: returns a Kproj array in the layout of K (rows past N_b are 0);
+    with kproj_scale ([Hkv]) the FP8 codes of project_keys_fp8 instead of bf16 values."""
     K = np.asarray(K)
     r = M.shape[1]
     out = np.zeros(K.shape[:-1] + (r,), np.float64)
@@ -233,7 +266,8 @@ def build_proj_cache(K, M, seqlens, page_table=None, page_size=64, heads=None):
     pairs = heads if heads is not None else [(b, h) for b in range(B) for h in range(Hkv)]
     for b, h in pairs:
         n = int(seqlens[b])
-        rows = project_keys(logical_rows(K, b, h, n, page_table, page_size), M[h])
+        kr = logical_rows(K, b, h, n, page_table, page_size)
+        rows = project_keys(kr, M[h]) if kproj_scale is None else project_keys_fp8(kr, M[h], kproj_scale[h])
         if page_table is None:
             out[b, h, :n] = rows
         else:

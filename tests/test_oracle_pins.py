@@ -318,3 +318,38 @@ def test_calibration_bound_and_optimality():
         for _ in range(10):
             Q = np.linalg.qr(RNG.standard_normal((d, r)))[0]
             assert lmarg <= O.marginal_objective(Q @ Q.T, Gq, Gk) + 1e-12
+
+
+# ------------------------------------------------------------------ FP8 E4M3 (projected cache)
+def test_e4m3_round_hand_values():
+    cases = {
+        0.0: 0.0, 1.0: 1.0, 1.0625: 1.0, 1.1875: 1.25,   # spacing 1/8 in [1, 2); ties to even
+        17.0: 16.0, 19.0: 20.0, 18.0: 18.0,               # spacing 2 in [16, 32)
+        448.0: 448.0, 500.0: 448.0, -1000.0: -448.0,      # saturation at the finite maximum
+        2.0 ** -9: 2.0 ** -9, 2.0 ** -10: 0.0, 3 * 2.0 ** -10: 2.0 ** -8,  # subnormal spacing 2**-9
+        0.001: 2.0 ** -9, -0.53125: -0.5,
+    }
+    for x, want in cases.items():
+        assert O.e4m3_round(x) == want, (x, O.e4m3_round(x), want)
+
+
+def test_e4m3_round_matches_torch_in_range():
+    rng = np.random.default_rng(5)
+    x = np.concatenate([rng.standard_normal(20000) * s for s in (1e-3, 1e-1, 1.0, 30.0, 150.0)])
+    x = np.clip(x, -448.0, 448.0).astype(np.float32)
+    want = torch.from_numpy(x).to(torch.float8_e4m3fn).to(torch.float64).numpy()
+    np.testing.assert_array_equal(O.e4m3_round(x.astype(np.float64)), want)
+
+
+def test_project_keys_fp8_identity_rows_round_the_scaled_channels():
+    rng = np.random.default_rng(6)
+    K = O.bf16_round(rng.standard_normal((64, 32)))
+    M = np.eye(32)[:8]
+    for scale in (2.0 ** -6, 1.0, 4.0):
+        codes = O.project_keys_fp8(K, M, scale)
+        np.testing.assert_array_equal(codes, O.e4m3_round(K[:, :8] / scale))
+        # the scored value is scale * code: within half an FP8 quantum of the true projection
+        err = np.abs(scale * codes - K[:, :8])
+        _, e = np.frexp(K[:, :8] / scale)
+        half_q = 0.5 * scale * np.ldexp(1.0, np.maximum(e - 4, -9))
+        assert np.all(err <= half_q + 1e-300)
