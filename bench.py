@@ -30,18 +30,20 @@ METRIC = "sparse decode steps/s & achieved HBM GB/s at N=128K, B=1/16; speedup v
 UNIT = "steps/s"
 DEFAULT_WORKLOAD = "long-128k-b16"
 SECONDARY_WORKLOAD = "long-128k-b1"
+FP8_WORKLOAD = "long-128k-b16-fp8"
 L2_BYTES = 126 * 1024 * 1024
 
 
 # ------------------------------------------------------------------------------ accounting
-def roofline_bytes(B, Hq, Hkv, d, r, seqlens, ks, lam):
+def roofline_bytes(B, Hq, Hkv, d, r, seqlens, ks, lam, kp_bytes=2):
     """Algorithmic HBM bytes of one step, per kernel and in total.
 
-    Per (sequence b, KV head): N_b*r*2 (projected cache scan) + k_b*2*d*2 (selected K and V
-    rows) + G*d*2 (queries) + G*d*4 (fp32 output) [+ N_b*4 gate inputs when lambda != 0].
+    Per (sequence b, KV head): N_b*r*kp_bytes (projected cache scan; 2 for bf16, 1 for FP8) +
+    k_b*2*d*2 (selected K and V rows) + G*d*2 (queries) + G*d*4 (fp32 output) [+ N_b*4 gate
+    inputs when lambda != 0].
     """
     G = Hq // Hkv
-    kproj = sum(int(n) * r * 2 for n in seqlens) * Hkv
+    kproj = sum(int(n) * r * kp_bytes for n in seqlens) * Hkv
     kv = sum(min(int(k), int(n)) * 2 * d * 2 for n, k in zip(seqlens, ks)) * Hkv
     q = B * Hq * d * 2
     out = B * Hq * d * 4
@@ -158,10 +160,12 @@ class Workload:
         self.p = p
         self.shape = shape_of(p)
         self.sess = DecodeSession(self.shape, p.k_max, device=device)
+        self.fp8 = p.kproj_scale is not None
+        kdt = torch.uint8 if self.fp8 else torch.bfloat16   # FP8 E4M3 codes or bf16 values
         if p.paged:
-            self.kproj = torch.zeros(p.num_pages, p.Hkv, 64, p.r, dtype=torch.bfloat16, device=device)
+            self.kproj = torch.zeros(p.num_pages, p.Hkv, 64, p.r, dtype=kdt, device=device)
         else:
-            self.kproj = torch.zeros(p.B, p.Hkv, p.n_cap, p.r, dtype=torch.bfloat16, device=device)
+            self.kproj = torch.zeros(p.B, p.Hkv, p.n_cap, p.r, dtype=kdt, device=device)
         lib.sas_build_proj_cache(self.shape, p.K, p.M, self.kproj, p.page_table, p.seqlens)
         # the newest key of every sequence (position N_b - 1), for the append of each step
         sl = p.seqlens.tolist()
@@ -175,7 +179,7 @@ class Workload:
         self.knew = knew
         self.seqlens_h = sl
         self.ks_h = p.k.tolist()
-        self.bytes = roofline_bytes(p.B, p.Hq, p.Hkv, p.d, p.r, sl, self.ks_h, p.lam)
+        self.bytes = roofline_bytes(p.B, p.Hq, p.Hkv, p.d, p.r, sl, self.ks_h, p.lam, kp_bytes=1 if self.fp8 else 2)
         self.dense_bytes = dense_bytes(p.B, p.Hq, p.Hkv, p.d, sl)
         self.cfg = dict(CONFIGS[name])
 
@@ -407,6 +411,30 @@ def run_ours(args):
                      "kernels_ms": kt}
         wl = w1
 
+    # --- the same 128K B=16 workload with the projected cache in FP8 E4M3 (the pages' setting)
+    fp8 = None
+    if not args.no_fp8 and args.workload == DEFAULT_WORKLOAD:
+        wl.free()
+        del wl
+        w8 = Workload(FP8_WORKLOAD, dev, torch)
+        for _ in range(3):
+            w8.step()
+        g8 = capture_graph(torch, w8.step)
+        n8 = max(10, min(args.steps, 300))
+        t8 = timed_block(torch, g8.replay if g8 is not None else w8.step, n8, dist)
+        evs8 = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(20)]
+        for i in range(20):
+            w8.step_parts(evs8[i])
+        torch.cuda.synchronize()
+        k8 = {nm: statistics.mean(e[i].elapsed_time(e[i + 1]) for e in evs8) for i, nm in enumerate(names)}
+        ms8 = t8 / n8 * 1e3
+        fp8 = {"workload": FP8_WORKLOAD, "ms_per_step": ms8, "steps_per_s": 1e3 / ms8,
+               "hbm_gbs": w8.bytes["step"] / (ms8 * 1e-3) / 1e9, "step_bytes": w8.bytes["step"],
+               "speedup_vs_bf16_kproj": ms / ms8, "kernels_ms": k8,
+               "score_hbm_gbs": w8.bytes["score"] / (k8["score"] * 1e-3) / 1e9,
+               "timing": "CUDA graph replay of the step" if g8 is not None else "stream launches"}
+        wl = w8
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(args.workload, budget_s=args.cpu_seconds)
@@ -438,6 +466,8 @@ def run_ours(args):
     line["dense"]["hbm_gbs"] = head_dense_bytes / (dense_ms * 1e-3) / 1e9
     if secondary:
         line["b1"] = secondary
+    if fp8:
+        line["fp8_kproj"] = fp8
     print(json.dumps(line), flush=True)
 
 
@@ -548,6 +578,7 @@ def main():
     ap.add_argument("--batch", type=int, default=None, help="override the workload's batch (profiling)")
     ap.add_argument("--no-secondary", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-fp8", action="store_true", help="skip the FP8 projected-cache line")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     args = ap.parse_args()
     if args.warmup < 3:

@@ -25,9 +25,10 @@
  *   - Query head hq belongs to KV head hq / G, G = Hq / Hkv (contiguous groups).
  *   - The softmax scale is sigma = 1/sqrt(d) on attention logits and on selection scores.
  *   - Cache layouts:
- *       contiguous (page_size == 0): K, V [B][Hkv][n_cap][d] bf16; Kproj [B][Hkv][n_cap][r] bf16;
+ *       contiguous (page_size == 0): K, V [B][Hkv][n_cap][d] bf16; Kproj [B][Hkv][n_cap][r];
  *       paged (page_size == 64):     K, V [num_pages][Hkv][64][d] bf16;
- *                                    Kproj [num_pages][Hkv][64][r] bf16;
+ *                                    Kproj [num_pages][Hkv][64][r];
+ *     Kproj elements are bf16 or FP8 E4M3 codes (shape.kproj_dtype);
  *                                    page_table [B][max_pages] int32, logical token t of
  *                                    sequence b lives in page page_table[b][t / 64], row t % 64.
  *     The logical capacity is cap = n_cap (contiguous) or max_pages * 64 (paged).
@@ -49,7 +50,7 @@
 extern "C" {
 #endif
 
-#define SAS_ABI_VERSION 1
+#define SAS_ABI_VERSION 2
 
 typedef enum {
   SAS_OK = 0,
@@ -59,8 +60,13 @@ typedef enum {
   SAS_ERR_DEVICE_CHECK = 4
 } sas_status;
 
-/* Storage type of the projected cache.  Only bf16 exists in this version. */
-typedef enum { SAS_KPROJ_BF16 = 0 } sas_kproj_dtype;
+/* Storage type of the projected cache.
+ *   SAS_KPROJ_BF16      bfloat16 values (2 bytes per element).
+ *   SAS_KPROJ_FP8_E4M3  FP8 E4M3 codes (1 byte per element) with a per-KV-head fp32 scale:
+ *                       the value scored is kproj_scale[h] * code (JSSA page, section
+ *                       FP8 打分缓存的影响可以忽略: the scoring cache is kept in FP8).  Codes
+ *                       are produced by rounding to nearest even and saturating at +-448. */
+typedef enum { SAS_KPROJ_BF16 = 0, SAS_KPROJ_FP8_E4M3 = 1 } sas_kproj_dtype;
 
 /* Problem shape shared by every call.
  *   B       sequences in the batch
@@ -70,7 +76,10 @@ typedef enum { SAS_KPROJ_BF16 = 0 } sas_kproj_dtype;
  *   n_cap   contiguous layout: rows per (sequence, KV head) slot, a multiple of 4; 0 if paged
  *   page_size 0 (contiguous) or 64 (paged)
  *   max_pages paged: columns of the page table; num_pages: physical pages in K/V/Kproj
- *   kproj_dtype SAS_KPROJ_BF16
+ *   kproj_dtype SAS_KPROJ_BF16 or SAS_KPROJ_FP8_E4M3
+ *   kproj_scale device fp32 [Hkv]: the per-KV-head scale of an FP8 projected cache (read by the
+ *           projection and scoring kernels); NULL for bf16.  Powers of two keep the projection's
+ *           division by the scale exact; other values are divided in fp32, rounded to nearest.
  */
 typedef struct {
   int32_t B, Hq, Hkv, d, r;
@@ -79,6 +88,7 @@ typedef struct {
   int32_t max_pages;
   int32_t num_pages;
   int32_t kproj_dtype;
+  const float* kproj_scale;
 } sas_shape;
 
 /* Longest logical capacity (tokens per sequence) the selection kernel holds on chip. */
@@ -113,7 +123,8 @@ sas_status sas_check_workspace(void* workspace, size_t ws_bytes, void* stream,
                                uint32_t* code_out, uint32_t* where_out);
 
 /* Projected score cache, built over the whole cache (prefill).
- *   Kproj[b,h,i,:] = bf16_rn( sum_c K[b,h,i,c] * M[h,:,c] ), fp32 accumulation, for i < N_b.
+ *   Kproj[b,h,i,:] = bf16_rn( sum_c K[b,h,i,c] * M[h,:,c] ), fp32 accumulation, for i < N_b;
+ *   FP8: e4m3_rn_satfinite( that fp32 sum / kproj_scale[h] ).
  *   K    bf16 cache (layout above), read;  M fp32 [Hkv][r][d] orthonormal rows, read;
  *   Kproj bf16 (same layout family as K, width r), rows i < N_b written, others untouched;
  *   page_table NULL for the contiguous layout.

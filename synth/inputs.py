@@ -33,6 +33,9 @@ CONFIGS = {
     "8b-32k": dict(B=1, Hq=32, Hkv=8, d=128, r=32, N=32768, k=2048, basis="eye", aniso=True),
     "long-128k-b1": dict(B=1, Hq=32, Hkv=8, d=128, r=32, N=131072, k=4096, basis="eye", aniso=True),
     "long-128k-b16": dict(B=16, Hq=32, Hkv=8, d=128, r=32, N=131072, k=4096, basis="eye", aniso=True),
+    # the same with the projected cache in FP8 E4M3 (per-KV-head power-of-two scale)
+    "long-128k-b16-fp8": dict(B=16, Hq=32, Hkv=8, d=128, r=32, N=131072, k=4096, basis="eye", aniso=True,
+                              kproj_fp8=True),
     "paged-b16": dict(B=16, Hq=32, Hkv=8, d=128, r=32, N=None, n_lo=8192, n_hi=131072,
                       k=None, k_div=32, basis="eye", aniso=True, paged=True),
     "gated-b4-k256": dict(B=4, Hq=32, Hkv=8, d=128, r=32, N=65536, k=256, lam=1.0, basis="eye", aniso=True),
@@ -89,6 +92,7 @@ class DecodeProblem:
     M: torch.Tensor
     page_table: Optional[torch.Tensor] = None
     log_g: Optional[torch.Tensor] = None
+    kproj_scale: Optional[torch.Tensor] = None  # [Hkv] fp32 power of two (FP8 projected cache) or None
     extra: dict = field(default_factory=dict)
 
     @property
@@ -105,7 +109,7 @@ class DecodeProblem:
 
     def to(self, device) -> "DecodeProblem":
         out = DecodeProblem(**{f: getattr(self, f) for f in self.__dataclass_fields__})
-        for f in ("seqlens", "k", "q", "K", "V", "M", "page_table", "log_g"):
+        for f in ("seqlens", "k", "q", "K", "V", "M", "page_table", "log_g", "kproj_scale"):
             t = getattr(self, f)
             if t is not None:
                 setattr(out, f, t.to(device))
@@ -182,6 +186,7 @@ def make_problem(
     name: str = "custom",
     poison_tail: bool = False,
     extra_pages: int = 0,
+    kproj_fp8: bool = False,
 ) -> DecodeProblem:
     """Build a decode problem.
 
@@ -190,6 +195,10 @@ def make_problem(
     poison_tail: fill cache rows at positions >= N_b (and unused gate entries) with huge
         values / NaN, so that any read past a sequence's end shows in the result.
     extra_pages: physical pages beyond those the sequences use (never referenced).
+    kproj_fp8: the projected cache is stored as FP8 E4M3 codes with a per-KV-head scale:
+        a power of two no smaller than max_i |K_i|_2 / 448 over the cached rows (with
+        orthonormal basis rows every projected element is at most |K_i|_2, so the codes stay
+        within the E4M3 range).
     """
     assert Hq % Hkv == 0
     seqlens = [int(x) for x in (seqlens if hasattr(seqlens, "__len__") else [seqlens] * B)]
@@ -264,13 +273,31 @@ def make_problem(
                 K[b, :, seqlens[b]:, :] = big
                 V[b, :, seqlens[b]:, :] = big
 
+    kproj_scale = None
+    if kproj_fp8:
+        kproj_scale = torch.empty(Hkv, dtype=torch.float32)
+        for h in range(Hkv):
+            norm = 0.0
+            for b in range(B):
+                n = seqlens[b]
+                if n == 0:
+                    continue
+                if paged:
+                    t = torch.arange(n, device=device)
+                    rows = K[page_table[b, t // PAGE_SIZE].long(), h, t % PAGE_SIZE]
+                else:
+                    rows = K[b, h, :n]
+                norm = max(norm, float(rows.double().norm(dim=-1).max()))
+            kproj_scale[h] = 2.0 ** math.ceil(math.log2(max(norm, 1e-30) / 448.0))
+        kproj_scale = kproj_scale.to(device)
+
     return DecodeProblem(
         name=name, seed=seed, B=B, Hq=Hq, Hkv=Hkv, d=d, r=r, paged=paged,
         n_cap=n_cap_eff, max_pages=max_pages, num_pages=num_pages, k_max=int(k_max),
         lam=float(lam),
         seqlens=torch.tensor(seqlens, dtype=torch.int32, device=device),
         k=torch.tensor(kk, dtype=torch.int32, device=device),
-        q=q, K=K, V=V, M=M, page_table=page_table, log_g=log_g,
+        q=q, K=K, V=V, M=M, page_table=page_table, log_g=log_g, kproj_scale=kproj_scale,
     )
 
 
@@ -292,5 +319,5 @@ def make_config(name: str, seed: int = 0, device="cpu", **over) -> DecodeProblem
         B=B, Hq=c["Hq"], Hkv=c["Hkv"], d=c["d"], r=c["r"], seqlens=seqlens, k=k, k_max=k_max,
         paged=bool(c.get("paged", False)), lam=float(c.get("lam", 0.0)), basis=c["basis"],
         aniso=bool(c["aniso"]), seed=seed, device=device, name=name,
-        poison_tail=bool(c.get("poison_tail", False)),
+        poison_tail=bool(c.get("poison_tail", False)), kproj_fp8=bool(c.get("kproj_fp8", False)),
     )

@@ -35,20 +35,37 @@ def check_build_rows(kp_g, kp_o, a, p):
     """GPU projected rows vs the oracle's correctly rounded ones.
 
     The kernel accumulates d products in fp32 (error at most d * 2**-24 * sum_c |M_jc K_c|)
-    and rounds once to bf16, the oracle rounds the exact sum: they may differ by that error
-    plus one bf16 spacing."""
+    and rounds once (to bf16, or to E4M3 after the exact division by a power-of-two scale),
+    the oracle rounds the exact sum: they may differ by that error plus one spacing."""
     mask = _rows_mask(p, a)
     Kabs = np.abs(a["K"])[mask]                         # [rows, d]
     heads = np.nonzero(mask)[1]                         # KV head of each row
     Mabs = np.abs(a["M"])[heads]                        # [rows, r, d]
     acc_bound = p.d * 2.0 ** -24 * np.einsum("nrd,nd->nr", Mabs, Kabs)
     g, o = kp_g[mask], kp_o[mask]
-    tol = bf16_ulp(np.maximum(np.abs(g), np.abs(o))) + 1.01 * acc_bound
+    sc = _scales(p)
+    if sc is None:
+        tol = bf16_ulp(np.maximum(np.abs(g), np.abs(o))) + 1.01 * acc_bound
+    else:
+        tol = e4m3_quantum(np.maximum(np.abs(g), np.abs(o))) + 1.01 * acc_bound / sc[heads][:, None]
     assert np.all(np.abs(g - o) <= tol), f"build: worst {np.max(np.abs(g - o) / tol):.3f} of bound"
 
 
-def kproj_tensor(kp_np, device):
-    return torch.from_numpy(np.ascontiguousarray(kp_np)).to(torch.float32).to(torch.bfloat16).to(device)
+def kproj_tensor(kp_np, device, fp8=False):
+    """The oracle's projected cache as the library stores it: bf16 values or FP8 E4M3 codes
+    (both representable exactly, so the conversion is exact)."""
+    dt = torch.float8_e4m3fn if fp8 else torch.bfloat16
+    return torch.from_numpy(np.ascontiguousarray(kp_np)).to(torch.float32).to(dt).to(device)
+
+
+def e4m3_quantum(x):
+    """Spacing of E4M3 values at |x| (2**(e-4) for x = m 2**e, 0.5 <= m < 1; 2**-9 below)."""
+    _, e = np.frexp(np.abs(np.asarray(x, np.float64)))
+    return np.ldexp(1.0, np.maximum(e - 4, -9))
+
+
+def _scales(p):
+    return None if getattr(p, "kproj_scale", None) is None else f64(p.kproj_scale)
 
 
 def _rows_mask(p, a):
@@ -107,11 +124,12 @@ def compare_head(p, a, b, h, kp_rows, idx_g, out_g, scores_g=None):
 def run_small(p_cpu, device="cuda", dense=True, check_build=True):
     """Full comparison on a problem small enough for the oracle to run entirely."""
     a = problem_arrays(p_cpu)
-    kp_o = O.build_proj_cache(a["K"], a["M"], a["seqlens"], a["page_table"])
+    sc = _scales(p_cpu)
+    kp_o = O.build_proj_cache(a["K"], a["M"], a["seqlens"], a["page_table"], kproj_scale=sc)
     p = p_cpu.to(device)
     shape = shape_of(p)
     sess = DecodeSession(shape, p.k_max, device=device)
-    kp_in = kproj_tensor(kp_o, device)
+    kp_in = kproj_tensor(kp_o, device, fp8=sc is not None)
     stats = {}
 
     if check_build:
@@ -137,6 +155,7 @@ def run_small(p_cpu, device="cuda", dense=True, check_build=True):
     assert code == 0, f"device check error {code} at {where}"
     assert torch.equal(idx, idx_sel), "decode_step and select_topk index lists differ"
     assert torch.equal(idx, idx_split), "score_scan + select_from_scores differ from decode_step"
+    sc_k = _scales(p_cpu)
     sc, ix, ot = f64(scores), f64(idx), f64(out)
     G = p.Hq // p.Hkv
     ndiff = 0
@@ -144,6 +163,8 @@ def run_small(p_cpu, device="cuda", dense=True, check_build=True):
         n = int(a["seqlens"][b])
         for h in range(p.Hkv):
             kp_rows = O.logical_rows(kp_o, b, h, n, a["page_table"])
+            if sc_k is not None:
+                kp_rows = sc_k[h] * kp_rows                 # the values the codes stand for
             ndiff += compare_head(p, a, b, h, kp_rows, ix[b, h], ot[b, h * G:(h + 1) * G], sc[b, h])
     stats["band_diffs"] = ndiff
 
@@ -163,10 +184,12 @@ def run_sampled(p, heads, device="cuda", dense_heads=None):
     the benchmark times); the oracle recomputes the listed (b, h) heads from the inputs."""
     shape = shape_of(p)
     sess = DecodeSession(shape, p.k_max, device=device)
+    sc = _scales(p)
+    kdt = torch.bfloat16 if sc is None else torch.float8_e4m3fn
     if p.paged:
-        kp = torch.zeros(p.num_pages, p.Hkv, 64, p.r, dtype=torch.bfloat16, device=device)
+        kp = torch.zeros(p.num_pages, p.Hkv, 64, p.r, dtype=kdt, device=device)
     else:
-        kp = torch.zeros(p.B, p.Hkv, p.n_cap, p.r, dtype=torch.bfloat16, device=device)
+        kp = torch.zeros(p.B, p.Hkv, p.n_cap, p.r, dtype=kdt, device=device)
     lib.sas_build_proj_cache(shape, p.K, p.M, kp, p.page_table, p.seqlens)
     out, idx = sess.decode(p.q, p.M, kp, p.K, p.V, p.page_table, p.seqlens, p.k, p.lam, p.log_g)
     torch.cuda.synchronize()
@@ -181,12 +204,18 @@ def run_sampled(p, heads, device="cuda", dense_heads=None):
         n = int(seqlens[b])
         a = _head_arrays(p, b, h, n, pt, seqlens, ks)
         kp_rows_g = _head_rows(kp, b, h, n, pt)
-        kp_rows_o = O.project_keys(a["K"][0, 0, :n], a["M"][0])
         acc_bound = p.d * 2.0 ** -24 * (np.abs(a["K"][0, 0, :n]) @ np.abs(a["M"][0]).T)
-        tol = bf16_ulp(np.maximum(np.abs(kp_rows_g), np.abs(kp_rows_o))) + 1.01 * acc_bound
+        if sc is None:
+            kp_rows_o = O.project_keys(a["K"][0, 0, :n], a["M"][0])
+            tol = bf16_ulp(np.maximum(np.abs(kp_rows_g), np.abs(kp_rows_o))) + 1.01 * acc_bound
+        else:
+            kp_rows_o = O.project_keys_fp8(a["K"][0, 0, :n], a["M"][0], sc[h])
+            tol = e4m3_quantum(np.maximum(np.abs(kp_rows_g), np.abs(kp_rows_o))) + 1.01 * acc_bound / sc[h]
         assert np.all(np.abs(kp_rows_g - kp_rows_o) <= tol), "build rows outside the fp32 bound"
         if np.array_equal(f64(p.M[h]), np.eye(p.d)[: p.r]):
             assert np.array_equal(kp_rows_g, kp_rows_o), "identity basis must copy channels exactly"
+        if sc is not None:
+            kp_rows_o = sc[h] * kp_rows_o                   # the values the codes stand for
         ndiff += compare_head(_HeadView(p), a, 0, 0, kp_rows_o, f64(idx[b, h]), f64(out[b, h * G:(h + 1) * G]))
     if dense_heads:
         dout = sess.dense(p.q, p.K, p.V, p.page_table, p.seqlens, out=torch.empty_like(out))

@@ -30,7 +30,8 @@ def test_library_loads_and_exports_every_declared_symbol():
     for name in declared:
         assert hasattr(lib, name), f"{name} declared in include/ but not exported"
     assert set(L.EXPORTED) == declared, set(L.EXPORTED) ^ declared
-    assert L.sas_abi_version() == 1
+    hdr = open(os.path.join(ROOT, "include", "sas.h")).read()
+    assert L.sas_abi_version() == int(re.search(r"#define SAS_ABI_VERSION (\d+)", hdr).group(1))
 
 
 def test_workspace_sizes_are_pure_and_sane():

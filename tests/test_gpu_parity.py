@@ -127,6 +127,51 @@ def test_append_matches_build(cuda_lib):
         assert torch.equal(kp_app, kp_build)
 
 
+# ------------------------------------------------------------------ FP8 E4M3 projected cache
+@pytest.mark.parametrize("paged", [False, True])
+@pytest.mark.parametrize("lam", [0.0, 1.0])
+def test_fp8_ragged_batch(cuda_lib, paged, lam):
+    p = make_problem(B=3, Hq=8, Hkv=2, d=128, r=32, seqlens=[5000, 777, 1], k=[300, 900, 5], k_max=900,
+                     paged=paged, n_cap=None if paged else 5004, lam=lam, basis="qr", aniso=True, seed=21,
+                     poison_tail=True, kproj_fp8=True)
+    run_small(p)
+
+
+@pytest.mark.parametrize("d,r,Hq,Hkv", [(64, 16, 4, 1), (128, 64, 8, 2)])
+def test_fp8_head_shapes(cuda_lib, d, r, Hq, Hkv):
+    p = make_problem(B=2, Hq=Hq, Hkv=Hkv, d=d, r=r, seqlens=[1500, 333], k=[100, 64], basis="qr", seed=22,
+                     kproj_fp8=True)
+    run_small(p)
+
+
+def test_fp8_append_matches_build(cuda_lib):
+    from token_level_sparse_head_b200 import lib, shape_of
+
+    for paged in (False, True):
+        p = make_problem(B=3, Hq=8, Hkv=2, d=128, r=32, seqlens=[70, 1, 200], k=[8, 1, 8], paged=paged,
+                         basis="qr", seed=23, kproj_fp8=True).to("cuda")
+        s = shape_of(p)
+        shp = (p.num_pages, p.Hkv, 64, p.r) if paged else (p.B, p.Hkv, p.n_cap, p.r)
+        kp_build = torch.zeros(shp, dtype=torch.uint8, device="cuda")
+        lib.sas_build_proj_cache(s, p.K, p.M, kp_build, p.page_table, p.seqlens)
+        kp_app = kp_build.clone()
+        knew = torch.empty(p.B, p.Hkv, p.d, dtype=torch.bfloat16, device="cuda")
+        for b in range(p.B):
+            n = int(p.seqlens[b])
+            for h in range(p.Hkv):
+                if paged:
+                    pg = int(p.page_table[b, (n - 1) // 64])
+                    knew[b, h] = p.K[pg, h, (n - 1) % 64]
+                    kp_app[pg, h, (n - 1) % 64] = 0
+                else:
+                    knew[b, h] = p.K[b, h, n - 1]
+                    kp_app[b, h, n - 1] = 0
+        lib.sas_append_proj(s, knew, p.M, kp_app, p.page_table, p.seqlens)
+        torch.cuda.synchronize()
+        assert torch.equal(kp_app, kp_build)
+        assert int(kp_build.count_nonzero()) > 0
+
+
 # ------------------------------------------------------------------------ full-size workloads
 def _heads(B, Hkv):
     pairs = {(0, 0), (B - 1, Hkv - 1), (B // 2, Hkv // 2)}
@@ -134,7 +179,8 @@ def _heads(B, Hkv):
 
 
 @pytest.mark.parametrize("name", ["8b-32k", "long-128k-b1", "long-128k-b16", "paged-b16",
-                                  "gated-b4-k256", "gated-b4-k1024", "gated-b4-k4096", "gated-b4-k16384"])
+                                  "gated-b4-k256", "gated-b4-k1024", "gated-b4-k4096", "gated-b4-k16384",
+                                  "long-128k-b16-fp8"])
 def test_full_size_sampled(cuda_lib, name):
     torch.cuda.empty_cache()
     p = make_config(name, device="cuda")

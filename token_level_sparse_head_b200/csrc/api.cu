@@ -93,7 +93,13 @@ sas_status check_shape(const sas_shape* s) {
   if (s->d != 64 && s->d != 128) return fail(SAS_ERR_UNSUPPORTED, "head dim d=%d (supported: 64, 128)", s->d);
   if (s->r != 16 && s->r != 32 && s->r != 64) return fail(SAS_ERR_UNSUPPORTED, "rank r=%d (supported: 16, 32, 64)", s->r);
   if (s->r > s->d) return fail(SAS_ERR_INVALID_ARG, "rank r=%d exceeds d=%d", s->r, s->d);
-  if (s->kproj_dtype != SAS_KPROJ_BF16) return fail(SAS_ERR_UNSUPPORTED, "kproj_dtype %d", s->kproj_dtype);
+  if (s->kproj_dtype != SAS_KPROJ_BF16 && s->kproj_dtype != SAS_KPROJ_FP8_E4M3)
+    return fail(SAS_ERR_UNSUPPORTED, "kproj_dtype %d", s->kproj_dtype);
+  if (s->kproj_dtype == SAS_KPROJ_FP8_E4M3) {
+    if (s->kproj_scale == nullptr) return fail(SAS_ERR_INVALID_ARG, "FP8 projected cache needs kproj_scale");
+    if ((reinterpret_cast<uintptr_t>(s->kproj_scale) & 3u) != 0)
+      return fail(SAS_ERR_INVALID_ARG, "kproj_scale is not 4-byte aligned");
+  }
   if (s->page_size == 0) {
     if (s->n_cap < 4 || (s->n_cap % 4)) return fail(SAS_ERR_INVALID_ARG, "n_cap=%d must be a positive multiple of 4", s->n_cap);
     if ((long long)s->B * s->Hkv * s->n_cap >= (1LL << 32)) return fail(SAS_ERR_UNSUPPORTED, "cache rows exceed 2^32");
@@ -193,7 +199,9 @@ sas_status plan_selection(const sas_shape* s, const void* q, const float* M, con
   sp = {};
   sp.q = static_cast<const __nv_bfloat16*>(q);
   sp.M = M;
-  sp.kproj = static_cast<const __nv_bfloat16*>(Kproj);
+  sp.kproj = Kproj;
+  sp.fp8 = s->kproj_dtype == SAS_KPROJ_FP8_E4M3 ? 1 : 0;
+  sp.kproj_scale = s->kproj_scale;
   sp.page_table = s->page_size ? page_table : nullptr;
   sp.seqlens = seqlens;
   sp.kvec = k;
@@ -329,7 +337,9 @@ sas_status sas_build_proj_cache(const sas_shape* shape, const void* K, const flo
   sas::ProjParams p = {};
   p.K = static_cast<const __nv_bfloat16*>(K);
   p.M = M;
-  p.Kproj = static_cast<__nv_bfloat16*>(Kproj);
+  p.Kproj = Kproj;
+  p.fp8 = shape->kproj_dtype == SAS_KPROJ_FP8_E4M3 ? 1 : 0;
+  p.kproj_scale = shape->kproj_scale;
   p.page_table = shape->page_size ? page_table : nullptr;
   p.seqlens = seqlens;
   p.err = nullptr;
@@ -350,7 +360,9 @@ sas_status sas_append_proj(const sas_shape* shape, const void* K_new, const floa
   sas::ProjParams p = {};
   p.K = static_cast<const __nv_bfloat16*>(K_new);
   p.M = M;
-  p.Kproj = static_cast<__nv_bfloat16*>(Kproj);
+  p.Kproj = Kproj;
+  p.fp8 = shape->kproj_dtype == SAS_KPROJ_FP8_E4M3 ? 1 : 0;
+  p.kproj_scale = shape->kproj_scale;
   p.page_table = shape->page_size ? page_table : nullptr;
   p.seqlens = seqlens;
   p.B = shape->B; p.Hkv = shape->Hkv; p.d = shape->d; p.r = shape->r; p.cap = cap_of(shape);

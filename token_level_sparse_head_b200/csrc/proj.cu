@@ -1,4 +1,5 @@
-// Projected score cache: Kproj = K M^T stored as bf16 (sm_100a).
+// Projected score cache: Kproj = K M^T stored as bf16, or as FP8 E4M3 codes of
+// (K M^T) / kproj_scale[h] (sm_100a).
 //
 // JSSA page, section 投影打分缓存与校准成本: besides the raw bf16 KV cache, a low-rank key
 // cache Kproj = K M^T (M in R^{r x d}, orthonormal rows, one per KV head) is kept for token
@@ -10,7 +11,10 @@
 // append: the newest key of every (b, h), one CTA per (b, h), 8 threads per output element.
 // Both use one summation order for each output: 8 partial sums over consecutive blocks of d/8
 // channels (fp32, in channel order), combined as ((p0+p1)+(p2+p3))+((p4+p5)+(p6+p7)), then
-// rounded to bf16 (nearest even); so an appended row is bit-identical to the same row built.
+// rounded to bf16 (nearest even) or divided by the head's scale and rounded to E4M3 (nearest
+// even, saturating at +-448); so an appended row is bit-identical to the same row built.
+#include <cuda_fp8.h>
+
 #include "sas_device.cuh"
 #include "sas_kernels.h"
 
@@ -19,7 +23,12 @@ namespace {
 
 constexpr int kBuildThreads = 256;
 
-template <int D, int R>
+// Two FP8 E4M3 codes (x in the low byte) of a / s and b / s, nearest even, saturating.
+__device__ __forceinline__ uint32_t fp8x2(float a, float b, float s) {
+  return (uint32_t)__nv_cvt_float2_to_fp8x2(make_float2(__fdiv_rn(a, s), __fdiv_rn(b, s)), __NV_SATFINITE, __NV_E4M3);
+}
+
+template <int D, int R, bool FP8>
 __global__ void __launch_bounds__(kBuildThreads) build_kernel(const ProjParams p) {
   pdl_wait();
   pdl_trigger();
@@ -53,7 +62,8 @@ __global__ void __launch_bounds__(kBuildThreads) build_kernel(const ProjParams p
   const uint2* src = reinterpret_cast<const uint2*>(p.K + row * D);
   constexpr int BLK = D / 8;  // channels per partial sum
   constexpr int JB = 4;       // outputs per pass
-  uint32_t outw[R / 2];
+  uint32_t outw[FP8 ? R / 4 : R / 2];
+  const float scale = FP8 ? p.kproj_scale[h] : 1.f;
 #pragma unroll
   for (int jb = 0; jb < R; jb += JB) {
     float part[JB][8];
@@ -84,20 +94,26 @@ __global__ void __launch_bounds__(kBuildThreads) build_kernel(const ProjParams p
       const float* q = part[jj];
       acc[jj] = ((q[0] + q[1]) + (q[2] + q[3])) + ((q[4] + q[5]) + (q[6] + q[7]));
     }
+    if constexpr (FP8) {
+      outw[jb / 4] = fp8x2(acc[0], acc[1], scale) | (fp8x2(acc[2], acc[3], scale) << 16);
+    } else {
 #pragma unroll
-    for (int jj = 0; jj < JB; jj += 2) {
-      const __nv_bfloat162 pr = __floats2bfloat162_rn(acc[jj], acc[jj + 1]);
-      outw[(jb + jj) / 2] = *reinterpret_cast<const uint32_t*>(&pr);
+      for (int jj = 0; jj < JB; jj += 2) {
+        const __nv_bfloat162 pr = __floats2bfloat162_rn(acc[jj], acc[jj + 1]);
+        outw[(jb + jj) / 2] = *reinterpret_cast<const uint32_t*>(&pr);
+      }
     }
   }
-  uint4* dst = reinterpret_cast<uint4*>(p.Kproj + row * R);
+  constexpr int ROW_BYTES = FP8 ? R : 2 * R;
+  uint4* dst = reinterpret_cast<uint4*>(static_cast<unsigned char*>(p.Kproj) + row * ROW_BYTES);
 #pragma unroll
-  for (int v = 0; v < R / 8; ++v) dst[v] = make_uint4(outw[4 * v], outw[4 * v + 1], outw[4 * v + 2], outw[4 * v + 3]);
+  for (int v = 0; v < ROW_BYTES / 16; ++v)
+    dst[v] = make_uint4(outw[4 * v], outw[4 * v + 1], outw[4 * v + 2], outw[4 * v + 3]);
 }
 
 // One CTA per (b, h); thread t computes the partial of output j = t / 8 (+32 per pass) over
 // channel block t % 8, and the 8 partials meet in a butterfly.
-template <int D, int R>
+template <int D, int R, bool FP8>
 __global__ void __launch_bounds__(256) append_kernel(const ProjParams p) {
   pdl_wait();
   pdl_trigger();
@@ -152,22 +168,34 @@ __global__ void __launch_bounds__(256) append_kernel(const ProjParams p) {
       a += __shfl_xor_sync(0xffffffffu, a, 1);
       a += __shfl_xor_sync(0xffffffffu, a, 2);
       a += __shfl_xor_sync(0xffffffffu, a, 4);
-      if (part == 0) p.Kproj[row * R + j] = __float2bfloat16_rn(a);
+      if (part == 0) {
+        if constexpr (FP8) {
+          static_cast<unsigned char*>(p.Kproj)[row * R + j] =
+              (unsigned char)__nv_cvt_float_to_fp8(__fdiv_rn(a, p.kproj_scale[h]), __NV_SATFINITE, __NV_E4M3);
+        } else {
+          static_cast<__nv_bfloat16*>(p.Kproj)[row * R + j] = __float2bfloat16_rn(a);
+        }
+      }
     }
   }
 }
 
-template <int D, int R>
-cudaError_t launch_dr(const ProjParams& p, cudaStream_t stream) {
+template <int D, int R, bool FP8>
+cudaError_t launch_drf(const ProjParams& p, cudaStream_t stream) {
   if (p.append) {
-    return launch_pdl(append_kernel<D, R>, dim3((unsigned)(p.B * p.Hkv)), dim3(256), 0, stream, p);
+    return launch_pdl(append_kernel<D, R, FP8>, dim3((unsigned)(p.B * p.Hkv)), dim3(256), 0, stream, p);
   }
   const size_t smem = (size_t)R * D * 4;
-  auto kern = build_kernel<D, R>;
+  auto kern = build_kernel<D, R, FP8>;
   cudaError_t e = prepare_kernel((const void*)kern, (int)smem);
   if (e != cudaSuccess) return e;
   dim3 grid((unsigned)((p.cap + p.rows_per_cta - 1) / p.rows_per_cta), (unsigned)(p.B * p.Hkv), 1);
   return launch_pdl(kern, grid, dim3(kBuildThreads), smem, stream, p);
+}
+
+template <int D, int R>
+cudaError_t launch_dr(const ProjParams& p, cudaStream_t stream) {
+  return p.fp8 ? launch_drf<D, R, true>(p, stream) : launch_drf<D, R, false>(p, stream);
 }
 
 template <int D>

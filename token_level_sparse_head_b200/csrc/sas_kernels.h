@@ -19,7 +19,9 @@ constexpr int kDigit3Bits = 9;
 struct ProjParams {
   const __nv_bfloat16* K;      // build: cache (layout below); append: K_new [B][Hkv][d]
   const float* M;              // [Hkv][r][d]
-  __nv_bfloat16* Kproj;        // cache layout, width r
+  void* Kproj;                 // cache layout, width r: bf16 values or FP8 E4M3 codes
+  int fp8;                     // 1: write FP8 codes of (sum / kproj_scale[h])
+  const float* kproj_scale;    // [Hkv] (FP8)
   const int32_t* page_table;   // [B][max_pages] or null (contiguous)
   const int32_t* seqlens;      // [B]
   uint32_t* err;               // device error word or null
@@ -34,7 +36,9 @@ cudaError_t launch_proj(const ProjParams& p, cudaStream_t stream);
 struct ScoreParams {
   const __nv_bfloat16* q;      // [B][Hq][d]
   const float* M;              // [Hkv][r][d]
-  const __nv_bfloat16* kproj;  // cache layout, width r
+  const void* kproj;           // cache layout, width r: bf16 values or FP8 E4M3 codes
+  int fp8;                     // 1: FP8 codes, scored as kproj_scale[h] * code
+  const float* kproj_scale;    // [Hkv] (FP8)
   const int32_t* page_table;
   const int32_t* seqlens;
   const int32_t* kvec;         // [B]

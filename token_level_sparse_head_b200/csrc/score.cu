@@ -17,6 +17,9 @@
 // butterfly reduction, key, histogram) overlaps the copies of its next two and about 144 KB of
 // rows stay in flight per SM.  Full blocks take a path without per-row tests.  Keys go to the workspace with
 // an L2 evict-last hint so that the selection kernel finds them on chip.
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
+
 #include "sas_device.cuh"
 #include "sas_kernels.h"
 
@@ -32,17 +35,19 @@ constexpr int kDepth = 3;                  // ring slots per consumer warp
 constexpr int kSlots = kConsumerWarps * kDepth;
 static_assert(kSlots <= kProducerWarps * 32, "one producer lane per ring slot");
 
-template <int R>
+// Row geometry of the projected cache: bf16 (KP8 = false) or FP8 E4M3 codes (KP8 = true).
+template <int R, bool KP8>
 struct Geo {
-  static constexpr int ROW_BYTES = 2 * R;
-  static constexpr int BLOCK_ROWS = kBlockBytes / ROW_BYTES;  // 128 / 64 / 32 for r = 16 / 32 / 64
+  static constexpr int ROW_BYTES = KP8 ? R : 2 * R;
+  static constexpr int BLOCK_ROWS = kBlockBytes / ROW_BYTES;  // bf16: 128 / 64 / 32 for r = 16 / 32 / 64
   static constexpr int NB = BLOCK_ROWS / 32;                  // 32-row batches per block
   static constexpr int LG_BYTES = BLOCK_ROWS * 4;             // gate values of one block
   static constexpr int SLOT_BYTES = kBlockBytes + LG_BYTES;
-  static constexpr int LPR = R / 8;     // lanes per row, 16 bytes each
-  static constexpr int RPI = 32 / LPR;  // rows per load instruction
-  static constexpr int NI = LPR;        // load instructions per 32-row batch
-  static constexpr int LOG_LPR = LPR == 2 ? 1 : LPR == 4 ? 2 : 3;
+  static constexpr int CPL = KP8 ? 16 : 8;  // channels per 16-byte load
+  static constexpr int LPR = R / CPL;       // lanes per row
+  static constexpr int RPI = 32 / LPR;      // rows per load instruction
+  static constexpr int NI = LPR;            // load instructions per 32-row batch
+  static constexpr int LOG_LPR = LPR == 1 ? 0 : LPR == 2 ? 1 : LPR == 4 ? 2 : 3;
 };
 
 // Position of a CTA's share in the block list, computed once by the producer warp.
@@ -52,9 +57,9 @@ struct Plan {
   int h0, c0; // KV head and block index within it
 };
 
-template <int R, int D>
+template <int R, int D, bool KP8>
 struct Smem {
-  unsigned char ring[kSlots][Geo<R>::SLOT_BYTES];
+  unsigned char ring[kSlots][Geo<R, KP8>::SLOT_BYTES];
   uint32_t hist[kHistBins];
   float qbar[D];
   float qhat[R];
@@ -62,8 +67,9 @@ struct Smem {
   uint64_t empty[kSlots];
   Plan plan;
 };
-static_assert(sizeof(Smem<16, 128>) <= 227 * 1024 && sizeof(Smem<32, 128>) <= 227 * 1024 &&
-                  sizeof(Smem<64, 128>) <= 227 * 1024,
+static_assert(sizeof(Smem<16, 128, false>) <= 227 * 1024 && sizeof(Smem<32, 128, false>) <= 227 * 1024 &&
+                  sizeof(Smem<64, 128, false>) <= 227 * 1024 && sizeof(Smem<16, 128, true>) <= 227 * 1024 &&
+                  sizeof(Smem<32, 128, true>) <= 227 * 1024 && sizeof(Smem<64, 128, true>) <= 227 * 1024,
               "score kernel shared memory");
 
 __device__ __forceinline__ void stg_hint(uint32_t* ptr, uint32_t v, uint64_t pol) {
@@ -83,6 +89,21 @@ __device__ __forceinline__ float dot8(const float2 (&qv)[4], uint4 w) {
   a = ffma2(qv[1], make_float2(bf16lo(w.y), bf16hi(w.y)), a);
   a = ffma2(qv[2], make_float2(bf16lo(w.z), bf16hi(w.z)), a);
   a = ffma2(qv[3], make_float2(bf16lo(w.w), bf16hi(w.w)), a);
+  return a.x + a.y;
+}
+
+// Dot product of 16 FP8 E4M3 codes (one 16-byte chunk of a row, code 2i in the low byte of
+// each 16-bit half) with this lane's 16 channels of q-hat (already times the head's scale).
+__device__ __forceinline__ float dot16_fp8(const float2 (&qv)[8], uint4 w) {
+  const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+  float2 a = make_float2(0.f, 0.f);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const __half2_raw lo = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(ws[i] & 0xffffu), __NV_E4M3);
+    const __half2_raw hi = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(ws[i] >> 16), __NV_E4M3);
+    a = ffma2(qv[2 * i], __half22float2(__half2(lo)), a);
+    a = ffma2(qv[2 * i + 1], __half22float2(__half2(hi)), a);
+  }
   return a.x + a.y;
 }
 
@@ -137,12 +158,12 @@ __device__ __forceinline__ void next_scored_seq(const ScoreParams& p, int& b, Se
   while (b < p.B && (si = seq_info<BR>(p, b, false)).blocks == 0) ++b;
 }
 
-template <int R, int D, bool GATED>
+template <int R, int D, bool GATED, bool KP8>
 __global__ void __launch_bounds__(kThreads, 1) score_kernel(const ScoreParams p) {
-  using Gm = Geo<R>;
+  using Gm = Geo<R, KP8>;
   constexpr int BR = Gm::BLOCK_ROWS;
   extern __shared__ __align__(128) unsigned char smem_raw[];
-  Smem<R, D>& S = *reinterpret_cast<Smem<R, D>*>(smem_raw);
+  Smem<R, D, KP8>& S = *reinterpret_cast<Smem<R, D, KP8>*>(smem_raw);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 
   if (tid == 0) {
@@ -288,7 +309,7 @@ __global__ void __launch_bounds__(kThreads, 1) score_kernel(const ScoreParams p)
   const uint64_t pol_keep = l2_evict_last();
   const int part = lane % Gm::LPR;  // this lane's 16-byte chunk of each row it loads
   const int rsub = lane / Gm::LPR;  // its row within each load instruction
-  float2 qv[4];
+  float2 qv[Gm::CPL / 2];
   int cur_bh = -1;
   bool cur_ranked = false;
 
@@ -332,10 +353,12 @@ __global__ void __launch_bounds__(kThreads, 1) score_kernel(const ScoreParams p)
       for (int i = 0; i < CH; ++i) sp = fmaf(mreg[i], S.qbar[qpart * CH + i], sp);
 #pragma unroll
       for (int o = TPR / 2; o; o >>= 1) sp += __shfl_xor_sync(0xffffffffu, sp, o);
-      if (qpart == 0 && qrow) S.qhat[qj] = sp * p.sigma;
+      // FP8: the head's scale multiplies q-hat, so the codes are used as they are
+      if (qpart == 0 && qrow) S.qhat[qj] = sp * p.sigma * (KP8 ? p.kproj_scale[h] : 1.f);
       consumers_sync();
 #pragma unroll
-      for (int e = 0; e < 4; ++e) qv[e] = make_float2(S.qhat[part * 8 + 2 * e], S.qhat[part * 8 + 2 * e + 1]);
+      for (int e = 0; e < Gm::CPL / 2; ++e)
+        qv[e] = make_float2(S.qhat[part * Gm::CPL + 2 * e], S.qhat[part * Gm::CPL + 2 * e + 1]);
       cur_bh = bh;
       cur_ranked = si.ranked;
     }
@@ -358,7 +381,7 @@ __global__ void __launch_bounds__(kThreads, 1) score_kernel(const ScoreParams p)
 #pragma unroll
           for (int i = 0; i < Gm::NI; ++i) {
             const uint4 w = *reinterpret_cast<const uint4*>(sb + (size_t)(i * Gm::RPI + rsub) * Gm::ROW_BYTES + part * 16);
-            v[i] = dot8(qv, w);
+            if constexpr (KP8) v[i] = dot16_fp8(qv, w); else v[i] = dot8(qv, w);
           }
           const float u0 = butterfly<Gm>(v, lane);
           const int lr = part * Gm::RPI + rsub;
@@ -381,7 +404,7 @@ __global__ void __launch_bounds__(kThreads, 1) score_kernel(const ScoreParams p)
               const int lr = i * Gm::RPI + rsub;
               uint4 w = make_uint4(0u, 0u, 0u, 0u);
               if (lr < wrows) w = *reinterpret_cast<const uint4*>(sb + (size_t)lr * Gm::ROW_BYTES + part * 16);
-              v[i] = dot8(qv, w);
+              if constexpr (KP8) v[i] = dot16_fp8(qv, w); else v[i] = dot8(qv, w);
             }
             const float u0 = butterfly<Gm>(v, lane);
             const int lr = part * Gm::RPI + rsub;
@@ -422,8 +445,10 @@ __global__ void __launch_bounds__(kThreads, 1) score_kernel(const ScoreParams p)
 
 template <int R, int D>
 cudaError_t launch_rd(const ScoreParams& p, cudaStream_t stream) {
-  const int smem = (int)sizeof(Smem<R, D>);
-  auto kern = p.log_g != nullptr ? score_kernel<R, D, true> : score_kernel<R, D, false>;
+  const bool gated = p.log_g != nullptr;
+  const int smem = p.fp8 ? (int)sizeof(Smem<R, D, true>) : (int)sizeof(Smem<R, D, false>);
+  auto kern = p.fp8 ? (gated ? score_kernel<R, D, true, true> : score_kernel<R, D, false, true>)
+                    : (gated ? score_kernel<R, D, true, false> : score_kernel<R, D, false, false>);
   cudaError_t e = prepare_kernel((const void*)kern, smem);
   if (e != cudaSuccess) return e;
   return launch_pdl(kern, dim3((unsigned)p.ctas), dim3(kThreads), (size_t)smem, stream, p);
@@ -433,7 +458,7 @@ cudaError_t launch_rd(const ScoreParams& p, cudaStream_t stream) {
 
 void plan_score(ScoreParams& p, int num_sms) {
   // Persistent: one CTA per SM, never more CTAs than there can be blocks.
-  const int br = kBlockBytes / (2 * p.r);
+  const int br = kBlockBytes / ((p.fp8 ? 1 : 2) * p.r);
   const long long blocks = (long long)p.B * p.Hkv * ((p.cap + br - 1) / br);
   long long ctas = num_sms;
   if (ctas > blocks) ctas = blocks;

@@ -25,7 +25,10 @@ _vp, _i32, _f32, _sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_float, ctypes.c
 class sas_shape(ctypes.Structure):
     _fields_ = [("B", _i32), ("Hq", _i32), ("Hkv", _i32), ("d", _i32), ("r", _i32),
                 ("n_cap", _i32), ("page_size", _i32), ("max_pages", _i32), ("num_pages", _i32),
-                ("kproj_dtype", _i32)]
+                ("kproj_dtype", _i32), ("kproj_scale", _vp)]
+
+
+SAS_KPROJ_BF16, SAS_KPROJ_FP8_E4M3 = 0, 1
 
 
 _SIGS = {
@@ -121,10 +124,11 @@ class Shape:
     max_pages: int = 0
     num_pages: int = 0
     kproj_dtype: int = 0
+    kproj_scale: Optional[object] = None  # device fp32 [Hkv] (tensor or pointer) for FP8
 
     def c(self) -> sas_shape:
         return sas_shape(self.B, self.Hq, self.Hkv, self.d, self.r, self.n_cap, self.page_size,
-                         self.max_pages, self.num_pages, self.kproj_dtype)
+                         self.max_pages, self.num_pages, self.kproj_dtype, _p(self.kproj_scale))
 
     @property
     def cap(self) -> int:
@@ -133,10 +137,12 @@ class Shape:
 
 def shape_of(problem) -> Shape:
     """Shape of a synth.DecodeProblem-like object (fields B, Hq, Hkv, d, r, paged, ...)."""
+    scale = getattr(problem, "kproj_scale", None)
+    dt = SAS_KPROJ_FP8_E4M3 if scale is not None else SAS_KPROJ_BF16
     if problem.paged:
         return Shape(problem.B, problem.Hq, problem.Hkv, problem.d, problem.r, 0, PAGE_SIZE,
-                     problem.max_pages, problem.num_pages)
-    return Shape(problem.B, problem.Hq, problem.Hkv, problem.d, problem.r, problem.n_cap)
+                     problem.max_pages, problem.num_pages, dt, scale)
+    return Shape(problem.B, problem.Hq, problem.Hkv, problem.d, problem.r, problem.n_cap, 0, 0, 0, dt, scale)
 
 
 # ------------------------------------------------------------------------------ entry points
