@@ -354,6 +354,45 @@ def run_ours(args):
     achieved = dom_bytes / (k_ms[dom] * 1e-3) / 1e9
     traffic = recorded_traffic({"score": "score.cu", "select": "select.cu", "attend": "attend.cu"}[dom], args.workload)
 
+    # --- gather-then-attend foil on the same selected rows: copy the rows, then dense decode
+    foil = None
+    if not args.no_foil:
+        from token_level_sparse_head_b200 import DecodeSession, lib as L
+
+        Kg = torch.empty(p.B, p.Hkv, p.k_max, p.d, dtype=torch.bfloat16, device=dev)
+        Vg = torch.empty_like(Kg)
+        counts = torch.empty(p.B, dtype=torch.int32, device=dev)
+        gshape = L.Shape(p.B, p.Hq, p.Hkv, p.d, p.r, p.k_max)
+        gsess = DecodeSession(gshape, p.k_max, device=dev)
+        gout = torch.empty_like(wl.sess.out)
+        idx_sel = wl.sess.idx
+
+        def gather():
+            L.sas_gather_selected(wl.shape, p.K, p.V, p.page_table, p.seqlens, idx_sel, p.k, p.k_max, Kg, Vg, counts)
+
+        def attend_gathered():
+            gsess.dense(p.q, Kg, Vg, None, counts, out=gout)
+
+        nf = max(5, min(args.steps, 100))
+        evf = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(nf)]
+        for _ in range(3):
+            gather()
+            attend_gathered()
+        torch.cuda.synchronize()
+        for i in range(nf):
+            evf[i][0].record()
+            gather()
+            evf[i][1].record()
+            attend_gathered()
+            evf[i][2].record()
+        torch.cuda.synchronize()
+        g_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evf)
+        a_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evf)
+        foil = {"gather_ms": g_ms, "attend_gathered_ms": a_ms, "total_ms": g_ms + a_ms,
+                "gather_free_attend_ms": k_ms["attend"], "gather_free_speedup": (g_ms + a_ms) / k_ms["attend"],
+                "note": "same selected rows; gather copies them to a contiguous buffer, then dense decode"}
+        del Kg, Vg, gsess
+
     # --- dense full-KV baseline on the same workload
     for _ in range(2):
         wl.dense()
@@ -468,6 +507,8 @@ def run_ours(args):
         line["b1"] = secondary
     if fp8:
         line["fp8_kproj"] = fp8
+    if foil:
+        line["gather_foil"] = foil
     print(json.dumps(line), flush=True)
 
 
@@ -579,6 +620,7 @@ def main():
     ap.add_argument("--no-secondary", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-fp8", action="store_true", help="skip the FP8 projected-cache line")
+    ap.add_argument("--no-foil", action="store_true", help="skip the gather-then-attend line")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     args = ap.parse_args()
     if args.warmup < 3:

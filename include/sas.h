@@ -206,6 +206,22 @@ sas_status sas_dense_decode(const sas_shape* shape, const void* q, const void* K
                             const int32_t* page_table, const int32_t* seqlens, float* out,
                             void* workspace, size_t ws_bytes, void* stream);
 
+/* Gather of the selected rows, for measuring the gather-then-attend alternative (not part of
+ * the decode step): copies the K and V rows at the first min(k_b, N_b) entries of every
+ * (b, h) index list into contiguous buffers -- the staging copy a gather-based sparse
+ * attention makes and sas_sparse_attention avoids (JSSA page, section gather 到底贵在哪).
+ * sas_dense_decode over the gathered rows (a contiguous shape with n_cap = k_max and seqlens =
+ * counts) then computes what sas_sparse_attention computes without a gate.
+ *   idx     int32 [B][Hkv][k_max] (device), as written by the selection; entries outside
+ *           [0, N_b) read position 0
+ *   Kg, Vg  bf16 [B][Hkv][k_max][d] (device), written for the first counts[b] rows
+ *   counts  int32 [B] (device), written: min(k_b, k_max, N_b)
+ */
+sas_status sas_gather_selected(const sas_shape* shape, const void* K, const void* V,
+                               const int32_t* page_table, const int32_t* seqlens,
+                               const int32_t* idx, const int32_t* k, int32_t k_max, void* Kg,
+                               void* Vg, int32_t* counts, void* stream);
+
 /* Bytes of the library's fixed scratch array (16 MiB), used by sas_decode_step_static_scratch. */
 #define SAS_STATIC_SCRATCH_BYTES (16u << 20)
 

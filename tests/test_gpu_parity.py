@@ -172,6 +172,49 @@ def test_fp8_append_matches_build(cuda_lib):
         assert int(kp_build.count_nonzero()) > 0
 
 
+# ------------------------------------------------------------- gather-then-attend (the foil)
+@pytest.mark.parametrize("paged", [False, True])
+def test_gather_then_dense_matches_gather_free(cuda_lib, paged):
+    """Gathering the selected rows and running the dense decode over them gives the outputs of
+    the gather-free attention (and of the oracle on the same rows)."""
+    from oracle import sas_oracle as O
+    from tests.helpers import check_output, f64
+    from token_level_sparse_head_b200 import DecodeSession, lib, shape_of
+
+    p = make_problem(B=3, Hq=8, Hkv=2, d=128, r=32, seqlens=[5000, 777, 1], k=[300, 900, 5], k_max=900,
+                     paged=paged, n_cap=None if paged else 5004, basis="qr", aniso=True, seed=31).to("cuda")
+    shape = shape_of(p)
+    kshp = (p.num_pages, p.Hkv, 64, p.r) if paged else (p.B, p.Hkv, p.n_cap, p.r)
+    kp = torch.zeros(kshp, dtype=torch.bfloat16, device="cuda")
+    lib.sas_build_proj_cache(shape, p.K, p.M, kp, p.page_table, p.seqlens)
+    sess = DecodeSession(shape, p.k_max)
+    out_free, idx = sess.decode(p.q, p.M, kp, p.K, p.V, p.page_table, p.seqlens, p.k)
+    Kg = torch.zeros(p.B, p.Hkv, p.k_max, p.d, dtype=torch.bfloat16, device="cuda")
+    Vg = torch.zeros_like(Kg)
+    counts = torch.full((p.B,), -1, dtype=torch.int32, device="cuda")
+    lib.sas_gather_selected(shape, p.K, p.V, p.page_table, p.seqlens, idx, p.k, p.k_max, Kg, Vg, counts)
+    gshape = lib.Shape(p.B, p.Hq, p.Hkv, p.d, p.r, p.k_max)
+    gsess = DecodeSession(gshape, p.k_max)
+    out_g = gsess.dense(p.q, Kg, Vg, None, counts, out=torch.empty_like(out_free))
+    torch.cuda.synchronize()
+    assert counts.tolist() == [300, 777, 1]
+    G = p.Hq // p.Hkv
+    of, og, ix = f64(out_free), f64(out_g), f64(idx)
+    sigma = O.softmax_scale(p.d)
+    for b in range(p.B):
+        c = int(counts[b])
+        for h in range(p.Hkv):
+            sel = ix[b, h, :c]
+            kr, vr = f64(Kg[b, h, :c]), f64(Vg[b, h, :c])
+            ref = O.sparse_attention(f64(p.q[b, h * G:(h + 1) * G]), kr, vr, sigma)
+            check_output(og[b, h * G:(h + 1) * G], ref, f"gathered (b={b},h={h})")
+            check_output(of[b, h * G:(h + 1) * G], ref, f"gather-free (b={b},h={h})")
+            # the gathered rows are the cache rows at the selected positions
+            n = int(p.seqlens[b])
+            rows = O.logical_rows(f64(p.K), b, h, n, None if p.page_table is None else f64(p.page_table))
+            assert np.array_equal(kr, rows[sel])
+
+
 # ------------------------------------------------------------------------ full-size workloads
 def _heads(B, Hkv):
     pairs = {(0, 0), (B - 1, Hkv - 1), (B // 2, Hkv // 2)}

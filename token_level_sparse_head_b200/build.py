@@ -21,7 +21,7 @@ INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libsas.so")
 
-SOURCES = ["api.cu", "proj.cu", "score.cu", "select.cu", "attend.cu"]
+SOURCES = ["api.cu", "proj.cu", "score.cu", "select.cu", "attend.cu", "gather.cu"]
 HEADERS = ["sas_device.cuh", "sas_kernels.h"]
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

@@ -487,6 +487,36 @@ sas_status sas_dense_decode(const sas_shape* shape, const void* q, const void* K
                    workspace, static_cast<cudaStream_t>(stream));
 }
 
+sas_status sas_gather_selected(const sas_shape* shape, const void* K, const void* V, const int32_t* page_table,
+                               const int32_t* seqlens, const int32_t* idx, const int32_t* k, int32_t k_max,
+                               void* Kg, void* Vg, int32_t* counts, void* stream) {
+  SAS_TRY(check_shape(shape));
+  if (k_max < 1) return fail(SAS_ERR_INVALID_ARG, "k_max must be >= 1");
+  SAS_TRY(check_ptr(K, "K"));
+  SAS_TRY(check_ptr(V, "V"));
+  SAS_TRY(check_ptr(idx, "idx"));
+  SAS_TRY(check_ptr(k, "k"));
+  SAS_TRY(check_ptr(Kg, "Kg"));
+  SAS_TRY(check_ptr(Vg, "Vg"));
+  SAS_TRY(check_ptr(counts, "counts"));
+  SAS_TRY(check_cache_ptrs(shape, page_table, seqlens));
+  sas::GatherParams p = {};
+  p.K = static_cast<const __nv_bfloat16*>(K);
+  p.V = static_cast<const __nv_bfloat16*>(V);
+  p.page_table = shape->page_size ? page_table : nullptr;
+  p.seqlens = seqlens;
+  p.idx = idx;
+  p.kvec = k;
+  p.Kg = static_cast<__nv_bfloat16*>(Kg);
+  p.Vg = static_cast<__nv_bfloat16*>(Vg);
+  p.counts = counts;
+  p.B = shape->B; p.Hkv = shape->Hkv; p.d = shape->d; p.cap = cap_of(shape);
+  p.max_pages = shape->max_pages; p.num_pages = shape->num_pages; p.paged = shape->page_size ? 1 : 0;
+  p.k_max = k_max;
+  const cudaError_t e = sas::launch_gather(p, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? SAS_OK : cuda_fail(e, "gather kernel launch");
+}
+
 }  // extern "C"
 
 // ---------------------------------------------------------------------------------------------

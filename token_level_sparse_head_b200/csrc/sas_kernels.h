@@ -72,6 +72,21 @@ struct SelectParams {
 bool plan_select(SelectParams& p, int num_sms);
 cudaError_t launch_select(const SelectParams& p, cudaStream_t stream);
 
+// ---------------------------------------------------------------------------- gather (foil)
+struct GatherParams {
+  const __nv_bfloat16* K;      // cache layout
+  const __nv_bfloat16* V;
+  const int32_t* page_table;
+  const int32_t* seqlens;
+  const int32_t* idx;          // [B][Hkv][k_max]
+  const int32_t* kvec;         // [B]
+  __nv_bfloat16* Kg;           // [B][Hkv][k_max][d]
+  __nv_bfloat16* Vg;
+  int32_t* counts;             // [B]
+  int B, Hkv, d, cap, max_pages, num_pages, paged, k_max;
+};
+cudaError_t launch_gather(const GatherParams& p, cudaStream_t stream);
+
 // ---------------------------------------------------------------------------- attention
 struct AttendParams {
   const __nv_bfloat16* q;      // [B][Hq][d]

@@ -55,6 +55,8 @@ _SIGS = {
                                         _sz, _vp]),
     "sas_decode_step_static_scratch": (ctypes.c_int, [ctypes.POINTER(sas_shape), _vp, _vp, _vp, _vp, _vp, _vp,
                                                       _vp, _vp, _i32, _f32, _vp, _vp, _vp, _vp]),
+    "sas_gather_selected": (ctypes.c_int, [ctypes.POINTER(sas_shape), _vp, _vp, _vp, _vp, _vp, _vp, _i32, _vp, _vp,
+                                           _vp, _vp]),
 }
 STATIC_SCRATCH_BYTES = 16 << 20  # SAS_STATIC_SCRATCH_BYTES
 EXPORTED = tuple(_SIGS)
@@ -233,3 +235,10 @@ def sas_decode_step_static_scratch(shape: Shape, q, M, Kproj, K, V, page_table, 
                                                  _p(page_table), _p(seqlens), _p(k), int(k_max), float(lam),
                                                  _p(log_g), _p(out), _p(idx_out), _stream(stream)),
            "sas_decode_step_static_scratch")
+
+
+def sas_gather_selected(shape: Shape, K, V, page_table, seqlens, idx, k, k_max: int, Kg, Vg, counts, stream=None):
+    """Copies the selected K/V rows into contiguous buffers (the gather-then-attend foil)."""
+    _check(load().sas_gather_selected(ctypes.byref(shape.c()), _p(K), _p(V), _p(page_table), _p(seqlens), _p(idx),
+                                      _p(k), int(k_max), _p(Kg), _p(Vg), _p(counts), _stream(stream)),
+           "sas_gather_selected")
