@@ -12,6 +12,8 @@ from .lib import (  # noqa: F401
     sas_decode_workspace_bytes,
     sas_dense_decode,
     sas_dense_workspace_bytes,
+    sas_decode_step_static_scratch,
+    sas_gather_selected,
     sas_score_scan,
     sas_select_from_scores,
     sas_select_topk,
@@ -19,3 +21,4 @@ from .lib import (  # noqa: F401
     sas_workspace_init,
 )
 from .session import DecodeSession  # noqa: F401
+from .calibrate import MomentAccumulator, calibrate, scoring_basis  # noqa: F401
