@@ -282,6 +282,28 @@ def flushed_steps(torch, fn, steps, flush_buf):
     return statistics.median(ts)
 
 
+def selection_recall(torch, wl):
+    """Mean over (sequence, KV head) of |projected top-k  ∩  exact top-k| / k, where the exact
+    set ranks the full-dimension score q-bar . k_i (contiguous caches; a report, not a check)."""
+    p = wl.p
+    if p.paged:
+        return None
+    G = p.Hq // p.Hkv
+    idx = wl.sess.idx
+    rec = []
+    for b in range(p.B):
+        n = int(wl.seqlens_h[b])
+        k = min(int(wl.ks_h[b]), n)
+        if k <= 0 or k >= n:
+            continue
+        for h in range(p.Hkv):
+            qbar = p.q[b, h * G:(h + 1) * G].float().mean(0)
+            exact = torch.topk(p.K[b, h, :n].float() @ qbar, k).indices
+            sel = idx[b, h, :k].long()
+            rec.append(float(torch.isin(sel, exact).sum()) / k)
+    return statistics.mean(rec) if rec else None
+
+
 def capture_graph(torch, fn):
     """fn captured into a CUDA graph (the library's calls allocate nothing and never synchronise,
     so a step can be captured as it is); None if capture is not possible here."""
@@ -353,6 +375,8 @@ def run_ours(args):
     head_dense_bytes = wl.dense_bytes
     achieved = dom_bytes / (k_ms[dom] * 1e-3) / 1e9
     traffic = recorded_traffic({"score": "score.cu", "select": "select.cu", "attend": "attend.cu"}[dom], args.workload)
+
+    recall = selection_recall(torch, wl)
 
     # --- gather-then-attend foil on the same selected rows: copy the rows, then dense decode
     foil = None
@@ -471,6 +495,7 @@ def run_ours(args):
                "hbm_gbs": w8.bytes["step"] / (ms8 * 1e-3) / 1e9, "step_bytes": w8.bytes["step"],
                "speedup_vs_bf16_kproj": ms / ms8, "kernels_ms": k8,
                "score_hbm_gbs": w8.bytes["score"] / (k8["score"] * 1e-3) / 1e9,
+               "selection_recall": selection_recall(torch, w8),
                "timing": "CUDA graph replay of the step" if g8 is not None else "stream launches"}
         wl = w8
 
@@ -509,6 +534,9 @@ def run_ours(args):
         line["fp8_kproj"] = fp8
     if foil:
         line["gather_foil"] = foil
+    line["selection_recall"] = {"value": recall, "definition": "mean over (sequence, KV head) of the fraction of "
+                                "the exact top-k by q-bar . k_i (full dimension) that the projected selection keeps; "
+                                "synthetic data"}
     print(json.dumps(line), flush=True)
 
 
