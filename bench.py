@@ -282,14 +282,15 @@ def flushed_steps(torch, fn, steps, flush_buf):
     return statistics.median(ts)
 
 
-def selection_recall(torch, wl):
-    """Mean over (sequence, KV head) of |projected top-k  ∩  exact top-k| / k, where the exact
-    set ranks the full-dimension score q-bar . k_i (contiguous caches; a report, not a check)."""
+def selection_recall(torch, wl, gate=True):
+    """Oracle top-k recall of the selection the last step made: the mean over (sequence, KV head)
+    of |selected set  ∩  exact top-k| / k, where the exact set ranks the full-dimension key
+    sigma * q-bar . k_i (+ lambda * log g_i when `gate` and the workload is gated).  Sequences
+    whose budget covers them are skipped.  A report, not a check."""
     p = wl.p
-    if p.paged:
-        return None
     G = p.Hq // p.Hkv
     idx = wl.sess.idx
+    lam = float(getattr(p, "lam", 0.0) or 0.0)
     rec = []
     for b in range(p.B):
         n = int(wl.seqlens_h[b])
@@ -297,11 +298,41 @@ def selection_recall(torch, wl):
         if k <= 0 or k >= n:
             continue
         for h in range(p.Hkv):
+            if p.paged:
+                pages = p.page_table[b, :(n + 63) // 64].long()
+                rows = p.K[pages, h].reshape(-1, p.K.shape[-1])[:n]
+            else:
+                rows = p.K[b, h, :n]
             qbar = p.q[b, h * G:(h + 1) * G].float().mean(0)
-            exact = torch.topk(p.K[b, h, :n].float() @ qbar, k).indices
+            key = (rows.float() @ qbar) / math.sqrt(rows.shape[-1])
+            if gate and lam != 0.0:
+                key = key + lam * p.log_g[b, h, :n].float()
+            exact = torch.topk(key, k).indices
             sel = idx[b, h, :k].long()
             rec.append(float(torch.isin(sel, exact).sum()) / k)
     return statistics.mean(rec) if rec else None
+
+
+def run_recall_report(args):
+    """One line per named workload: the oracle top-k recall of one decode step's selection."""
+    import torch
+
+    from synth import CONFIGS
+
+    torch.cuda.set_device(0)
+    for name in CONFIGS:
+        wl = Workload(name, "cuda:0", torch)
+        wl.step()
+        torch.cuda.synchronize()
+        p = wl.p
+        line = {"report": "selection_recall", "workload": name, "B": p.B, "N_max": max(wl.seqlens_h),
+                "k_max": p.k_max, "r": p.r, "d": p.d, "lam": p.lam, "fp8_kproj": wl.fp8,
+                "recall": selection_recall(torch, wl)}
+        if p.lam:
+            line["recall_vs_ungated_score"] = selection_recall(torch, wl, gate=False)
+        print(json.dumps(line), flush=True)
+        wl.free()
+        del wl
 
 
 def capture_graph(torch, fn):
@@ -650,10 +681,14 @@ def main():
     ap.add_argument("--no-fp8", action="store_true", help="skip the FP8 projected-cache line")
     ap.add_argument("--no-foil", action="store_true", help="skip the gather-then-attend line")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--recall-report", action="store_true",
+                    help="print the selection recall of every named workload instead of timing")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
-    if args.impl == "reference":
+    if args.recall_report:
+        run_recall_report(args)
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_ours(args)
