@@ -9,9 +9,10 @@
 // each CTA owns a contiguous chunk of positions.  The k-th largest key T is found as three radix
 // digits (13, 10 and 9 bits); ties on T go to the lower positions.
 //   1. The global histogram gives digit 1.  Each CTA streams its chunk of keys once through a
-//      shared-memory ring (bulk copies; one ballot per 32 keys is a bitmap word), setting a position bitmap of the keys whose digit 1 is
-//      larger (they are selected) and appending the keys whose digit 1 equals it (the
-//      candidates, a few percent of the positions) to a list.
+//      shared-memory ring (bulk copies; each lane turns 4 keys into 4 bits of a bitmap word),
+//      setting a position bitmap of the keys whose digit 1 is larger (they are selected) and
+//      appending the keys whose digit 1 equals it (the candidates, a few percent of the
+//      positions) to a list.
 //   2. The candidate lists are gathered into CTA 0 of the cluster through distributed shared
 //      memory; CTA 0 finds digits 2 and 3 among them, resolves the ties, marks the chosen
 //      candidates in the owners' bitmaps and hands every CTA its first output slot.
@@ -271,28 +272,39 @@ __global__ void __launch_bounds__(kThreads, 1) select_topk_kernel(const SelectPa
     for (int s = 0; s < nst; ++s) {
       const int slot = s % kStages;
       if (!mbar_wait_bounded(&S.full[slot], (uint32_t)(s / kStages) & 1u)) waited_ok = false;
-      // the warp's 128 keys as 4 words of 32: lane l holds key 32 e + l of word e, so a ballot
-      // is a bitmap word
-      const uint32_t* st = S.ring[slot] + warp * 128;
-      const int lp = s * kStageKeys + warp * 128 + lane;  // chunk position of key e = 0
+      // the warp's 128 keys: lane l takes keys 4l .. 4l+3 (one 16-byte read) and forms their
+      // 4 bits; the 8 lanes of a bitmap word combine their nibbles with three shuffles
+      const uint4 kv = reinterpret_cast<const uint4*>(S.ring[slot] + warp * 128)[lane];
+      const int lp = s * kStageKeys + warp * 128 + 4 * lane;  // chunk position of the lane's first key
       const int wbase = s * (kStageKeys / 32) + warp * 4;
-      const bool full_stage = (s + 1) * kStageKeys <= len;
+      const uint32_t kk[4] = {kv.x, kv.y, kv.z, kv.w};
+      uint32_t ab = 0u, cb = 0u;
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const uint32_t key = st[e * 32 + lane];
-        const bool valid = full_stage || lp + e * 32 < len;
-        const uint32_t ab = __ballot_sync(0xffffffffu, valid && key > hi);
-        const uint32_t cb = __ballot_sync(0xffffffffu, valid && key - lo <= hi - lo);
-        if (lane == e) S.bm[wbase + e] = ab;
-        my_above += (lane == e) ? (uint32_t)__popc(ab) : 0u;
-        if (cb) {
-          uint32_t base = 0u;
-          if (lane == 0) base = atomicAdd(&S.ctl.ccount, (uint32_t)__popc(cb));
-          base = __shfl_sync(0xffffffffu, base, 0);
-          const uint32_t j = base + (uint32_t)__popc(cb & ((1u << lane) - 1u));
-          if (((cb >> lane) & 1u) && j < (uint32_t)kCap) {
-            S.ckey[j] = key;
-            S.cpos[j] = c0 + lp + e * 32;
+      for (int j = 0; j < 4; ++j) {
+        ab |= (kk[j] > hi ? 1u : 0u) << j;
+        cb |= (kk[j] - lo <= hi - lo ? 1u : 0u) << j;
+      }
+      if ((s + 1) * kStageKeys > len) {  // the last, partial stage: drop keys past the chunk
+        const uint32_t vm = (1u << min(max(len - lp, 0), 4)) - 1u;
+        ab &= vm;
+        cb &= vm;
+      }
+      uint32_t word = ab << (4 * (lane & 7));
+      word |= __shfl_xor_sync(0xffffffffu, word, 1);
+      word |= __shfl_xor_sync(0xffffffffu, word, 2);
+      word |= __shfl_xor_sync(0xffffffffu, word, 4);
+      if ((lane & 7) == 0) S.bm[wbase + (lane >> 3)] = word;
+      my_above += (uint32_t)__popc(ab);
+      if (cb) {
+        uint32_t j = atomicAdd(&S.ctl.ccount, (uint32_t)__popc(cb));
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          if ((cb >> e) & 1u) {
+            if (j < (uint32_t)kCap) {
+              S.ckey[j] = kk[e];
+              S.cpos[j] = c0 + lp + e;
+            }
+            ++j;
           }
         }
       }
