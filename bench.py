@@ -35,6 +35,9 @@ L2_BYTES = 126 * 1024 * 1024
 
 
 # ------------------------------------------------------------------------------ accounting
+NOMINAL_HBM_GBS = 8000.0
+
+
 def roofline_bytes(B, Hq, Hkv, d, r, seqlens, ks, lam, kp_bytes=2):
     """Algorithmic HBM bytes of one step, per kernel and in total.
 
@@ -558,6 +561,8 @@ def run_ours(args):
     }
     line["hbm_gbs"] = head_bytes["step"] / (ms * 1e-3) / 1e9
     line["step_roofline_frac"] = line["hbm_gbs"] / peak
+    # the same step against the nominal B200 HBM3e figure (about 8 TB/s), for context
+    line["step_frac_of_nominal_8tbs"] = line["hbm_gbs"] / NOMINAL_HBM_GBS
     line["dense"]["hbm_gbs"] = head_dense_bytes / (dense_ms * 1e-3) / 1e9
     if secondary:
         line["b1"] = secondary
