@@ -662,7 +662,7 @@ def run_reference(args):
     value = 1.0 / (per_head * heads_per_step)
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": per_head * heads_per_step * 1e3,
+        "steps": len(ts), "warmup": args.warmup, "ms_per_step": per_head * heads_per_step * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic", "config": dict(workload=args.workload, **CONFIGS_VIEW(args.workload)),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": _threads_used(), "kind": "oracle",
