@@ -64,6 +64,7 @@ struct SelectParams {
   uint32_t* err;
   int B, Hkv, cap, k_max;
   int cluster;                 // CTAs per (b, h)
+  int threads;                 // threads per CTA (512 or 1024)
   int chunk;                   // max positions per CTA (multiple of 512)
   int cand_cap;                // candidate list capacity per CTA
   int off_hist, off_ctl, smem_bytes;

@@ -29,12 +29,8 @@ namespace cg = cooperative_groups;
 namespace sas {
 namespace {
 
-constexpr int kThreads = 1024;
-constexpr int kWarps = kThreads / 32;
 constexpr int kBins2 = 1 << kDigit2Bits;      // 1024
 constexpr int kBins3 = 1 << kDigit3Bits;      // 512
-constexpr int kStageKeys = kWarps * 128;      // keys per ring stage: 4 per lane
-constexpr int kStages = 8;
 constexpr int kChunkMax = 131072;             // positions per CTA at most
 constexpr int kMaxWords = kChunkMax / 32;     // bitmap words per CTA
 constexpr int kCap = 4096;                    // candidate list entries (CTA 0: the whole head's)
@@ -58,8 +54,22 @@ struct Ctl {
   uint32_t tie_of[kMaxCluster];
 };
 
+// Block shape: THREADS threads per CTA, and a ring of 128 KB of keys in stages of 4 keys per
+// thread.  1024 threads serve a head per CTA (B=16); clusters of several CTAs per head (small
+// batches) use 512, which spend less time in block-wide barriers.
+template <int THREADS>
+struct Cfg {
+  static constexpr int kThreads = THREADS;
+  static constexpr int kWarps = THREADS / 32;
+  static constexpr int kStageKeys = kWarps * 128;  // keys per ring stage: 4 per lane
+  static constexpr int kStages = 8 * 1024 / THREADS;
+};
+
+template <int THREADS>
 struct SelSmem {
-  uint32_t ring[kStages][kStageKeys];
+  static constexpr int kStages = Cfg<THREADS>::kStages;
+  static constexpr int kWarps = Cfg<THREADS>::kWarps;
+  uint32_t ring[kStages][Cfg<THREADS>::kStageKeys];
   uint32_t bm[kMaxWords];     // selected positions of the chunk
   uint32_t ckey[kCap];        // candidate keys (slow path: tie bits per bitmap word)
   int32_t cpos[kCap];         // candidate positions in the head
@@ -75,7 +85,9 @@ struct SelSmem {
 };
 
 // Exclusive prefix sum over the block; *total receives the block sum.
+template <int THREADS>
 __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t* wsum, uint32_t* total) {
+  constexpr int kWarps = THREADS / 32;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   uint32_t x = v;
 #pragma unroll
@@ -102,8 +114,9 @@ __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t* wsum, 
 // covers digits [NB - (t+1)*PER, NB - t*PER), highest first (threads past NB / PER hold none).
 // Writes *out (digit, count above it, count in it); out is left unchanged if the histogram
 // holds fewer keys.
-template <int NB>
+template <int NB, int THREADS>
 __device__ __forceinline__ void find_digit(const uint32_t* H, uint32_t k_rem, uint32_t* wsum, Found* out) {
+  constexpr int kThreads = THREADS;
   constexpr int PER = NB >= kThreads ? NB / kThreads : 1;
   constexpr int ACT = NB / PER;
   const int lo = NB - ((int)threadIdx.x + 1) * PER;
@@ -128,7 +141,7 @@ __device__ __forceinline__ void find_digit(const uint32_t* H, uint32_t k_rem, ui
 #pragma unroll
   for (int j = 0; j < PER; ++j) tsum += c[j];
   uint32_t tot;
-  const uint32_t above = block_excl_scan(tsum, wsum, &tot);
+  const uint32_t above = block_excl_scan<THREADS>(tsum, wsum, &tot);
   if (above < k_rem && k_rem <= above + tsum) {
     uint32_t a = above;
 #pragma unroll
@@ -181,9 +194,14 @@ __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
-__global__ void __launch_bounds__(kThreads, 1) select_topk_kernel(const SelectParams p) {
+template <int THREADS>
+__global__ void __launch_bounds__(THREADS, 1) select_topk_kernel(const SelectParams p) {
+  constexpr int kThreads = Cfg<THREADS>::kThreads;
+  constexpr int kWarps = Cfg<THREADS>::kWarps;
+  constexpr int kStageKeys = Cfg<THREADS>::kStageKeys;
+  constexpr int kStages = Cfg<THREADS>::kStages;
   extern __shared__ __align__(128) unsigned char smem_raw[];
-  SelSmem& S = *reinterpret_cast<SelSmem*>(smem_raw);
+  SelSmem<THREADS>& S = *reinterpret_cast<SelSmem<THREADS>*>(smem_raw);
   const uint32_t rank = cg::this_cluster().block_rank();
   const int C = (int)cg::this_cluster().num_blocks();
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -204,7 +222,7 @@ __global__ void __launch_bounds__(kThreads, 1) select_topk_kernel(const SelectPa
   const int len = c1 - c0;
   const uint32_t* gk = p.keys + (size_t)bh * p.cap + c0;
   const int nwords = (len + 31) >> 5;
-  const int wpt = (nwords + kThreads - 1) / kThreads;  // bitmap words per thread (<= 4)
+  const int wpt = (nwords + kThreads - 1) / kThreads;  // bitmap words per thread (<= 8)
   const int w0 = min(tid * wpt, nwords), w1 = min(w0 + wpt, nwords);
 
   if (!sel.ranked) {
@@ -256,7 +274,7 @@ __global__ void __launch_bounds__(kThreads, 1) select_topk_kernel(const SelectPa
 
   // ---- digit 1 from the global histogram ----
   const uint32_t* ghist = p.hist + (size_t)bh * kHistBins;
-  find_digit<kHistBins>(ghist, (uint32_t)k_eff, S.wsum, &S.found);
+  find_digit<kHistBins, kThreads>(ghist, (uint32_t)k_eff, S.wsum, &S.found);
   const uint32_t d1 = S.found.digit;
   const uint32_t above1 = S.found.above;  // keys of the head with a larger digit 1
   const uint32_t eq1 = S.found.eq;        // keys of the head with this digit 1: the candidates
@@ -353,14 +371,14 @@ __global__ void __launch_bounds__(kThreads, 1) select_topk_kernel(const SelectPa
         for (uint32_t i = tid; i < total; i += kThreads)
           atomicAdd(&S.hloc[(S.ckey[i] >> kDigit3Bits) & (kBins2 - 1)], 1u);
         __syncthreads();
-        find_digit<kBins2>(S.hloc, k_rem, S.wsum, &S.found);
+        find_digit<kBins2, kThreads>(S.hloc, k_rem, S.wsum, &S.found);
         const uint32_t d2 = S.found.digit;
         k_rem -= S.found.above;
         const uint32_t pre = (d1 << kDigit2Bits) | d2;
         for (uint32_t i = tid; i < total; i += kThreads)
           if ((S.ckey[i] >> kDigit3Bits) == pre) atomicAdd(&S.hacc3[S.ckey[i] & (kBins3 - 1)], 1u);
         __syncthreads();
-        find_digit<kBins3>(S.hacc3, k_rem, S.wsum, &S.found);
+        find_digit<kBins3, kThreads>(S.hacc3, k_rem, S.wsum, &S.found);
         T = (pre << kDigit3Bits) | S.found.digit;
         k_rem -= S.found.above;
         need = k_rem;  // ties on T to take, 1 <= need <= eq
@@ -445,7 +463,7 @@ __global__ void __launch_bounds__(kThreads, 1) select_topk_kernel(const SelectPa
     for (int i = tid; i < kBins2; i += kThreads)
       if (S.hloc[i]) dsmem_red_add(dsmem_addr(&S.hacc2[i], 0), S.hloc[i]);
     cluster_sync();
-    find_digit<kBins2>(cg::this_cluster().map_shared_rank(S.hacc2, 0), k_rem, S.wsum, &S.found);
+    find_digit<kBins2, kThreads>(cg::this_cluster().map_shared_rank(S.hacc2, 0), k_rem, S.wsum, &S.found);
     const uint32_t pre = (d1 << kDigit2Bits) | S.found.digit;
     k_rem -= S.found.above;
     // digit 3
@@ -459,7 +477,7 @@ __global__ void __launch_bounds__(kThreads, 1) select_topk_kernel(const SelectPa
     for (int i = tid; i < kBins3; i += kThreads)
       if (S.hloc[i]) dsmem_red_add(dsmem_addr(&S.hacc3[i], 0), S.hloc[i]);
     cluster_sync();
-    find_digit<kBins3>(cg::this_cluster().map_shared_rank(S.hacc3, 0), k_rem, S.wsum, &S.found);
+    find_digit<kBins3, kThreads>(cg::this_cluster().map_shared_rank(S.hacc3, 0), k_rem, S.wsum, &S.found);
     const uint32_t T = (pre << kDigit3Bits) | S.found.digit;
     const uint32_t need = k_rem - S.found.above;
     // bits above T and ties on T, word by word; counts per CTA
@@ -477,8 +495,8 @@ __global__ void __launch_bounds__(kThreads, 1) select_topk_kernel(const SelectPa
       n_tie += (uint32_t)__popc(tb);
     }
     uint32_t tot_above, tot_tie;
-    const uint32_t tie_pre = block_excl_scan(n_tie, S.wsum, &tot_tie);
-    block_excl_scan(n_above, S.wsum, &tot_above);
+    const uint32_t tie_pre = block_excl_scan<kThreads>(n_tie, S.wsum, &tot_tie);
+    block_excl_scan<kThreads>(n_above, S.wsum, &tot_above);
     if (tid == 0) {
       dsmem_st(dsmem_addr(&S.ctl.above_of[rank], 0), tot_above);
       dsmem_st(dsmem_addr(&S.ctl.tie_of[rank], 0), tot_tie);
@@ -518,7 +536,7 @@ __global__ void __launch_bounds__(kThreads, 1) select_topk_kernel(const SelectPa
     uint32_t cnt = 0u;
     for (int w = w0; w < w1; ++w) cnt += (uint32_t)__popc(S.bm[w]);
     uint32_t tot;
-    uint32_t o = out_base + block_excl_scan(cnt, S.wsum, &tot);
+    uint32_t o = out_base + block_excl_scan<kThreads>(cnt, S.wsum, &tot);
     for (int w = w0; w < w1; ++w) {
       uint32_t bits = S.bm[w];
       while (bits) {
@@ -548,16 +566,17 @@ bool plan_select(SelectParams& p, int num_sms) {
   p.cand_cap = kCap;
   p.off_hist = 0;
   p.off_ctl = 0;
-  p.smem_bytes = (int)sizeof(SelSmem);
+  p.threads = C >= 2 ? 512 : 1024;
+  p.smem_bytes = p.threads == 512 ? (int)sizeof(SelSmem<512>) : (int)sizeof(SelSmem<1024>);
   return true;
 }
 
 cudaError_t launch_select(const SelectParams& p, cudaStream_t stream) {
-  auto kern = select_topk_kernel;
+  auto kern = p.threads == 512 ? select_topk_kernel<512> : select_topk_kernel<1024>;
   const cudaError_t e = prepare_kernel((const void*)kern, p.smem_bytes, p.cluster > 8);
   if (e != cudaSuccess) return e;
-  return launch_pdl(kern, dim3((unsigned)p.cluster, (unsigned)(p.B * p.Hkv), 1), dim3(kThreads), (size_t)p.smem_bytes,
-                    stream, p, (unsigned)p.cluster);
+  return launch_pdl(kern, dim3((unsigned)p.cluster, (unsigned)(p.B * p.Hkv), 1), dim3((unsigned)p.threads),
+                    (size_t)p.smem_bytes, stream, p, (unsigned)p.cluster);
 }
 
 }  // namespace sas
