@@ -67,6 +67,17 @@ def test_exact_ties_take_lowest_positions(cuda_lib):
     run_small(p, dense=False)
 
 
+@pytest.mark.parametrize("B,Hkv,N", [(1, 2, 20000), (40, 2, 10000)])
+def test_candidate_overflow_takes_the_slow_path(cuda_lib, B, Hkv, N):
+    # more than 4096 keys share the k-th key's first digit (half the positions tie), so the
+    # candidate list cannot hold them: clusters of CTAs per head (B=1) and one CTA per head
+    # (80 heads) both fall back to re-reading the keys
+    p = make_problem(B=B, Hq=2 * Hkv, Hkv=Hkv, d=64, r=16, seqlens=[N] * B, k=[700] * B, basis="eye", seed=8)
+    p.K[:, :, :N // 2, :16] = 0.5
+    p.K[:, :, N // 2:, :16] = 0.25
+    run_small(p, dense=False)
+
+
 def test_device_checks_set_the_error_word(cuda_lib):
     from token_level_sparse_head_b200 import DecodeSession, lib, shape_of
 
