@@ -635,9 +635,21 @@ def cpu_baseline(name, budget_s=15.0):
     while sum(ts) < budget_s and len(ts) < 100000:
         ts.append(oracle_head_seconds(distinct[len(ts) % len(distinct)]))
     per_head = statistics.mean(ts)
-    return {"value": 1.0 / (per_head * heads_per_step), "unit": UNIT, "cores": _threads_used(),
-            "kind": "oracle", "sample": f"{len(ts)} oracle runs over {len(distinct)} distinct (sequence, KV head) "
-            f"pairs of the workload ({sum(ts):.1f} s of oracle time); one step = {heads_per_step} pairs"}
+    out = {"value": 1.0 / (per_head * heads_per_step), "unit": UNIT, "cores": _threads_used(),
+           "kind": "oracle", "sample": f"{len(ts)} oracle runs over {len(distinct)} distinct (sequence, KV head) "
+           f"pairs of the workload ({sum(ts):.1f} s of oracle time); one step = {heads_per_step} pairs"}
+    # the same oracle held to one thread, on a third of the budget
+    try:
+        from threadpoolctl import threadpool_limits
+
+        t1 = []
+        with threadpool_limits(limits=1):
+            while sum(t1) < budget_s / 3 and len(t1) < 100000:
+                t1.append(oracle_head_seconds(distinct[len(t1) % len(distinct)]))
+        out["value_1_thread"] = 1.0 / (statistics.mean(t1) * heads_per_step)
+    except ImportError:
+        pass
+    return out
 
 
 def run_reference(args):
