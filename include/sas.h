@@ -28,9 +28,9 @@
  *       contiguous (page_size == 0): K, V [B][Hkv][n_cap][d] bf16; Kproj [B][Hkv][n_cap][r];
  *       paged (page_size == 64):     K, V [num_pages][Hkv][64][d] bf16;
  *                                    Kproj [num_pages][Hkv][64][r];
- *     Kproj elements are bf16 or FP8 E4M3 codes (shape.kproj_dtype);
  *                                    page_table [B][max_pages] int32, logical token t of
  *                                    sequence b lives in page page_table[b][t / 64], row t % 64.
+ *     Kproj elements are bf16 or FP8 E4M3 codes (shape.kproj_dtype).
  *     The logical capacity is cap = n_cap (contiguous) or max_pages * 64 (paged).
  *   - seqlens [B] int32: cached tokens N_b of each sequence (0 <= N_b <= cap).
  *   - Host-side validation rejects bad shapes, null or misaligned pointers and unsupported
