@@ -46,3 +46,40 @@ def test_sampled_moments_capture_the_leading_channels():
         np.testing.assert_allclose(M[h] @ M[h].T, np.eye(p.r), atol=1e-6)
         captured = (M[h][:, : p.r // 2] ** 2).sum(axis=0)   # |M e_j|^2 for the leading channels
         assert np.all(captured > 0.9), captured
+
+
+def _oracle_recall(M, qbars, K, k):
+    """Mean over queries of |top-k of (M q-bar).(M k_i)  ∩  top-k of q-bar.k_i| / k (oracle's
+    own projection, scores and ranking)."""
+    kp = O.project_keys(K, M)
+    rec = []
+    for qb in qbars:
+        exact = set(O.top_k_positions(O.decision_keys(K @ qb), k).tolist())
+        u = O.selection_scores(O.project_query(M, qb), kp, 1.0)
+        sel = set(O.top_k_positions(O.decision_keys(u), k).tolist())
+        rec.append(len(exact & sel) / k)
+    return float(np.mean(rec))
+
+
+def test_joint_basis_keeps_the_ranking_a_key_only_basis_loses():
+    # JSSA page, sections 问题形式化 / 迹归一化: the basis must preserve query-key interaction,
+    # not key reconstruction.  Keys vary most in channels 0-3, where queries are almost zero;
+    # queries vary most in channels 4-7.  The scores live in channels 4-7: the joint basis
+    # (trace-normalised query + key moments) finds them, the key-only principal basis does not.
+    rng = np.random.default_rng(11)
+    d, r, G, N, T, k = 32, 4, 4, 4096, 4000, 128
+    sk = np.ones(d); sk[:4] = 3.0
+    sq = np.full(d, 0.3); sq[:4] = 0.1; sq[4:8] = 3.0
+    K = rng.standard_normal((N, d)) * sk
+    q = rng.standard_normal((T, 1, G, d)) * sq            # [T][Hkv=1][G][d]
+    acc = MomentAccumulator(1, d)
+    acc.add_queries(torch.from_numpy(q.reshape(T, G, d)))
+    acc.add_keys(torch.from_numpy(K[None]))
+    M_joint = calibrate(acc, r).double().numpy()[0]
+    w, V = np.linalg.eigh(acc.Gk[0].numpy())
+    M_key = V[:, np.argsort(w)[::-1][:r]].T               # principal key directions
+    np.testing.assert_allclose((M_joint[:, 4:8] ** 2).sum(axis=1), 1.0, atol=0.05)  # spans channels 4-7
+    qbars = [O.group_mean_query(rng.standard_normal((G, d)) * sq) for _ in range(20)]
+    rec_joint = _oracle_recall(M_joint, qbars, K, k)
+    rec_key = _oracle_recall(M_key, qbars, K, k)
+    assert rec_joint > 0.5 and rec_joint > rec_key + 0.3, (rec_joint, rec_key)
