@@ -83,3 +83,28 @@ def test_joint_basis_keeps_the_ranking_a_key_only_basis_loses():
     rec_joint = _oracle_recall(M_joint, qbars, K, k)
     rec_key = _oracle_recall(M_key, qbars, K, k)
     assert rec_joint > 0.5 and rec_joint > rec_key + 0.3, (rec_joint, rec_key)
+
+
+def test_trace_normalisation_keeps_the_query_side():
+    # JSSA page, section 迹归一化 (Table 9): the key second moment's trace can exceed the query
+    # side's by orders of magnitude; summing the raw moments then returns a key-reconstruction
+    # basis.  Same channels as above with the keys 10x larger: the normalised basis is unchanged
+    # (scale-free), the raw sum picks the key channels and loses the ranking.
+    rng = np.random.default_rng(12)
+    d, r, G, N, T, k = 32, 4, 4, 4096, 4000, 128
+    sk = np.ones(d) * 10.0; sk[:4] = 30.0
+    sq = np.full(d, 0.3); sq[:4] = 0.1; sq[4:8] = 3.0
+    K = rng.standard_normal((N, d)) * sk
+    q = rng.standard_normal((T, G, d)) * sq
+    acc = MomentAccumulator(1, d)
+    acc.add_queries(torch.from_numpy(q))
+    acc.add_keys(torch.from_numpy(K[None]))
+    Gq, Gk = acc.Gq[0].numpy() / acc.nq, acc.Gk[0].numpy() / acc.nk
+    assert np.trace(Gk) / np.trace(Gq) > 100
+    M_norm = calibrate(acc, r).double().numpy()[0]
+    w, V = np.linalg.eigh(Gq + Gk)
+    M_raw = V[:, np.argsort(w)[::-1][:r]].T
+    qbars = [O.group_mean_query(rng.standard_normal((G, d)) * sq) for _ in range(20)]
+    rec_norm = _oracle_recall(M_norm, qbars, K, k)
+    rec_raw = _oracle_recall(M_raw, qbars, K, k)
+    assert rec_norm > 0.5 and rec_norm > rec_raw + 0.3, (rec_norm, rec_raw)
