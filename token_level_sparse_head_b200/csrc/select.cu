@@ -54,22 +54,23 @@ struct Ctl {
   uint32_t tie_of[kMaxCluster];
 };
 
-// Block shape: THREADS threads per CTA, and a ring of 128 KB of keys in stages of 4 keys per
-// thread.  1024 threads serve a head per CTA (B=16); clusters of several CTAs per head (small
-// batches) use 512, which spend less time in block-wide barriers.
+// Block shape: THREADS threads per CTA.  1024 threads serve a head per CTA (B=16); clusters of
+// several CTAs per head (small batches) use 512, which spend less time in block-wide barriers.
+// Each warp streams its own tiles of 512 keys (2 KB) through a ring of its own, kSlots deep, so
+// 128 KB of keys are in flight per CTA either way.
 template <int THREADS>
 struct Cfg {
   static constexpr int kThreads = THREADS;
   static constexpr int kWarps = THREADS / 32;
-  static constexpr int kStageKeys = kWarps * 128;  // keys per ring stage: 4 per lane
-  static constexpr int kStages = 8 * 1024 / THREADS;
+  static constexpr int kTileKeys = 512;            // keys per tile: 16 per lane
+  static constexpr int kSlots = 2 * 1024 / THREADS;
 };
 
 template <int THREADS>
 struct SelSmem {
-  static constexpr int kStages = Cfg<THREADS>::kStages;
+  static constexpr int kSlots = Cfg<THREADS>::kSlots;
   static constexpr int kWarps = Cfg<THREADS>::kWarps;
-  uint32_t ring[kStages][Cfg<THREADS>::kStageKeys];
+  uint32_t ring[kWarps][kSlots][Cfg<THREADS>::kTileKeys];
   uint32_t bm[kMaxWords];     // selected positions of the chunk
   uint32_t ckey[kCap];        // candidate keys (slow path: tie bits per bitmap word)
   int32_t cpos[kCap];         // candidate positions in the head
@@ -77,8 +78,7 @@ struct SelSmem {
   uint32_t hacc2[kBins2];     // CTA 0, slow path: cluster histogram of digit 2
   uint32_t hacc3[kBins3];     // CTA 0: histogram of digit 3
   int32_t tpos[kMaxTies];
-  uint64_t full[kStages];
-  uint64_t empty[kStages];
+  uint64_t full[kWarps][kSlots];
   uint32_t wsum[kWarps];
   Ctl ctl;
   Found found;
@@ -198,8 +198,8 @@ template <int THREADS>
 __global__ void __launch_bounds__(THREADS, 1) select_topk_kernel(const SelectParams p) {
   constexpr int kThreads = Cfg<THREADS>::kThreads;
   constexpr int kWarps = Cfg<THREADS>::kWarps;
-  constexpr int kStageKeys = Cfg<THREADS>::kStageKeys;
-  constexpr int kStages = Cfg<THREADS>::kStages;
+  constexpr int kTileKeys = Cfg<THREADS>::kTileKeys;
+  constexpr int kSlots = Cfg<THREADS>::kSlots;
   extern __shared__ __align__(128) unsigned char smem_raw[];
   SelSmem<THREADS>& S = *reinterpret_cast<SelSmem<THREADS>*>(smem_raw);
   const uint32_t rank = cg::this_cluster().block_rank();
@@ -234,12 +234,12 @@ __global__ void __launch_bounds__(THREADS, 1) select_topk_kernel(const SelectPar
   }
 
   // ---------------------------------------------------------------- set-up
-  const int nst = (len + kStageKeys - 1) / kStageKeys;
+  // warp w streams tiles w, w + kWarps, ... of the chunk
+  const int ntiles = (len + kTileKeys - 1) / kTileKeys;
+  const int my_tiles = ntiles > warp ? (ntiles - warp + kWarps - 1) / kWarps : 0;
   if (tid == 0) {
-    for (int s = 0; s < kStages; ++s) {
-      mbar_init(&S.full[s], 1);
-      mbar_init(&S.empty[s], kWarps);
-    }
+    for (int w = 0; w < kWarps; ++w)
+      for (int s = 0; s < kSlots; ++s) mbar_init(&S.full[w][s], 1);
     fence_barrier_init();
   }
   for (int i = tid; i < kMaxWords; i += kThreads) S.bm[i] = 0u;
@@ -260,17 +260,19 @@ __global__ void __launch_bounds__(THREADS, 1) select_topk_kernel(const SelectPar
   pdl_wait();
   pdl_trigger();
 
-  // Stage s of the chunk: keys [s * kStageKeys, +kStageKeys) as whole 16-byte units (the key
-  // rows have a multiple of 4 entries, so the rounding stays inside this (b, h)'s row).
-  auto issue = [&](int s) {
-    const int slot = s % kStages;
-    const int keys = min(kStageKeys, len - s * kStageKeys);
+  // The warp's j-th tile (tile warp + j * kWarps of the chunk) into its slot j % kSlots, as whole
+  // 16-byte units (the key rows have a multiple of 4 entries, so the rounding stays inside this
+  // (b, h)'s row).  Issued by lane 0.
+  auto issue = [&](int j) {
+    const int t = warp + j * kWarps;
+    const int slot = j % kSlots;
+    const int keys = min(kTileKeys, len - t * kTileKeys);
     const uint32_t bytes = (uint32_t)((keys + 3) & ~3) * 4u;
-    mbar_arrive_expect_tx(&S.full[slot], bytes);
-    bulk_g2s(S.ring[slot], gk + (size_t)s * kStageKeys, bytes, &S.full[slot]);
+    mbar_arrive_expect_tx(&S.full[warp][slot], bytes);
+    bulk_g2s(S.ring[warp][slot], gk + (size_t)t * kTileKeys, bytes, &S.full[warp][slot]);
   };
-  if (tid == 0)
-    for (int s = 0; s < min(kStages, nst); ++s) issue(s);
+  if (lane == 0)
+    for (int j = 0; j < min(kSlots, my_tiles); ++j) issue(j);
 
   // ---- digit 1 from the global histogram ----
   const uint32_t* ghist = p.hist + (size_t)bh * kHistBins;
@@ -287,51 +289,52 @@ __global__ void __launch_bounds__(THREADS, 1) select_topk_kernel(const SelectPar
     uint32_t my_above = 0u;
     // keys of digit d1 are [lo, hi]; above: key > hi (never true when d1 is the top digit)
     const uint32_t lo = d1 << kHistShift, hi = lo | ((1u << kHistShift) - 1u);
-    for (int s = 0; s < nst; ++s) {
-      const int slot = s % kStages;
-      if (!mbar_wait_bounded(&S.full[slot], (uint32_t)(s / kStages) & 1u)) waited_ok = false;
-      // the warp's 128 keys: lane l takes keys 4l .. 4l+3 (one 16-byte read) and forms their
-      // 4 bits; the 8 lanes of a bitmap word combine their nibbles with three shuffles
-      const uint4 kv = reinterpret_cast<const uint4*>(S.ring[slot] + warp * 128)[lane];
-      const int lp = s * kStageKeys + warp * 128 + 4 * lane;  // chunk position of the lane's first key
-      const int wbase = s * (kStageKeys / 32) + warp * 4;
-      const uint32_t kk[4] = {kv.x, kv.y, kv.z, kv.w};
+    for (int j = 0; j < my_tiles; ++j) {
+      const int slot = j % kSlots;
+      if (!mbar_wait_bounded(&S.full[warp][slot], (uint32_t)(j / kSlots) & 1u)) waited_ok = false;
+      // lane l takes keys 16l .. 16l+15 of the tile: four 16-byte reads, lane pairs rotating
+      // their order so that each read of the warp covers all banks; 2 lanes make a bitmap word
+      const int t = warp + j * kWarps;
+      const uint32_t* row = S.ring[warp][slot] + 16 * lane;
+      const int lp = t * kTileKeys + 16 * lane;  // chunk position of the lane's first key
       uint32_t ab = 0u, cb = 0u;
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        ab |= (kk[j] > hi ? 1u : 0u) << j;
-        cb |= (kk[j] - lo <= hi - lo ? 1u : 0u) << j;
+      for (int q = 0; q < 4; ++q) {
+        const int c = (q + (lane >> 1)) & 3;
+        const uint4 kv = reinterpret_cast<const uint4*>(row)[c];
+        const uint32_t k4[4] = {kv.x, kv.y, kv.z, kv.w};
+        uint32_t a4 = 0u, c4 = 0u;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          a4 |= (k4[e] > hi ? 1u : 0u) << e;
+          c4 |= (k4[e] - lo <= hi - lo ? 1u : 0u) << e;
+        }
+        ab |= a4 << (4 * c);
+        cb |= c4 << (4 * c);
       }
-      if ((s + 1) * kStageKeys > len) {  // the last, partial stage: drop keys past the chunk
-        const uint32_t vm = (1u << min(max(len - lp, 0), 4)) - 1u;
+      if ((t + 1) * kTileKeys > len) {  // the last, partial tile: drop keys past the chunk
+        const uint32_t vm = (1u << min(max(len - lp, 0), 16)) - 1u;
         ab &= vm;
         cb &= vm;
       }
-      uint32_t word = ab << (4 * (lane & 7));
+      uint32_t word = ab << (16 * (lane & 1));
       word |= __shfl_xor_sync(0xffffffffu, word, 1);
-      word |= __shfl_xor_sync(0xffffffffu, word, 2);
-      word |= __shfl_xor_sync(0xffffffffu, word, 4);
-      if ((lane & 7) == 0) S.bm[wbase + (lane >> 3)] = word;
+      if ((lane & 1) == 0) S.bm[lp >> 5] = word;
       my_above += (uint32_t)__popc(ab);
       if (cb) {
-        uint32_t j = atomicAdd(&S.ctl.ccount, (uint32_t)__popc(cb));
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          if ((cb >> e) & 1u) {
-            if (j < (uint32_t)kCap) {
-              S.ckey[j] = kk[e];
-              S.cpos[j] = c0 + lp + e;
-            }
-            ++j;
+        uint32_t jj = atomicAdd(&S.ctl.ccount, (uint32_t)__popc(cb));
+        while (cb) {
+          const int e = __ffs(cb) - 1;
+          cb &= cb - 1u;
+          if (jj < (uint32_t)kCap) {
+            S.ckey[jj] = row[e];
+            S.cpos[jj] = c0 + lp + e;
           }
+          ++jj;
         }
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&S.empty[slot]);
-      if (tid == 0 && s + kStages < nst) {
-        if (!mbar_wait_bounded(&S.empty[slot], (uint32_t)(s / kStages) & 1u)) waited_ok = false;
-        issue(s + kStages);
-      }
+      __syncwarp();  // every lane is done with the slot
+      if (lane == 0 && j + kSlots < my_tiles) issue(j + kSlots);
     }
 #pragma unroll
     for (int o = 16; o; o >>= 1) my_above += __shfl_xor_sync(0xffffffffu, my_above, o);
@@ -430,9 +433,9 @@ __global__ void __launch_bounds__(THREADS, 1) select_topk_kernel(const SelectPar
       for (int i = tid; i < kHistBins; i += kThreads) const_cast<uint32_t*>(ghist)[i] = 0u;  // for the next call
   } else {
     // Too many candidates for the list: drain the copies issued above, then take the slow path.
-    if (tid == 0)
-      for (int s = 0; s < min(kStages, nst); ++s)
-        if (!mbar_wait_bounded(&S.full[s], 0u)) waited_ok = false;
+    if (lane == 0)
+      for (int j = 0; j < min(kSlots, my_tiles); ++j)
+        if (!mbar_wait_bounded(&S.full[warp][j % kSlots], 0u)) waited_ok = false;
     __syncthreads();
     cluster_wait();
     if (rank == 0)
