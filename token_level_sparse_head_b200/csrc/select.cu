@@ -8,11 +8,11 @@
 // A cluster of C CTAs serves one (b, h) (C = 1 when there are enough heads to fill the GPU);
 // each CTA owns a contiguous chunk of positions.  The k-th largest key T is found as three radix
 // digits (13, 10 and 9 bits); ties on T go to the lower positions.
-//   1. The global histogram gives digit 1.  Each CTA streams its chunk of keys once through a
-//      shared-memory ring (bulk copies; each lane turns 4 keys into 4 bits of a bitmap word),
-//      setting a position bitmap of the keys whose digit 1 is larger (they are selected) and
-//      appending the keys whose digit 1 equals it (the candidates, a few percent of the
-//      positions) to a list.
+//   1. The global histogram gives digit 1.  Each CTA streams its chunk of keys once: every warp
+//      takes tiles of 512 keys in turn through a shared-memory ring of its own (bulk copies;
+//      each lane turns 16 keys into 16 bits of a bitmap word), setting a position bitmap of the
+//      keys whose digit 1 is larger (they are selected) and appending the keys whose digit 1
+//      equals it (the candidates, a few percent of the positions) to a list.
 //   2. The candidate lists are gathered into CTA 0 of the cluster through distributed shared
 //      memory; CTA 0 finds digits 2 and 3 among them, resolves the ties, marks the chosen
 //      candidates in the owners' bitmaps and hands every CTA its first output slot.
