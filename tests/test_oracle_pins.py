@@ -292,6 +292,66 @@ def test_paged_layout_equals_contiguous_layout():
     assert rp[(1, 0)][0].tolist() == list(range(64))
 
 
+# A hand-written page table over three physical 64-token pages of two KV heads.  Every
+# physical slot (page, head, row) holds the number 1000*page + 100*head + row, so a value
+# read back names the slot it came from.  Sequence 0 (100 tokens) lives in page 2 (tokens
+# 0..63) and then page 0 (tokens 64..99); sequence 1 (10 tokens) in page 1.  The expected
+# logical rows below are written out from that description, not computed by the oracle.
+HAND_PAGE_TABLE = np.array([[2, 0], [1, -1]])
+HAND_SEQLENS = [100, 10]
+
+
+def _hand_paged_cache(width):
+    cache = np.zeros((3, 2, 64, width))
+    for page in range(3):
+        for head in range(2):
+            for row in range(64):
+                cache[page, head, row, :] = 1000 * page + 100 * head + row
+    # make the channels distinguishable too: channel c adds c / 8 (exact in float64)
+    cache += np.arange(width)[None, None, None, :] / 8.0
+    return cache
+
+
+def test_paged_logical_rows_follow_a_hand_written_page_table():
+    cache = _hand_paged_cache(4)
+    for head in range(2):
+        want0 = [2000 + 100 * head + t for t in range(64)] + [0 + 100 * head + (t - 64) for t in range(64, 100)]
+        got0 = O.logical_rows(cache, 0, head, 100, HAND_PAGE_TABLE)
+        assert got0.shape == (100, 4)
+        assert got0[:, 0].tolist() == want0
+        assert got0[:, 3].tolist() == [v + 3 / 8.0 for v in want0]
+        want1 = [1000 + 100 * head + t for t in range(10)]
+        assert O.logical_rows(cache, 1, head, 10, HAND_PAGE_TABLE)[:, 0].tolist() == want1
+    # the contiguous layout indexes [b][h][t] directly
+    cont = np.arange(2 * 2 * 5 * 1, dtype=np.float64).reshape(2, 2, 5, 1)
+    assert O.logical_rows(cont, 1, 0, 3)[:, 0].tolist() == [10.0, 11.0, 12.0]
+
+
+def test_paged_build_scatters_rows_to_their_physical_slots():
+    # Key channels (page, head, row, 0.5) of every physical slot: small integers, exact in bf16.
+    K = np.zeros((3, 2, 64, 4))
+    for page in range(3):
+        for head in range(2):
+            for row in range(64):
+                K[page, head, row] = [page, head, row, 0.5]
+    # one basis per KV head picking key channels 2, 0, 1: Kproj of a slot = (row, page, head)
+    M = np.stack([np.eye(4)[[2, 0, 1]]] * 2)
+    kp = O.build_proj_cache(K, M, HAND_SEQLENS, HAND_PAGE_TABLE)
+    assert kp.shape == (3, 2, 64, 3)
+    for head in range(2):
+        # sequence 0: page 2 rows 0..63 and page 0 rows 0..35 are written
+        for row in range(64):
+            assert kp[2, head, row].tolist() == [row, 2, head]
+        for row in range(36):
+            assert kp[0, head, row].tolist() == [row, 0, head]
+        # sequence 1: page 1 rows 0..9
+        for row in range(10):
+            assert kp[1, head, row].tolist() == [row, 1, head]
+        # slots no logical token maps to stay zero
+        assert not kp[0, head, 36:].any()
+        assert not kp[1, head, 10:].any()
+
+
 # ----------------------------------------------------------------------------- calibration
 def test_calibration_closed_form_for_anisotropic_keys():
     # q ~ N(0, I): E[q-bar q-bar^T] = I / G ; K = Z diag(s): E[k k^T] = diag(s^2).
@@ -318,6 +378,31 @@ def test_calibration_bound_and_optimality():
         for _ in range(10):
             Q = np.linalg.qr(RNG.standard_normal((d, r)))[0]
             assert lmarg <= O.marginal_objective(Q @ Q.T, Gq, Gk) + 1e-12
+
+
+def test_selection_objective_closed_forms():
+    # Diagonal second moments and a coordinate projector onto the set S: the error of the
+    # projected score comes only from the channels outside S, L_sel = sum_{j not in S} a_j b_j,
+    # and L_marg = sum_{j not in S} (a_j + b_j).
+    a = np.array([3.0, 0.5, 2.0, 1.5, 0.25])
+    b = np.array([1.0, 4.0, 0.5, 2.0, 8.0])
+    S = [0, 2]
+    P = np.diag([1.0 if j in S else 0.0 for j in range(5)])
+    rest = [j for j in range(5) if j not in S]
+    assert O.selection_objective(P, np.diag(a), np.diag(b)) == sum(a[j] * b[j] for j in rest)  # 0.5*4 + 1.5*2 + 0.25*8
+    assert O.marginal_objective(P, np.diag(a), np.diag(b)) == sum(a[j] + b[j] for j in rest)
+    # A rank-1 complement I - P = v v^T with non-diagonal moments: L_sel = (v^T Gq v)(v^T Gk v).
+    # P projects on (1, 1)/sqrt 2, v = (1, -1)/sqrt 2; by hand v^T Gq v = (2 - 2 + 2)/2 = 1 and
+    # v^T Gk v = (1 - 2 + 3)/2 = 1.
+    Gq = np.array([[2.0, 1.0], [1.0, 2.0]])
+    Gk = np.array([[1.0, 1.0], [1.0, 3.0]])
+    P = np.full((2, 2), 0.5)
+    assert abs(O.selection_objective(P, Gq, Gk) - 1.0) < 1e-15
+    assert abs(O.marginal_objective(P, Gq, Gk) - 2.0) < 1e-15
+    # and with P = e1 e1^T the complement is e2: L_sel = Gq[1,1] * Gk[1,1] = 6 (not 7, which a
+    # product missing the second (I - P) factor gives)
+    P = np.diag([1.0, 0.0])
+    assert O.selection_objective(P, Gq, Gk) == 6.0
 
 
 # ------------------------------------------------------------------ FP8 E4M3 (projected cache)
