@@ -3,20 +3,34 @@
 // JSSA page, section 打分误差的定义: the selection score of cached token i under KV head h is
 // s-hat_i = q-bar^T M^T (M k_i) = q-hat . Kproj_i, with q-bar the mean of the G query heads of
 // h; section Triton 内核的三个设计点: scoring is not sparse, it scans every candidate.  The gate
-// of the SAS page (section 2.1) adds lambda * log g_i.  Each score is kept as the order-preserving
-// uint32 key of u_i = sigma * s-hat_i (+ lambda log g_i); a per-(b, h) histogram of the keys' top
-// 13 bits is accumulated for the selection that follows.
+// of the SAS page (section 2.1) adds lambda * log g_i.  Each score is turned into the
+// order-preserving uint32 key of u_i = sigma * s-hat_i (+ lambda log g_i) for the selection that
+// follows, in one of two forms chosen per launch:
+//
+//   keys mode        every key is written to the workspace (L2 evict-last hint) and a histogram
+//                    of the keys' top 13 bits is accumulated per (b, h);
+//   candidate mode   only keys at or above a running lower bound tau of the head's k-th largest
+//                    key are written, as (key, position) pairs.  The k-th largest key among the
+//                    rows a CTA has scanned so far can only be at or below the k-th largest of the
+//                    whole head, so a key below tau can never be selected and is dropped.  A
+//                    threshold warp keeps tau up to date from a shared-memory histogram of the
+//                    written keys' top 12 bits.  With long per-CTA segments (many heads) this
+//                    writes a few k keys per head instead of N.
 //
 // Persistent kernel, one CTA per SM.  The work is the list of 4 KB blocks of projected rows
-// (64 rows at r = 32) of every (b, h) that needs scores, in (b, h, position) order; each CTA
-// takes one contiguous, equal share of it, so a CTA walks the rows of one or a few heads front
-// to back.  Two producer warps stream the blocks into a shared-memory ring with bulk copies (TMA
-// engine: one copy per block, or per 64-token page piece for the paged layout, plus the block's
-// gate values); each producer lane owns one ring slot.  Twelve consumer warps take the blocks in
-// turn, each with its own three ring slots, so a warp's processing of one block (dot products,
-// butterfly reduction, key, histogram) overlaps the copies of its next two and about 144 KB of
-// rows stay in flight per SM.  Full blocks take a path without per-row tests.  Keys go to the workspace with
-// an L2 evict-last hint so that the selection kernel finds them on chip.
+// (64 rows at r = 32 in bf16) of every (b, h) that needs scores, in (b, h, position) order; each
+// CTA takes one contiguous, equal share of it.  Its consumer warps take the share's blocks in
+// turn; each warp owns three ring slots in shared memory and keeps them full itself: lane 0
+// issues the bulk copy (TMA engine, mbarrier completion) of the warp's next block into a slot as
+// soon as the warp has finished reading it, so no warp waits on another to release a slot.  Per
+// 32-row batch the lanes form 16-byte dot products with q-hat and meet in a transposing butterfly.
+//
+// Candidate storage: a warp writes the candidates of its blocks of one head, in order, into the
+// 64-row slot ranges of those same blocks (the n-th candidate into the (n / BR)-th of its blocks,
+// at offset n % BR); the count never outruns the rows scanned, so no space is shared.  At the end
+// of its part of a head the warp pads the count to even with a sentinel (key 0, which no score
+// maps to, never selected) and appends a record (first block | warps << 24, count) to the head's
+// record list; the warp count is the block stride of the record.
 #include <cuda_fp16.h>
 #include <cuda_fp8.h>
 
@@ -26,14 +40,13 @@
 namespace sas {
 namespace {
 
-constexpr int kConsumerWarps = 12;
-constexpr int kConsumers = kConsumerWarps * 32;
-constexpr int kProducerWarps = 2;          // one lane per ring slot
-constexpr int kThreads = kConsumers + kProducerWarps * 32;
-constexpr int kBlockBytes = 4096;          // projected bytes per block (one ring stage)
-constexpr int kDepth = 3;                  // ring slots per consumer warp
-constexpr int kSlots = kConsumerWarps * kDepth;
-static_assert(kSlots <= kProducerWarps * 32, "one producer lane per ring slot");
+constexpr int kBlockBytes = 4096;   // projected bytes per block (one ring stage)
+constexpr int kDepth = 3;           // ring slots per consumer warp
+constexpr int kMaxWarps = 16;       // consumer warps per CTA at most
+constexpr int kSmemLimit = 227 * 1024;
+constexpr int kSmemMisc = 2048;     // q-bar, q-hat, barriers, plan and threshold state (upper bound)
+constexpr uint32_t kTauDone = 0xffffffffu;  // generation that tells the threshold warp to stop
+constexpr uint32_t kTauPasses = 1u << 20;   // threshold passes at most (each ends in a short sleep)
 
 // Row geometry of the projected cache: bf16 (KP8 = false) or FP8 E4M3 codes (KP8 = true).
 template <int R, bool KP8>
@@ -41,8 +54,6 @@ struct Geo {
   static constexpr int ROW_BYTES = KP8 ? R : 2 * R;
   static constexpr int BLOCK_ROWS = kBlockBytes / ROW_BYTES;  // bf16: 128 / 64 / 32 for r = 16 / 32 / 64
   static constexpr int NB = BLOCK_ROWS / 32;                  // 32-row batches per block
-  static constexpr int LG_BYTES = BLOCK_ROWS * 4;             // gate values of one block
-  static constexpr int SLOT_BYTES = kBlockBytes + LG_BYTES;
   static constexpr int CPL = KP8 ? 16 : 8;  // channels per 16-byte load
   static constexpr int LPR = R / CPL;       // lanes per row
   static constexpr int RPI = 32 / LPR;      // rows per load instruction
@@ -50,37 +61,81 @@ struct Geo {
   static constexpr int LOG_LPR = LPR == 1 ? 0 : LPR == 2 ? 1 : LPR == 4 ? 2 : 3;
 };
 
-// Position of a CTA's share in the block list, computed once by the producer warp.
+// Block shape of one instantiation: as many consumer warps (three slots each) as shared memory
+// holds next to the histogram, at most 16; candidate mode adds the threshold warp.
+template <int R, bool GATED, bool KP8, bool CANDS>
+struct Cfg {
+  using Gm = Geo<R, KP8>;
+  static constexpr int kBins = CANDS ? (1 << kCandHistBits) : kHistBins;
+  static constexpr int kSlotBytes = kBlockBytes + (GATED ? Gm::BLOCK_ROWS * 4 : 0);
+  static constexpr int kMaxSlots = (kSmemLimit - kSmemMisc - kBins * 4) / kSlotBytes;
+  static constexpr int kWarps = kMaxSlots / kDepth >= kMaxWarps ? kMaxWarps : kMaxSlots / kDepth;
+  static constexpr int kSlots = kWarps * kDepth;
+  static constexpr int kConsumers = kWarps * 32;
+  static constexpr int kThreads = kConsumers + (CANDS ? 32 : 0);
+};
+
+// Position of a CTA's share in the block list, computed once by warp 0.
 struct Plan {
   int count;  // blocks of this CTA
   int b0;     // sequence of the first block
   int h0, c0; // KV head and block index within it
 };
 
-template <int R, int D, bool KP8>
+template <int R, int D, bool GATED, bool KP8, bool CANDS>
 struct Smem {
-  unsigned char ring[kSlots][Geo<R, KP8>::SLOT_BYTES];
-  uint32_t hist[kHistBins];
+  using C = Cfg<R, GATED, KP8, CANDS>;
+  unsigned char ring[C::kSlots][C::kSlotBytes];
+  uint32_t hist[C::kBins];
   float qbar[D];
   float qhat[R];
-  uint64_t full[kSlots];
-  uint64_t empty[kSlots];
+  uint64_t full[C::kSlots];
+  unsigned long long tau_state;  // candidate mode: (generation << 32) | threshold bin
+  int head_k;                    // candidate mode: k_eff of the head being scanned (0: none)
   Plan plan;
 };
-static_assert(sizeof(Smem<16, 128, false>) <= 227 * 1024 && sizeof(Smem<32, 128, false>) <= 227 * 1024 &&
-                  sizeof(Smem<64, 128, false>) <= 227 * 1024 && sizeof(Smem<16, 128, true>) <= 227 * 1024 &&
-                  sizeof(Smem<32, 128, true>) <= 227 * 1024 && sizeof(Smem<64, 128, true>) <= 227 * 1024,
+
+template <int R, int D, bool GATED, bool KP8, bool CANDS>
+constexpr bool smem_fits() {
+  return sizeof(Smem<R, D, GATED, KP8, CANDS>) <= (size_t)kSmemLimit;
+}
+static_assert(smem_fits<16, 128, true, true, true>() && smem_fits<16, 128, true, true, false>() &&
+                  smem_fits<32, 128, true, true, true>() && smem_fits<32, 128, true, true, false>() &&
+                  smem_fits<64, 128, true, true, true>() && smem_fits<64, 128, true, true, false>() &&
+                  smem_fits<16, 128, true, false, true>() && smem_fits<16, 128, true, false, false>() &&
+                  smem_fits<32, 128, true, false, true>() && smem_fits<32, 128, true, false, false>() &&
+                  smem_fits<64, 128, true, false, true>() && smem_fits<64, 128, true, false, false>() &&
+                  smem_fits<32, 128, false, false, false>() && smem_fits<32, 128, false, false, true>(),
               "score kernel shared memory");
 
 __device__ __forceinline__ void stg_hint(uint32_t* ptr, uint32_t v, uint64_t pol) {
   asm volatile("st.global.L2::cache_hint.u32 [%0], %1, %2;" ::"l"(ptr), "r"(v), "l"(pol) : "memory");
 }
-__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+__device__ __forceinline__ void stg_hint_v2(uint2* ptr, uint32_t a, uint32_t b, uint64_t pol) {
+  asm volatile("st.global.L2::cache_hint.v2.u32 [%0], {%1, %2}, %3;" ::"l"(ptr), "r"(a), "r"(b), "l"(pol) : "memory");
 }
-// Barrier 1 among the consumer warps only (the producer warp never joins it).
+__device__ __forceinline__ uint32_t ld_volatile_u32(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.volatile.shared.u32 %0, [%1];" : "=r"(v) : "r"(smem_u32(p)) : "memory");
+  return v;
+}
+__device__ __forceinline__ unsigned long long ld_volatile_u64(const unsigned long long* p) {
+  unsigned long long v;
+  asm volatile("ld.volatile.shared.u64 %0, [%1];" : "=l"(v) : "r"(smem_u32(p)) : "memory");
+  return v;
+}
+__device__ __forceinline__ uint4 ld_volatile_v4(const uint32_t* p) {
+  uint4 v;
+  asm volatile("ld.volatile.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "r"(smem_u32(p))
+               : "memory");
+  return v;
+}
+// Barrier 1 among the consumer warps only (the threshold warp never joins it).
+template <int N>
 __device__ __forceinline__ void consumers_sync() {
-  asm volatile("bar.sync 1, %0;" ::"n"(kConsumers) : "memory");
+  asm volatile("bar.sync 1, %0;" ::"n"(N) : "memory");
 }
 
 // Dot product of 8 bf16 values (one 16-byte chunk of a row) with this lane's 8 channels of q-hat.
@@ -126,12 +181,13 @@ __device__ __forceinline__ float butterfly(float (&v)[Gm::NI], int lane) {
   return v[0];
 }
 
-// Cached length and scored block count of one sequence.  Both sides of the kernel compute
-// the same values (the producer records bad inputs, once, in CTA 0).
+// Cached length, budget and scored block count of one sequence.  Every warp computes the same
+// values (bad inputs are recorded once, by CTA 0's plan).
 struct SeqInfo {
   int n;        // N_b (0 if out of range)
+  int k_eff;    // min(k_b, N_b), k_b clamped to k_max
   int blocks;   // blocks that need scores (0 when nothing is ranked or reported)
-  bool ranked;  // the selection ranks this sequence: histogram needed
+  bool ranked;  // the selection ranks this sequence
 };
 template <int BR>
 __device__ __forceinline__ SeqInfo seq_info(const ScoreParams& p, int b, bool record) {
@@ -147,7 +203,9 @@ __device__ __forceinline__ SeqInfo seq_info(const ScoreParams& p, int b, bool re
   }
   SeqInfo s;
   s.n = n;
-  s.ranked = seq_selection(kb, n).ranked;
+  const SeqSelection sel = seq_selection(kb, n);
+  s.k_eff = sel.k_eff;
+  s.ranked = sel.ranked;
   s.blocks = (s.ranked || p.scores_out != nullptr) ? (n + BR - 1) / BR : 0;
   return s;
 }
@@ -158,25 +216,80 @@ __device__ __forceinline__ void next_scored_seq(const ScoreParams& p, int& b, Se
   while (b < p.B && (si = seq_info<BR>(p, b, false)).blocks == 0) ++b;
 }
 
-template <int R, int D, bool GATED, bool KP8>
-__global__ void __launch_bounds__(kThreads, 1) score_kernel(const ScoreParams p) {
+// Candidate mode: keeps the shared threshold at the bin of the k-th largest key counted so far
+// for the head being scanned.  Counts read while the consumers add to them are at most the true
+// counts, so the bin found is never above the true one; a pass that straddles a change of head
+// (the generation moved on) is discarded by the compare-and-swap.
+template <int BINS>
+__device__ void threshold_warp(const uint32_t* hist, unsigned long long* state, const int* head_k, int lane) {
+  constexpr int PER = BINS / 32;  // bins per lane, lane 0 holding the top ones
+  for (uint32_t it = 0; it < kTauPasses; ++it) {
+    const unsigned long long st = ld_volatile_u64(state);
+    const uint32_t gen = (uint32_t)(st >> 32);
+    if (gen == kTauDone) return;
+    const uint32_t cur = (uint32_t)st;
+    __threadfence_block();
+    const int kk = (int)ld_volatile_u32(reinterpret_cast<const uint32_t*>(head_k));
+    if (kk > 0) {
+      const int lo = BINS - (lane + 1) * PER;
+      uint32_t s = 0u;
+      if (lo + PER > (int)cur) {
+#pragma unroll 4
+        for (int i = 0; i < PER; i += 4) {
+          const uint4 v = ld_volatile_v4(hist + lo + i);
+          const int bin = lo + i;
+          s += (bin + 0 >= (int)cur ? v.x : 0u) + (bin + 1 >= (int)cur ? v.y : 0u) +
+               (bin + 2 >= (int)cur ? v.z : 0u) + (bin + 3 >= (int)cur ? v.w : 0u);
+        }
+      }
+      uint32_t incl = s;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      const uint32_t hit = __ballot_sync(0xffffffffu, incl >= (uint32_t)kk);
+      if (hit != 0u && lane == __ffs(hit) - 1) {
+        uint32_t acc = incl - s;  // counted keys in the bins above this lane's
+        int found = -1;
+        for (int bin = lo + PER - 1; bin >= lo && bin >= (int)cur; --bin) {
+          acc += ld_volatile_u32(hist + bin);
+          if (acc >= (uint32_t)kk) {
+            found = bin;
+            break;
+          }
+        }
+        if (found > (int)cur)
+          atomicCAS(state, st, ((unsigned long long)gen << 32) | (unsigned long long)(uint32_t)found);
+      }
+    }
+    __syncwarp();
+    __nanosleep(256);
+  }
+}
+
+template <int R, int D, bool GATED, bool KP8, bool CANDS>
+__global__ void __launch_bounds__(Cfg<R, GATED, KP8, CANDS>::kThreads, 1) score_kernel(const ScoreParams p) {
+  using C = Cfg<R, GATED, KP8, CANDS>;
   using Gm = Geo<R, KP8>;
   constexpr int BR = Gm::BLOCK_ROWS;
+  constexpr int NW = C::kWarps;
+  constexpr int kConsumers = C::kConsumers;
+  constexpr int kBinShift = CANDS ? 32 - kCandHistBits : kHistShift;
   extern __shared__ __align__(128) unsigned char smem_raw[];
-  Smem<R, D, KP8>& S = *reinterpret_cast<Smem<R, D, KP8>*>(smem_raw);
+  Smem<R, D, GATED, KP8, CANDS>& S = *reinterpret_cast<Smem<R, D, GATED, KP8, CANDS>*>(smem_raw);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 
   if (tid == 0) {
-    for (int s = 0; s < kSlots; ++s) {
-      mbar_init(&S.full[s], 1);
-      mbar_init(&S.empty[s], 1);
-    }
+    for (int s = 0; s < C::kSlots; ++s) mbar_init(&S.full[s], 1);
     fence_barrier_init();
+    S.tau_state = 0ull;
+    S.head_k = 0;
   }
-  for (int i = tid; i < kHistBins; i += kThreads) S.hist[i] = 0u;
+  for (int i = tid; i < C::kBins; i += C::kThreads) S.hist[i] = 0u;
 
-  // ---- this CTA's share of the block list (producer warp) ----
-  if (warp == kConsumerWarps) {
+  // ---- this CTA's share of the block list (warp 0) ----
+  if (warp == 0) {
     // per-lane block counts of sequences lane, lane + 32, ...; the first 32 are kept
     long long mine = 0;
     long long first = 0;
@@ -230,88 +343,136 @@ __global__ void __launch_bounds__(kThreads, 1) score_kernel(const ScoreParams p)
     }
   }
   __syncthreads();
-  // The projected cache (appended to by the previous kernel), the keys, the histograms and the
-  // error word are touched only from here on.
+  // The projected cache (appended to by the previous kernel), the keys or candidates, the
+  // histograms, the record lists and the error word are touched only from here on.
   pdl_wait();
   pdl_trigger();
   const Plan pl = S.plan;
-  const bool gated = GATED;
-  const bool scores = p.scores_out != nullptr;
-  bool waited_ok = true;
 
-  if (warp >= kConsumerWarps) {
-    // ---------------------------------------------------------------- producers
-    // Producer lane L owns ring slot L and issues the CTA's blocks L, L + kSlots, ... into it,
-    // each once consumer warp L % kConsumerWarps has released the slot.
-    const int L = (warp - kConsumerWarps) * 32 + lane;
-    if (L < kSlots && pl.count > L) {
-      const unsigned char* kp = reinterpret_cast<const unsigned char*>(p.kproj);
-      int b = pl.b0, h = pl.h0, c = pl.c0;
-      SeqInfo si = seq_info<BR>(p, b, false);
-      // advance the walk by k blocks
-      auto advance = [&](int k) {
-        while (k > 0 && b < p.B) {
-          const int take = min(k, si.blocks - c);
-          c += take;
-          k -= take;
-          if (c == si.blocks) {
-            c = 0;
-            if (++h == p.Hkv) {
-              h = 0;
-              ++b;
-              next_scored_seq<BR>(p, b, si);
-            }
-          }
-        }
-      };
-      advance(L);
-      const int slot = L;
-      uint32_t phase = 0u;
-      for (int t = L; t < pl.count; t += kSlots) {
-        if (t >= kSlots) {
-          if (!mbar_wait_bounded(&S.empty[slot], phase)) waited_ok = false;
-          phase ^= 1u;
-        }
-        const int row0 = c * BR;
-        const int rows = min(BR, si.n - row0);
-        const int bh = b * p.Hkv + h;
-        // gate values: a whole number of 16-byte units, inside the [cap] row (cap % 4 == 0)
-        const uint32_t lg_bytes = gated ? (uint32_t)((rows + 3) & ~3) * 4u : 0u;
-        unsigned char* dst = S.ring[slot];
-        mbar_arrive_expect_tx(&S.full[slot], (uint32_t)rows * Gm::ROW_BYTES + lg_bytes);
-        if (!p.paged) {
-          bulk_g2s(dst, kp + ((size_t)bh * p.cap + row0) * Gm::ROW_BYTES, (uint32_t)rows * Gm::ROW_BYTES,
-                   &S.full[slot]);
-        } else {
-          const int32_t* pt = p.page_table + (size_t)b * p.max_pages;
-          for (int g = row0; g < row0 + rows;) {
-            const int pr = min(64 - (g & 63), row0 + rows - g);  // rows in this page piece
-            int pg = pt[g >> 6];
-            if (pg < 0 || pg >= p.num_pages) {
-              record_error(p.err, kDevBadPage, (uint32_t)b);
-              pg = 0;
-            }
-            bulk_g2s(dst + (size_t)(g - row0) * Gm::ROW_BYTES,
-                     kp + (((size_t)pg * p.Hkv + h) * 64 + (g & 63)) * Gm::ROW_BYTES, (uint32_t)pr * Gm::ROW_BYTES,
-                     &S.full[slot]);
-            g += pr;
-          }
-        }
-        if (gated) bulk_g2s(dst + kBlockBytes, p.log_g + (size_t)bh * p.cap + row0, lg_bytes, &S.full[slot]);
-        advance(kSlots);
-      }
-      if (!waited_ok) record_error(p.err, kDevWaitTimeout, blockIdx.x);
+  if constexpr (CANDS) {
+    if (warp == NW) {
+      threshold_warp<C::kBins>(S.hist, &S.tau_state, &S.head_k, lane);
+      return;
     }
-    return;
   }
 
-  // ------------------------------------------------------------------ consumers
+  // ------------------------------------------------------------------ consumer warps
+  bool waited_ok = true;
+  const unsigned char* kp = reinterpret_cast<const unsigned char*>(p.kproj);
+  const int my_blocks = pl.count > warp ? (pl.count - warp + NW - 1) / NW : 0;
+
+  // Issue cursor of this warp (lane 0): the warp's i-th block is block warp + i * NW of the share.
+  int ib = pl.b0, ih = pl.h0, ic = pl.c0;
+  SeqInfo isi = seq_info<BR>(p, ib < p.B ? ib : 0, false);
+  auto advance = [&](int k) {
+    while (k > 0 && ib < p.B) {
+      const int take = min(k, isi.blocks - ic);
+      ic += take;
+      k -= take;
+      if (ic == isi.blocks) {
+        ic = 0;
+        if (++ih == p.Hkv) {
+          ih = 0;
+          ++ib;
+          next_scored_seq<BR>(p, ib, isi);
+        }
+      }
+    }
+  };
+  // Copy the block under the cursor into slot `slot` (one bulk copy, or one per 64-token page
+  // piece for the paged layout, plus the block's gate values), then move the cursor to the warp's
+  // next block.
+  auto issue = [&](int slot) {
+    const int row0 = ic * BR;
+    const int rows = min(BR, isi.n - row0);
+    const int bh = ib * p.Hkv + ih;
+    // gate values: a whole number of 16-byte units, inside the [cap] row (cap % 4 == 0)
+    const uint32_t lg_bytes = GATED ? (uint32_t)((rows + 3) & ~3) * 4u : 0u;
+    unsigned char* dst = S.ring[slot];
+    mbar_arrive_expect_tx(&S.full[slot], (uint32_t)rows * Gm::ROW_BYTES + lg_bytes);
+    if (!p.paged) {
+      bulk_g2s(dst, kp + ((size_t)bh * p.cap + row0) * Gm::ROW_BYTES, (uint32_t)rows * Gm::ROW_BYTES, &S.full[slot]);
+    } else {
+      const int32_t* pt = p.page_table + (size_t)ib * p.max_pages;
+      for (int g = row0; g < row0 + rows;) {
+        const int pr = min(64 - (g & 63), row0 + rows - g);  // rows in this page piece
+        int pg = pt[g >> 6];
+        if (pg < 0 || pg >= p.num_pages) {
+          record_error(p.err, kDevBadPage, (uint32_t)ib);
+          pg = 0;
+        }
+        bulk_g2s(dst + (size_t)(g - row0) * Gm::ROW_BYTES,
+                 kp + (((size_t)pg * p.Hkv + ih) * 64 + (g & 63)) * Gm::ROW_BYTES, (uint32_t)pr * Gm::ROW_BYTES,
+                 &S.full[slot]);
+        g += pr;
+      }
+    }
+    if (GATED) bulk_g2s(dst + kBlockBytes, p.log_g + (size_t)bh * p.cap + row0, lg_bytes, &S.full[slot]);
+    advance(NW);
+  };
+  if (lane == 0) {
+    advance(warp);
+    for (int i = 0; i < min(kDepth, my_blocks); ++i) issue(warp * kDepth + i);
+  }
+  __syncwarp();
+
   const uint64_t pol_keep = l2_evict_last();
   const int part = lane % Gm::LPR;  // this lane's 16-byte chunk of each row it loads
   const int rsub = lane / Gm::LPR;  // its row within each load instruction
   float2 qv[Gm::CPL / 2];
   int cur_bh = -1;
   bool cur_ranked = false;
+  // candidate mode: this warp's candidates of the current head and its first block there
+  uint32_t m_cand = 0u;
+  int c_first = 0;
+  const uint32_t* tau_lo = reinterpret_cast<const uint32_t*>(&S.tau_state);  // low word: the bin
+
+  // Candidate mode: pad the warp's count of head `bh` to even and append its record.
+  auto close_record = [&](int bh) {
+    if constexpr (CANDS) {
+      if (m_cand > 0u) {
+        if (lane == 0) {
+          if (m_cand & 1u) {
+            uint2* dst = p.cand + (size_t)bh * p.cand_stride + (size_t)(c_first + (int)(m_cand / BR) * NW) * BR +
+                         m_cand % BR;
+            stg_hint_v2(dst, 0u, 0xffffffffu, pol_keep);
+          }
+          const uint32_t r = atomicAdd(&p.rec_cnt[bh], 1u);
+          if (r < (uint32_t)p.rec_stride)
+            p.recs[(size_t)bh * p.rec_stride + r] =
+                make_uint2((uint32_t)c_first | ((uint32_t)NW << 24), (m_cand + 1u) & ~1u);
+          else
+            record_error(p.err, kDevCandidates, (uint32_t)bh);
+        }
+        m_cand = 0u;
+      }
+    }
+  };
+
+  // Scores of one 32-row batch: this lane's row is lr (< wrows are valid); the key goes to the
+  // keys buffer (keys mode) or, when at or above tau, to the warp's candidates.
+  auto take_key = [&](float u, int bh, int pos, bool valid, uint32_t tau) {
+    const uint32_t key = float_key(u);
+    if constexpr (!CANDS) {
+      if (valid) {
+        stg_hint(p.keys + (size_t)bh * p.cap + pos, key, pol_keep);
+        if (cur_ranked) atomicAdd(&S.hist[key >> kBinShift], 1u);
+      }
+    } else {
+      if (cur_ranked) {
+        const bool em = valid && key >= tau;
+        const uint32_t ball = __ballot_sync(0xffffffffu, em);
+        if (em) {
+          const uint32_t mm = m_cand + (uint32_t)__popc(ball & ((1u << lane) - 1u));
+          uint2* dst = p.cand + (size_t)bh * p.cand_stride + (size_t)(c_first + (int)(mm / BR) * NW) * BR + mm % BR;
+          stg_hint_v2(dst, key, (uint32_t)pos, pol_keep);
+          atomicAdd(&S.hist[key >> kBinShift], 1u);
+        }
+        m_cand += (uint32_t)__popc(ball);
+      }
+    }
+    if (valid && p.scores_out != nullptr) p.scores_out[(size_t)bh * p.cap + pos] = u;
+  };
 
   int b = pl.b0, h = pl.h0, c = pl.c0;
   SeqInfo si = seq_info<BR>(p, b < p.B ? b : 0, false);
@@ -330,15 +491,19 @@ __global__ void __launch_bounds__(kThreads, 1) score_kernel(const ScoreParams p)
       const float* Mrow = p.M + ((size_t)h * R + (qrow ? qj : 0)) * D + qpart * CH;
 #pragma unroll
       for (int i = 0; i < CH; ++i) mreg[i] = Mrow[i];
-      consumers_sync();  // every warp is done with the previous head's rows
+      consumers_sync<kConsumers>();  // every warp is done with the previous head's rows
       if (cur_bh >= 0) {
-        uint32_t* gh = p.hist + (size_t)cur_bh * kHistBins;
-        for (int i = tid; i < kHistBins; i += kConsumers) {
-          const uint32_t v = S.hist[i];
-          if (v) {
-            if (cur_ranked) atomicAdd(&gh[i], v);
-            S.hist[i] = 0u;
+        if constexpr (!CANDS) {
+          uint32_t* gh = p.hist + (size_t)cur_bh * kHistBins;
+          for (int i = tid; i < C::kBins; i += kConsumers) {
+            const uint32_t v = S.hist[i];
+            if (v) {
+              if (cur_ranked) atomicAdd(&gh[i], v);
+              S.hist[i] = 0u;
+            }
           }
+        } else {
+          for (int i = tid; i < C::kBins; i += kConsumers) S.hist[i] = 0u;
         }
       }
       if (tid < D) {
@@ -347,7 +512,7 @@ __global__ void __launch_bounds__(kThreads, 1) score_kernel(const ScoreParams p)
         for (int g = 0; g < p.G; ++g) sq += __bfloat162float(qg[(size_t)g * D]);
         S.qbar[tid] = sq / (float)p.G;
       }
-      consumers_sync();
+      consumers_sync<kConsumers>();
       float sp = 0.f;
 #pragma unroll
       for (int i = 0; i < CH; ++i) sp = fmaf(mreg[i], S.qbar[qpart * CH + i], sp);
@@ -355,7 +520,16 @@ __global__ void __launch_bounds__(kThreads, 1) score_kernel(const ScoreParams p)
       for (int o = TPR / 2; o; o >>= 1) sp += __shfl_xor_sync(0xffffffffu, sp, o);
       // FP8: the head's scale multiplies q-hat, so the codes are used as they are
       if (qpart == 0 && qrow) S.qhat[qj] = sp * p.sigma * (KP8 ? p.kproj_scale[h] : 1.f);
-      consumers_sync();
+      if constexpr (CANDS) {
+        if (tid == 0) {
+          // the histogram is clear (previous barrier); a new generation restarts the threshold
+          *reinterpret_cast<volatile int*>(&S.head_k) = si.ranked ? si.k_eff : 0;
+          __threadfence_block();
+          const unsigned long long st = ld_volatile_u64(&S.tau_state);
+          atomicExch(&S.tau_state, ((st >> 32) + 1ull) << 32);
+        }
+      }
+      consumers_sync<kConsumers>();
 #pragma unroll
       for (int e = 0; e < Gm::CPL / 2; ++e)
         qv[e] = make_float2(S.qhat[part * Gm::CPL + 2 * e], S.qhat[part * Gm::CPL + 2 * e + 1]);
@@ -363,15 +537,18 @@ __global__ void __launch_bounds__(kThreads, 1) score_kernel(const ScoreParams p)
       cur_ranked = si.ranked;
     }
 
-    // ---- this warp's blocks of the segment: CTA block indices j = t.. with j % 16 == warp ----
-    for (int j = t + ((warp - t) % kConsumerWarps + kConsumerWarps) % kConsumerWarps; j < t + seg;
-         j += kConsumerWarps) {
-      const int slot = j % kSlots;
-      if (!mbar_wait_bounded(&S.full[slot], (uint32_t)(j / kSlots) & 1u)) waited_ok = false;
+    // ---- this warp's blocks of the segment: CTA block indices j = t.. with j % NW == warp ----
+    const int j0 = t + ((warp - t) % NW + NW) % NW;
+    if constexpr (CANDS) c_first = c + (j0 - t);
+    for (int j = j0; j < t + seg; j += NW) {
+      const int i = (j - warp) / NW;  // the warp's own block number
+      const int slot = warp * kDepth + i % kDepth;
+      if (!mbar_wait_bounded(&S.full[slot], (uint32_t)(i / kDepth) & 1u)) waited_ok = false;
       const int row0 = (c + (j - t)) * BR;
       const int rows = min(BR, si.n - row0);
       const unsigned char* st = S.ring[slot];
       const float* lgs = reinterpret_cast<const float*>(st + kBlockBytes);
+      const uint32_t tau = CANDS ? ld_volatile_u32(tau_lo) << (32 - kCandHistBits) : 0u;
       if (rows == BR) {
         // full block: every row valid, no per-row tests
 #pragma unroll
@@ -379,18 +556,14 @@ __global__ void __launch_bounds__(kThreads, 1) score_kernel(const ScoreParams p)
           const unsigned char* sb = st + (size_t)bt * 32 * Gm::ROW_BYTES;
           float v[Gm::NI];
 #pragma unroll
-          for (int i = 0; i < Gm::NI; ++i) {
-            const uint4 w = *reinterpret_cast<const uint4*>(sb + (size_t)(i * Gm::RPI + rsub) * Gm::ROW_BYTES + part * 16);
-            if constexpr (KP8) v[i] = dot16_fp8(qv, w); else v[i] = dot8(qv, w);
+          for (int ii = 0; ii < Gm::NI; ++ii) {
+            const uint4 w = *reinterpret_cast<const uint4*>(sb + (size_t)(ii * Gm::RPI + rsub) * Gm::ROW_BYTES + part * 16);
+            if constexpr (KP8) v[ii] = dot16_fp8(qv, w); else v[ii] = dot8(qv, w);
           }
           const float u0 = butterfly<Gm>(v, lane);
           const int lr = part * Gm::RPI + rsub;
           const float u = GATED ? fmaf(p.lam, lgs[bt * 32 + lr], u0) : u0;
-          const uint32_t key = float_key(u);
-          const size_t kidx = (size_t)bh * p.cap + row0 + bt * 32 + lr;
-          stg_hint(p.keys + kidx, key, pol_keep);
-          if (scores) p.scores_out[kidx] = u;
-          if (cur_ranked) atomicAdd(&S.hist[key >> kHistShift], 1u);
+          take_key(u, bh, row0 + bt * 32 + lr, true, tau);
         }
       } else {
 #pragma unroll
@@ -400,28 +573,24 @@ __global__ void __launch_bounds__(kThreads, 1) score_kernel(const ScoreParams p)
             const unsigned char* sb = st + (size_t)bt * 32 * Gm::ROW_BYTES;
             float v[Gm::NI];
 #pragma unroll
-            for (int i = 0; i < Gm::NI; ++i) {
-              const int lr = i * Gm::RPI + rsub;
+            for (int ii = 0; ii < Gm::NI; ++ii) {
+              const int lr = ii * Gm::RPI + rsub;
               uint4 w = make_uint4(0u, 0u, 0u, 0u);
               if (lr < wrows) w = *reinterpret_cast<const uint4*>(sb + (size_t)lr * Gm::ROW_BYTES + part * 16);
-              if constexpr (KP8) v[i] = dot16_fp8(qv, w); else v[i] = dot8(qv, w);
+              if constexpr (KP8) v[ii] = dot16_fp8(qv, w); else v[ii] = dot8(qv, w);
             }
             const float u0 = butterfly<Gm>(v, lane);
             const int lr = part * Gm::RPI + rsub;
-            if (lr < wrows) {
-              const float u = GATED ? fmaf(p.lam, lgs[bt * 32 + lr], u0) : u0;
-              const uint32_t key = float_key(u);
-              const size_t kidx = (size_t)bh * p.cap + row0 + bt * 32 + lr;
-              stg_hint(p.keys + kidx, key, pol_keep);
-              if (scores) p.scores_out[kidx] = u;
-              if (cur_ranked) atomicAdd(&S.hist[key >> kHistShift], 1u);
-            }
+            const bool valid = lr < wrows;
+            const float u = (GATED && valid) ? fmaf(p.lam, lgs[bt * 32 + lr], u0) : u0;
+            take_key(u, bh, row0 + bt * 32 + lr, valid, tau);
           }
         }
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&S.empty[slot]);
+      __syncwarp();  // every lane is done with the slot
+      if (lane == 0 && i + kDepth < my_blocks) issue(slot);
     }
+    close_record(bh);
 
     // ---- next head ----
     t += seg;
@@ -432,26 +601,40 @@ __global__ void __launch_bounds__(kThreads, 1) score_kernel(const ScoreParams p)
       next_scored_seq<BR>(p, b, si);
     }
   }
-  if (cur_bh >= 0) {
-    consumers_sync();
-    uint32_t* gh = p.hist + (size_t)cur_bh * kHistBins;
-    for (int i = tid; i < kHistBins; i += kConsumers) {
-      const uint32_t v = S.hist[i];
-      if (v && cur_ranked) atomicAdd(&gh[i], v);
+  consumers_sync<kConsumers>();
+  if constexpr (!CANDS) {
+    if (cur_bh >= 0) {
+      uint32_t* gh = p.hist + (size_t)cur_bh * kHistBins;
+      for (int i = tid; i < C::kBins; i += kConsumers) {
+        const uint32_t v = S.hist[i];
+        if (v && cur_ranked) atomicAdd(&gh[i], v);
+      }
     }
+  } else {
+    if (tid == 0) atomicExch(&S.tau_state, (unsigned long long)kTauDone << 32);
   }
   if (!waited_ok) record_error(p.err, kDevWaitTimeout, blockIdx.x);
+}
+
+template <int R, int D, bool GATED, bool KP8, bool CANDS>
+cudaError_t launch_v(const ScoreParams& p, cudaStream_t stream) {
+  using C = Cfg<R, GATED, KP8, CANDS>;
+  auto kern = score_kernel<R, D, GATED, KP8, CANDS>;
+  const int smem = (int)sizeof(Smem<R, D, GATED, KP8, CANDS>);
+  cudaError_t e = prepare_kernel((const void*)kern, smem);
+  if (e != cudaSuccess) return e;
+  return launch_pdl(kern, dim3((unsigned)p.ctas), dim3(C::kThreads), (size_t)smem, stream, p);
 }
 
 template <int R, int D>
 cudaError_t launch_rd(const ScoreParams& p, cudaStream_t stream) {
   const bool gated = p.log_g != nullptr;
-  const int smem = p.fp8 ? (int)sizeof(Smem<R, D, true>) : (int)sizeof(Smem<R, D, false>);
-  auto kern = p.fp8 ? (gated ? score_kernel<R, D, true, true> : score_kernel<R, D, false, true>)
-                    : (gated ? score_kernel<R, D, true, false> : score_kernel<R, D, false, false>);
-  cudaError_t e = prepare_kernel((const void*)kern, smem);
-  if (e != cudaSuccess) return e;
-  return launch_pdl(kern, dim3((unsigned)p.ctas), dim3(kThreads), (size_t)smem, stream, p);
+  if (p.cands) {
+    if (p.fp8) return gated ? launch_v<R, D, true, true, true>(p, stream) : launch_v<R, D, false, true, true>(p, stream);
+    return gated ? launch_v<R, D, true, false, true>(p, stream) : launch_v<R, D, false, false, true>(p, stream);
+  }
+  if (p.fp8) return gated ? launch_v<R, D, true, true, false>(p, stream) : launch_v<R, D, false, true, false>(p, stream);
+  return gated ? launch_v<R, D, true, false, false>(p, stream) : launch_v<R, D, false, false, false>(p, stream);
 }
 
 }  // namespace
@@ -463,6 +646,7 @@ void plan_score(ScoreParams& p, int num_sms) {
   long long ctas = num_sms;
   if (ctas > blocks) ctas = blocks;
   p.ctas = (int)(ctas < 1 ? 1 : ctas);
+  p.block_rows = br;
 }
 
 cudaError_t launch_score(const ScoreParams& p, cudaStream_t stream) {

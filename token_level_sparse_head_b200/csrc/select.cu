@@ -36,6 +36,7 @@ constexpr int kMaxWords = kChunkMax / 32;     // bitmap words per CTA
 constexpr int kCap = 4096;                    // candidate list entries (CTA 0: the whole head's)
 constexpr int kMaxTies = 256;                 // ties on T resolved by CTA 0; more take the slow path
 constexpr uint32_t kFast = 1u, kSlow = 2u;
+constexpr long long kSmemLimitSel = 227 * 1024;
 
 struct Found {
   uint32_t digit, above, eq, pad;
@@ -554,9 +555,217 @@ __global__ void __launch_bounds__(THREADS, 1) select_topk_kernel(const SelectPar
   if (!waited_ok) record_error(p.err, kDevWaitTimeout, (uint32_t)bh);
 }
 
+// ---------------------------------------------------------------------------------------------
+// Candidate mode.  The score kernel has left, per head, a list of records (first block and block
+// stride, even count) that point at (key, position) pairs: every key at or above a lower bound of the head's
+// k-th largest key, plus sentinels of key 0.  Since the candidates hold every key that can be
+// selected and at least k of them, the k-th largest candidate key is the head's k-th largest
+// key T.  One CTA per head: the candidates are copied into shared memory (one bulk copy per block
+// run of a record) when they fit, else every pass reads them from L2.  T is found as three radix
+// digits (11, 11 and 10 bits); when T has more ties than the budget takes, the lowest positions
+// among them are found as two 9-bit digits of the position.  The chosen positions are set in a
+// bitmap of the head and written out in ascending order.
+constexpr int kCandBins = 2048;
+
+struct CandCtl {
+  uint32_t hist[kCandBins];
+  uint32_t wsum[32];
+  Found found;
+  uint64_t bar;
+  uint32_t pad[2];
+};
+static_assert(sizeof(CandCtl) % 16 == 0, "candidate array alignment");
+
+template <int THREADS>
+__global__ void __launch_bounds__(THREADS, 1) select_cand_kernel(const SelectParams p) {
+  extern __shared__ __align__(128) unsigned char smem_raw[];
+  CandCtl& S = *reinterpret_cast<CandCtl*>(smem_raw);
+  uint32_t* bm = reinterpret_cast<uint32_t*>(smem_raw + sizeof(CandCtl));
+  uint2* cs = reinterpret_cast<uint2*>(smem_raw + sizeof(CandCtl) + (size_t)p.bm_words * 4);
+  const int tid = threadIdx.x;
+  const int bh = blockIdx.x;
+  const int b = bh / p.Hkv;
+
+  // per-sequence values (range errors were recorded by the score kernel)
+  int n = p.seqlens[b];
+  if (n < 0 || n > p.cap) n = 0;
+  const SeqSelection sel = seq_selection(min(p.kvec[b], p.k_max), n);
+  const int k_eff = sel.k_eff;
+  int32_t* idx = p.idx_out + (size_t)bh * p.k_max;
+
+  if (!sel.ranked) {
+    // Nothing to rank (the scan wrote no candidates): the first k_eff positions, or none.
+    pdl_wait();
+    pdl_trigger();
+    for (int j = tid; j < p.k_max; j += THREADS) idx[j] = (j < k_eff) ? j : -1;
+    return;
+  }
+
+  const int nwords = (n + 31) >> 5;
+  for (int i = tid; i < nwords; i += THREADS) bm[i] = 0u;
+  for (int i = tid; i < kCandBins; i += THREADS) S.hist[i] = 0u;
+  if (tid == 0) {
+    mbar_init(&S.bar, 1);
+    fence_barrier_init();
+    S.found = Found{};
+  }
+  __syncthreads();
+  // The candidates, records and record counts of the score pass are read only from here on.
+  pdl_wait();
+  pdl_trigger();
+
+  const uint32_t R = min(p.rec_cnt[bh], (uint32_t)p.rec_stride);
+  const uint2* recs = p.recs + (size_t)bh * p.rec_stride;
+  const uint2* cand = p.cand + (size_t)bh * p.cand_stride;
+  const int BR = p.block_rows;
+  const int lbr = __ffs(BR) - 1;  // BR is a power of two
+  // a record is (first block | block stride << 24, even count)
+  // thread t sums the counts of records [r0, r1)
+  const int rpt = (int)((R + THREADS - 1) / THREADS);
+  const int r0 = min(tid * rpt, (int)R), r1 = min(r0 + rpt, (int)R);
+  uint32_t mine = 0u;
+  for (int r = r0; r < r1; ++r) mine += recs[r].y;
+  uint32_t total;
+  const uint32_t off = block_excl_scan<THREADS>(mine, S.wsum, &total);
+  if (tid == 0) p.rec_cnt[bh] = 0u;  // every thread has read it: ready for the next scan
+
+  if ((uint32_t)k_eff > total) {
+    // Cannot happen (every key >= T is a candidate); leave a defined output and report it.
+    if (tid == 0) record_error(p.err, kDevCandidates, (uint32_t)bh);
+    for (int j = tid; j < p.k_max; j += THREADS) idx[j] = -1;
+    return;
+  }
+
+  bool waited_ok = true;
+  const bool in_smem = total <= (uint32_t)p.cand_smem;
+  if (in_smem) {
+    if (tid == 0) mbar_arrive_expect_tx(&S.bar, total * 8u);
+    __syncthreads();
+    uint32_t o = off;
+    for (int r = r0; r < r1; ++r) {
+      const uint2 rc = recs[r];
+      for (uint32_t e = 0; e < rc.y; e += (uint32_t)BR) {
+        const uint32_t cnt = min((uint32_t)BR, rc.y - e);
+        bulk_g2s(cs + o + e, cand + ((size_t)(rc.x & 0xffffffu) + (size_t)(e >> lbr) * (rc.x >> 24)) * BR, cnt * 8u,
+                 &S.bar);
+      }
+      o += rc.y;
+    }
+    if (!mbar_wait_bounded(&S.bar, 0u)) waited_ok = false;
+  }
+
+  // fn(key, position) over every candidate (sentinels included), this thread's share of them
+  auto for_each = [&](auto&& fn) {
+    if (in_smem) {
+      for (uint32_t e = tid; e < total; e += THREADS) {
+        const uint2 v = cs[e];
+        fn(v.x, v.y);
+      }
+    } else {
+      for (uint32_t r = 0; r < R; ++r) {
+        const uint2 rc = recs[r];
+        for (uint32_t e = tid; e < rc.y; e += THREADS) {
+          const uint2 v =
+              cand[((size_t)(rc.x & 0xffffffu) + (size_t)(e >> lbr) * (rc.x >> 24)) * BR + (e & (uint32_t)(BR - 1))];
+          fn(v.x, v.y);
+        }
+      }
+    }
+  };
+  auto clear_hist = [&]() {
+    for (int i = tid; i < kCandBins; i += THREADS) S.hist[i] = 0u;
+    __syncthreads();
+  };
+
+  // ---- T as three digits of the key: 11, 11 and 10 bits ----
+  for_each([&](uint32_t key, uint32_t) { atomicAdd(&S.hist[key >> 21], 1u); });
+  __syncthreads();
+  find_digit<kCandBins, THREADS>(S.hist, (uint32_t)k_eff, S.wsum, &S.found);
+  const uint32_t d1 = S.found.digit;
+  uint32_t k_rem = (uint32_t)k_eff - S.found.above;
+  clear_hist();
+  for_each([&](uint32_t key, uint32_t) {
+    if ((key >> 21) == d1) atomicAdd(&S.hist[(key >> 10) & (kCandBins - 1)], 1u);
+  });
+  __syncthreads();
+  find_digit<kCandBins, THREADS>(S.hist, k_rem, S.wsum, &S.found);
+  const uint32_t pre = (d1 << 11) | S.found.digit;
+  k_rem -= S.found.above;
+  clear_hist();
+  for_each([&](uint32_t key, uint32_t) {
+    if ((key >> 10) == pre) atomicAdd(&S.hist[key & 1023u], 1u);
+  });
+  __syncthreads();
+  find_digit<1024, THREADS>(S.hist, k_rem, S.wsum, &S.found);
+  const uint32_t T = (pre << 10) | S.found.digit;
+  const uint32_t need = k_rem - S.found.above;  // ties on T to take, 1 <= need <= eq
+  const uint32_t eq = S.found.eq;
+
+  // ---- ties: the need lowest positions among the keys equal to T (positions < 2^18) ----
+  uint32_t cut = 0xffffffffu;
+  if (need < eq) {
+    clear_hist();
+    for_each([&](uint32_t key, uint32_t pos) {
+      if (key == T) atomicAdd(&S.hist[511u - (pos >> 9)], 1u);
+    });
+    __syncthreads();
+    find_digit<512, THREADS>(S.hist, need, S.wsum, &S.found);
+    const uint32_t ph = 511u - S.found.digit;
+    const uint32_t need2 = need - S.found.above;
+    clear_hist();
+    for_each([&](uint32_t key, uint32_t pos) {
+      if (key == T && (pos >> 9) == ph) atomicAdd(&S.hist[511u - (pos & 511u)], 1u);
+    });
+    __syncthreads();
+    find_digit<512, THREADS>(S.hist, need2, S.wsum, &S.found);
+    cut = (ph << 9) | (511u - S.found.digit);
+  }
+
+  // ---- the chosen positions into the bitmap ----
+  for_each([&](uint32_t key, uint32_t pos) {
+    if (key > T || (key == T && pos <= cut)) atomicOr(&bm[pos >> 5], 1u << (pos & 31));
+  });
+  __syncthreads();
+
+  // ---- ordered output ----
+  {
+    const int wpt = (nwords + THREADS - 1) / THREADS;
+    const int w0 = min(tid * wpt, nwords), w1 = min(w0 + wpt, nwords);
+    uint32_t cnt = 0u;
+    for (int w = w0; w < w1; ++w) cnt += (uint32_t)__popc(bm[w]);
+    uint32_t tot;
+    uint32_t o = block_excl_scan<THREADS>(cnt, S.wsum, &tot);
+    for (int w = w0; w < w1; ++w) {
+      uint32_t bits = bm[w];
+      while (bits) {
+        const int e = __ffs(bits) - 1;
+        bits &= bits - 1u;
+        if (o < (uint32_t)k_eff) idx[o] = w * 32 + e;
+        ++o;
+      }
+    }
+  }
+  for (int j = k_eff + tid; j < p.k_max; j += THREADS) idx[j] = -1;
+  if (!waited_ok) record_error(p.err, kDevWaitTimeout, (uint32_t)bh);
+}
+
 }  // namespace
 
 bool plan_select(SelectParams& p, int num_sms) {
+  if (p.cands) {
+    // one CTA per head; the candidates of a whole head in shared memory when they fit
+    p.cluster = 1;
+    p.threads = 1024;
+    p.chunk = p.cap;
+    p.bm_words = (((p.cap + 31) / 32) + 3) & ~3;
+    const long long fixed = (long long)sizeof(CandCtl) + (long long)p.bm_words * 4;
+    long long want = fixed + (long long)p.cand_stride * 8;
+    if (want > kSmemLimitSel) want = kSmemLimitSel;
+    if (want < fixed + 16) return false;
+    p.smem_bytes = (int)want;
+    p.cand_smem = (int)((want - fixed) / 8);
+    return true;
+  }
   const int heads = p.B * p.Hkv;
   // One CTA per SM.  Split a head over a cluster while its chunk is too long, and while the
   // grid still leaves SMs idle (up to the portable cluster size).
@@ -575,6 +784,12 @@ bool plan_select(SelectParams& p, int num_sms) {
 }
 
 cudaError_t launch_select(const SelectParams& p, cudaStream_t stream) {
+  if (p.cands) {
+    auto kern = select_cand_kernel<1024>;
+    const cudaError_t e = prepare_kernel((const void*)kern, p.smem_bytes);
+    if (e != cudaSuccess) return e;
+    return launch_pdl(kern, dim3((unsigned)(p.B * p.Hkv)), dim3(1024u), (size_t)p.smem_bytes, stream, p);
+  }
   auto kern = p.threads == 512 ? select_topk_kernel<512> : select_topk_kernel<1024>;
   const cudaError_t e = prepare_kernel((const void*)kern, p.smem_bytes, p.cluster > 8);
   if (e != cudaSuccess) return e;
