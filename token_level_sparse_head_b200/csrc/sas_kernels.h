@@ -46,7 +46,8 @@ struct ScoreParams {
   const int32_t* kvec;         // [B]
   const float* log_g;          // [B][Hkv][cap] or null
   uint32_t* keys;              // workspace: [B][Hkv][cap] order-preserving keys of u_i
-  uint32_t* hist;              // workspace: [B][Hkv][kHistBins] counts of the keys' first digit (zero on entry)
+  uint32_t* hist;              // workspace, zero on entry: keys mode [B*Hkv][kHistBins] counts of the keys'
+                               // top 13 bits; candidate mode [B*Hkv][4096] counts of the candidates' top 12
   float* scores_out;           // [B][Hkv][cap] or null
   uint32_t* err;
   int B, Hq, Hkv, G, d, r, cap, max_pages, num_pages, paged, k_max;
@@ -87,7 +88,7 @@ struct SelectParams {
   uint32_t* rec_cnt;           // cleared here after use
   int cand_stride, rec_stride, block_rows;
   int bm_words;                // bitmap words in shared memory
-  int cand_smem;               // candidates that fit in shared memory
+  int rec_cap;                 // records per head held in shared memory (>= 16 * scan CTAs)
 };
 // Chooses cluster size and chunk (keys mode) or the shared-memory split (candidate mode) for a
 // shape; returns false if unsupported.

@@ -10,20 +10,24 @@
 //   keys mode        every key is written to the workspace (L2 evict-last hint) and a histogram
 //                    of the keys' top 13 bits is accumulated per (b, h);
 //   candidate mode   only keys at or above a running lower bound tau of the head's k-th largest
-//                    key are written, as (key, position) pairs.  The k-th largest key among the
-//                    rows a CTA has scanned so far can only be at or below the k-th largest of the
-//                    whole head, so a key below tau can never be selected and is dropped.  A
-//                    threshold warp keeps tau up to date from a shared-memory histogram of the
-//                    written keys' top 12 bits.  With long per-CTA segments (many heads) this
-//                    writes a few k keys per head instead of N.
+//                    key are written, as (key, position) pairs.  Every written key is also counted
+//                    in a per-head histogram of its top 12 bits in global memory, shared by all
+//                    CTAs that scan the head.  The k-th largest of the keys counted so far can
+//                    only be at or below the k-th largest of the whole head, so a key below tau
+//                    can never be selected and is dropped.  A threshold warp per CTA keeps tau at
+//                    the bin of that k-th largest counted key, reading the shared histogram; with
+//                    many heads this writes a few k keys per head instead of N, and the selection
+//                    takes its first digit from the histogram.
 //
 // Persistent kernel, one CTA per SM.  The work is the list of 4 KB blocks of projected rows
 // (64 rows at r = 32 in bf16) of every (b, h) that needs scores, in (b, h, position) order; each
 // CTA takes one contiguous, equal share of it.  Its consumer warps take the share's blocks in
-// turn; each warp owns three ring slots in shared memory and keeps them full itself: lane 0
-// issues the bulk copy (TMA engine, mbarrier completion) of the warp's next block into a slot as
-// soon as the warp has finished reading it, so no warp waits on another to release a slot.  Per
-// 32-row batch the lanes form 16-byte dot products with q-hat and meet in a transposing butterfly.
+// turn; each warp owns two ring slots in shared memory and keeps them full itself: once its
+// lanes have moved a landed block into registers, lane 0 issues the bulk copy (TMA engine,
+// mbarrier completion) of the warp's next block into that slot, and only then does the warp
+// compute, so a slot is out of flight only for the few shared-memory loads that empty it and no
+// warp waits on another.  Per 32-row batch the lanes form 16-byte dot products with q-hat and
+// meet in a transposing butterfly.
 //
 // Candidate storage: a warp writes the candidates of its blocks of one head, in order, into the
 // 64-row slot ranges of those same blocks (the n-th candidate into the (n / BR)-th of its blocks,
@@ -41,7 +45,7 @@ namespace sas {
 namespace {
 
 constexpr int kBlockBytes = 4096;   // projected bytes per block (one ring stage)
-constexpr int kDepth = 3;           // ring slots per consumer warp
+constexpr int kDepth = 2;           // ring slots per consumer warp
 constexpr int kMaxWarps = 16;       // consumer warps per CTA at most
 constexpr int kSmemLimit = 227 * 1024;
 constexpr int kSmemMisc = 2048;     // q-bar, q-hat, barriers, plan and threshold state (upper bound)
@@ -61,12 +65,12 @@ struct Geo {
   static constexpr int LOG_LPR = LPR == 1 ? 0 : LPR == 2 ? 1 : LPR == 4 ? 2 : 3;
 };
 
-// Block shape of one instantiation: as many consumer warps (three slots each) as shared memory
+// Block shape of one instantiation: as many consumer warps (two slots each) as shared memory
 // holds next to the histogram, at most 16; candidate mode adds the threshold warp.
 template <int R, bool GATED, bool KP8, bool CANDS>
 struct Cfg {
   using Gm = Geo<R, KP8>;
-  static constexpr int kBins = CANDS ? (1 << kCandHistBits) : kHistBins;
+  static constexpr int kBins = CANDS ? 4 : kHistBins;  // candidate mode counts in global memory
   static constexpr int kSlotBytes = kBlockBytes + (GATED ? Gm::BLOCK_ROWS * 4 : 0);
   static constexpr int kMaxSlots = (kSmemLimit - kSmemMisc - kBins * 4) / kSlotBytes;
   static constexpr int kWarps = kMaxSlots / kDepth >= kMaxWarps ? kMaxWarps : kMaxSlots / kDepth;
@@ -92,6 +96,7 @@ struct Smem {
   uint64_t full[C::kSlots];
   unsigned long long tau_state;  // candidate mode: (generation << 32) | threshold bin
   int head_k;                    // candidate mode: k_eff of the head being scanned (0: none)
+  int head_bh;                   // candidate mode: that head's (b * Hkv + h)
   Plan plan;
 };
 
@@ -113,6 +118,9 @@ __device__ __forceinline__ void stg_hint(uint32_t* ptr, uint32_t v, uint64_t pol
 }
 __device__ __forceinline__ void stg_hint_v2(uint2* ptr, uint32_t a, uint32_t b, uint64_t pol) {
   asm volatile("st.global.L2::cache_hint.v2.u32 [%0], {%1, %2}, %3;" ::"l"(ptr), "r"(a), "r"(b), "l"(pol) : "memory");
+}
+__device__ __forceinline__ void red_add(uint32_t* p) {
+  asm volatile("red.relaxed.gpu.global.add.u32 [%0], 1;" ::"l"(p) : "memory");
 }
 __device__ __forceinline__ uint32_t ld_volatile_u32(const uint32_t* p) {
   uint32_t v;
@@ -216,12 +224,14 @@ __device__ __forceinline__ void next_scored_seq(const ScoreParams& p, int& b, Se
   while (b < p.B && (si = seq_info<BR>(p, b, false)).blocks == 0) ++b;
 }
 
-// Candidate mode: keeps the shared threshold at the bin of the k-th largest key counted so far
-// for the head being scanned.  Counts read while the consumers add to them are at most the true
-// counts, so the bin found is never above the true one; a pass that straddles a change of head
-// (the generation moved on) is discarded by the compare-and-swap.
-template <int BINS>
-__device__ void threshold_warp(const uint32_t* hist, unsigned long long* state, const int* head_k, int lane) {
+// Candidate mode: keeps the CTA's threshold at the bin of the k-th largest key counted so far for
+// the head being scanned, over every CTA that scans it (the global histogram).  Counts read while
+// other warps still add to them are at most the true counts, so the bin found is never above the
+// true one; a pass that straddles a change of head (the generation moved on) is discarded by the
+// compare-and-swap.
+__device__ void threshold_warp(const uint32_t* ghist, unsigned long long* state, const int* head_k,
+                               const int* head_bh, int lane) {
+  constexpr int BINS = 1 << kCandHistBits;
   constexpr int PER = BINS / 32;  // bins per lane, lane 0 holding the top ones
   for (uint32_t it = 0; it < kTauPasses; ++it) {
     const unsigned long long st = ld_volatile_u64(state);
@@ -230,13 +240,15 @@ __device__ void threshold_warp(const uint32_t* hist, unsigned long long* state, 
     const uint32_t cur = (uint32_t)st;
     __threadfence_block();
     const int kk = (int)ld_volatile_u32(reinterpret_cast<const uint32_t*>(head_k));
+    const int bh = (int)ld_volatile_u32(reinterpret_cast<const uint32_t*>(head_bh));
     if (kk > 0) {
+      const uint32_t* H = ghist + (size_t)bh * BINS;
       const int lo = BINS - (lane + 1) * PER;
       uint32_t s = 0u;
       if (lo + PER > (int)cur) {
-#pragma unroll 4
+#pragma unroll 8
         for (int i = 0; i < PER; i += 4) {
-          const uint4 v = ld_volatile_v4(hist + lo + i);
+          const uint4 v = __ldcg(reinterpret_cast<const uint4*>(H + lo + i));
           const int bin = lo + i;
           s += (bin + 0 >= (int)cur ? v.x : 0u) + (bin + 1 >= (int)cur ? v.y : 0u) +
                (bin + 2 >= (int)cur ? v.z : 0u) + (bin + 3 >= (int)cur ? v.w : 0u);
@@ -253,7 +265,7 @@ __device__ void threshold_warp(const uint32_t* hist, unsigned long long* state, 
         uint32_t acc = incl - s;  // counted keys in the bins above this lane's
         int found = -1;
         for (int bin = lo + PER - 1; bin >= lo && bin >= (int)cur; --bin) {
-          acc += ld_volatile_u32(hist + bin);
+          acc += __ldcg(H + bin);
           if (acc >= (uint32_t)kk) {
             found = bin;
             break;
@@ -264,7 +276,7 @@ __device__ void threshold_warp(const uint32_t* hist, unsigned long long* state, 
       }
     }
     __syncwarp();
-    __nanosleep(256);
+    __nanosleep(128);
   }
 }
 
@@ -285,6 +297,7 @@ __global__ void __launch_bounds__(Cfg<R, GATED, KP8, CANDS>::kThreads, 1) score_
     fence_barrier_init();
     S.tau_state = 0ull;
     S.head_k = 0;
+    S.head_bh = 0;
   }
   for (int i = tid; i < C::kBins; i += C::kThreads) S.hist[i] = 0u;
 
@@ -351,7 +364,7 @@ __global__ void __launch_bounds__(Cfg<R, GATED, KP8, CANDS>::kThreads, 1) score_
 
   if constexpr (CANDS) {
     if (warp == NW) {
-      threshold_warp<C::kBins>(S.hist, &S.tau_state, &S.head_k, lane);
+      threshold_warp(p.hist, &S.tau_state, &S.head_k, &S.head_bh, lane);
       return;
     }
   }
@@ -466,7 +479,7 @@ __global__ void __launch_bounds__(Cfg<R, GATED, KP8, CANDS>::kThreads, 1) score_
           const uint32_t mm = m_cand + (uint32_t)__popc(ball & ((1u << lane) - 1u));
           uint2* dst = p.cand + (size_t)bh * p.cand_stride + (size_t)(c_first + (int)(mm / BR) * NW) * BR + mm % BR;
           stg_hint_v2(dst, key, (uint32_t)pos, pol_keep);
-          atomicAdd(&S.hist[key >> kBinShift], 1u);
+          red_add(p.hist + (size_t)bh * (1 << kCandHistBits) + (key >> kBinShift));
         }
         m_cand += (uint32_t)__popc(ball);
       }
@@ -502,8 +515,6 @@ __global__ void __launch_bounds__(Cfg<R, GATED, KP8, CANDS>::kThreads, 1) score_
               S.hist[i] = 0u;
             }
           }
-        } else {
-          for (int i = tid; i < C::kBins; i += kConsumers) S.hist[i] = 0u;
         }
       }
       if (tid < D) {
@@ -522,8 +533,9 @@ __global__ void __launch_bounds__(Cfg<R, GATED, KP8, CANDS>::kThreads, 1) score_
       if (qpart == 0 && qrow) S.qhat[qj] = sp * p.sigma * (KP8 ? p.kproj_scale[h] : 1.f);
       if constexpr (CANDS) {
         if (tid == 0) {
-          // the histogram is clear (previous barrier); a new generation restarts the threshold
+          // a new generation restarts the threshold for the new head
           *reinterpret_cast<volatile int*>(&S.head_k) = si.ranked ? si.k_eff : 0;
+          *reinterpret_cast<volatile int*>(&S.head_bh) = bh;
           __threadfence_block();
           const unsigned long long st = ld_volatile_u64(&S.tau_state);
           atomicExch(&S.tau_state, ((st >> 32) + 1ull) << 32);
@@ -547,48 +559,37 @@ __global__ void __launch_bounds__(Cfg<R, GATED, KP8, CANDS>::kThreads, 1) score_
       const int row0 = (c + (j - t)) * BR;
       const int rows = min(BR, si.n - row0);
       const unsigned char* st = S.ring[slot];
-      const float* lgs = reinterpret_cast<const float*>(st + kBlockBytes);
-      const uint32_t tau = CANDS ? ld_volatile_u32(tau_lo) << (32 - kCandHistBits) : 0u;
-      if (rows == BR) {
-        // full block: every row valid, no per-row tests
+      // The whole block into registers (8 16-byte pieces per lane) and the slot straight back to
+      // the copy engine, so the arithmetic below overlaps the copy of the warp's next blocks.
+      // Rows past a partial block's end hold older data; their results are dropped below.
+      uint4 wv[Gm::NB][Gm::NI];
+      float lgv[Gm::NB];
 #pragma unroll
-        for (int bt = 0; bt < Gm::NB; ++bt) {
-          const unsigned char* sb = st + (size_t)bt * 32 * Gm::ROW_BYTES;
+      for (int bt = 0; bt < Gm::NB; ++bt) {
+#pragma unroll
+        for (int ii = 0; ii < Gm::NI; ++ii)
+          wv[bt][ii] = *reinterpret_cast<const uint4*>(st + (size_t)(bt * 32 + ii * Gm::RPI + rsub) * Gm::ROW_BYTES +
+                                                       part * 16);
+        if constexpr (GATED) lgv[bt] = reinterpret_cast<const float*>(st + kBlockBytes)[bt * 32 + part * Gm::RPI + rsub];
+      }
+      const uint32_t tau = CANDS ? ld_volatile_u32(tau_lo) << (32 - kCandHistBits) : 0u;
+      __syncwarp();  // every lane has read the slot
+      if (lane == 0 && i + kDepth < my_blocks) issue(slot);
+#pragma unroll
+      for (int bt = 0; bt < Gm::NB; ++bt) {
+        const int wrows = rows - bt * 32;  // rows of this 32-row batch (warp-uniform)
+        if (wrows > 0) {
           float v[Gm::NI];
 #pragma unroll
           for (int ii = 0; ii < Gm::NI; ++ii) {
-            const uint4 w = *reinterpret_cast<const uint4*>(sb + (size_t)(ii * Gm::RPI + rsub) * Gm::ROW_BYTES + part * 16);
-            if constexpr (KP8) v[ii] = dot16_fp8(qv, w); else v[ii] = dot8(qv, w);
+            if constexpr (KP8) v[ii] = dot16_fp8(qv, wv[bt][ii]); else v[ii] = dot8(qv, wv[bt][ii]);
           }
           const float u0 = butterfly<Gm>(v, lane);
           const int lr = part * Gm::RPI + rsub;
-          const float u = GATED ? fmaf(p.lam, lgs[bt * 32 + lr], u0) : u0;
-          take_key(u, bh, row0 + bt * 32 + lr, true, tau);
-        }
-      } else {
-#pragma unroll
-        for (int bt = 0; bt < Gm::NB; ++bt) {
-          const int wrows = rows - bt * 32;  // rows of this 32-row batch
-          if (wrows > 0) {
-            const unsigned char* sb = st + (size_t)bt * 32 * Gm::ROW_BYTES;
-            float v[Gm::NI];
-#pragma unroll
-            for (int ii = 0; ii < Gm::NI; ++ii) {
-              const int lr = ii * Gm::RPI + rsub;
-              uint4 w = make_uint4(0u, 0u, 0u, 0u);
-              if (lr < wrows) w = *reinterpret_cast<const uint4*>(sb + (size_t)lr * Gm::ROW_BYTES + part * 16);
-              if constexpr (KP8) v[ii] = dot16_fp8(qv, w); else v[ii] = dot8(qv, w);
-            }
-            const float u0 = butterfly<Gm>(v, lane);
-            const int lr = part * Gm::RPI + rsub;
-            const bool valid = lr < wrows;
-            const float u = (GATED && valid) ? fmaf(p.lam, lgs[bt * 32 + lr], u0) : u0;
-            take_key(u, bh, row0 + bt * 32 + lr, valid, tau);
-          }
+          const float u = GATED ? fmaf(p.lam, lgv[bt], u0) : u0;
+          take_key(u, bh, row0 + bt * 32 + lr, lr < wrows, tau);
         }
       }
-      __syncwarp();  // every lane is done with the slot
-      if (lane == 0 && i + kDepth < my_blocks) issue(slot);
     }
     close_record(bh);
 

@@ -557,31 +557,39 @@ __global__ void __launch_bounds__(THREADS, 1) select_topk_kernel(const SelectPar
 
 // ---------------------------------------------------------------------------------------------
 // Candidate mode.  The score kernel has left, per head, a list of records (first block and block
-// stride, even count) that point at (key, position) pairs: every key at or above a lower bound of the head's
-// k-th largest key, plus sentinels of key 0.  Since the candidates hold every key that can be
-// selected and at least k of them, the k-th largest candidate key is the head's k-th largest
-// key T.  One CTA per head: the candidates are copied into shared memory (one bulk copy per block
-// run of a record) when they fit, else every pass reads them from L2.  T is found as three radix
-// digits (11, 11 and 10 bits); when T has more ties than the budget takes, the lowest positions
-// among them are found as two 9-bit digits of the position.  The chosen positions are set in a
-// bitmap of the head and written out in ascending order.
-constexpr int kCandBins = 2048;
+// stride, even count) that point at (key, position) pairs: every key at or above a lower bound of
+// the head's k-th largest key, plus sentinels of key 0; and a histogram of the top 12 bits of those
+// keys.  The candidates hold every key that can be selected and at least k of them, so the k-th
+// largest candidate key is the head's k-th largest key T.  One CTA per head:
+//   1. digit 1 of T (12 bits) from the histogram;
+//   2. one pass over the candidates (read from L2, eight 16-byte loads in flight per thread): keys
+//      with a larger digit 1 are selected and set in a bitmap of the head's positions, keys with
+//      digit 1 equal to T's go to a list in shared memory;
+//   3. digits 2 and 3 of T (10 bits each) among the list, then, when T has more ties than the
+//      budget takes, the lowest positions among them as two 9-bit digits of the position;
+//   4. the chosen list entries into the bitmap, and the bitmap out as ascending positions.
+// If the list does not fit on chip (many keys share T's digit 1), steps 3 and 4 make their passes
+// over all candidates instead.
+constexpr int kCandBins1 = 1 << kCandHistBits;  // 4096: digit 1
+constexpr int kListCap = 8192;                  // on-chip entries of digit 1's bin
 
 struct CandCtl {
-  uint32_t hist[kCandBins];
+  uint32_t hist[1024];
   uint32_t wsum[32];
   Found found;
-  uint64_t bar;
-  uint32_t pad[2];
+  uint32_t nlist;
+  uint32_t pad[3];
 };
-static_assert(sizeof(CandCtl) % 16 == 0, "candidate array alignment");
+static_assert(sizeof(CandCtl) % 16 == 0, "shared-memory layout alignment");
 
 template <int THREADS>
 __global__ void __launch_bounds__(THREADS, 1) select_cand_kernel(const SelectParams p) {
   extern __shared__ __align__(128) unsigned char smem_raw[];
   CandCtl& S = *reinterpret_cast<CandCtl*>(smem_raw);
-  uint32_t* bm = reinterpret_cast<uint32_t*>(smem_raw + sizeof(CandCtl));
-  uint2* cs = reinterpret_cast<uint2*>(smem_raw + sizeof(CandCtl) + (size_t)p.bm_words * 4);
+  uint2* list = reinterpret_cast<uint2*>(smem_raw + sizeof(CandCtl));
+  uint2* rrec = list + kListCap;
+  uint32_t* rpre = reinterpret_cast<uint32_t*>(rrec + p.rec_cap);
+  uint32_t* bm = rpre + ((p.rec_cap + 4) & ~3);
   const int tid = threadIdx.x;
   const int bh = blockIdx.x;
   const int b = bh / p.Hkv;
@@ -603,96 +611,127 @@ __global__ void __launch_bounds__(THREADS, 1) select_cand_kernel(const SelectPar
 
   const int nwords = (n + 31) >> 5;
   for (int i = tid; i < nwords; i += THREADS) bm[i] = 0u;
-  for (int i = tid; i < kCandBins; i += THREADS) S.hist[i] = 0u;
   if (tid == 0) {
-    mbar_init(&S.bar, 1);
-    fence_barrier_init();
     S.found = Found{};
+    S.nlist = 0u;
   }
   __syncthreads();
-  // The candidates, records and record counts of the score pass are read only from here on.
+  // The candidates, records, record counts and histograms of the score pass are read only from
+  // here on.
   pdl_wait();
   pdl_trigger();
 
-  const uint32_t R = min(p.rec_cnt[bh], (uint32_t)p.rec_stride);
+  // ---- records: copied on chip, with the offsets of their entries in one flat order ----
+  uint32_t R = p.rec_cnt[bh];
+  if (R > (uint32_t)p.rec_cap) {  // cannot happen: at most 16 warps of every scanning CTA
+    if (tid == 0) record_error(p.err, kDevCandidates, (uint32_t)bh);
+    R = (uint32_t)p.rec_cap;
+  }
   const uint2* recs = p.recs + (size_t)bh * p.rec_stride;
-  const uint2* cand = p.cand + (size_t)bh * p.cand_stride;
-  const int BR = p.block_rows;
-  const int lbr = __ffs(BR) - 1;  // BR is a power of two
-  // a record is (first block | block stride << 24, even count)
-  // thread t sums the counts of records [r0, r1)
   const int rpt = (int)((R + THREADS - 1) / THREADS);
   const int r0 = min(tid * rpt, (int)R), r1 = min(r0 + rpt, (int)R);
   uint32_t mine = 0u;
-  for (int r = r0; r < r1; ++r) mine += recs[r].y;
+  for (int r = r0; r < r1; ++r) {
+    const uint2 rc = recs[r];
+    rrec[r] = rc;
+    mine += rc.y;
+  }
   uint32_t total;
-  const uint32_t off = block_excl_scan<THREADS>(mine, S.wsum, &total);
-  if (tid == 0) p.rec_cnt[bh] = 0u;  // every thread has read it: ready for the next scan
+  uint32_t off = block_excl_scan<THREADS>(mine, S.wsum, &total);
+  for (int r = r0; r < r1; ++r) {
+    rpre[r] = off;
+    off += rrec[r].y;
+  }
+  if (tid == 0) {
+    rpre[R] = total;
+    p.rec_cnt[bh] = 0u;  // every thread has read it: ready for the next scan
+  }
 
-  if ((uint32_t)k_eff > total) {
-    // Cannot happen (every key >= T is a candidate); leave a defined output and report it.
+  // ---- digit 1 from the score pass's histogram, which is then cleared for the next scan ----
+  uint32_t* gh = p.hist + (size_t)bh * kCandBins1;
+  find_digit<kCandBins1, THREADS>(gh, (uint32_t)k_eff, S.wsum, &S.found);  // ends with a barrier
+  const uint32_t d1 = S.found.digit;
+  const uint32_t eq1 = S.found.eq;
+  uint32_t k_rem = (uint32_t)k_eff - S.found.above;
+  for (int i = tid; i < kCandBins1 / 4; i += THREADS) reinterpret_cast<uint4*>(gh)[i] = make_uint4(0u, 0u, 0u, 0u);
+
+  if ((uint32_t)k_eff > total || eq1 == 0u) {
+    // Cannot happen (every key >= T is a candidate and counted); leave a defined output.
     if (tid == 0) record_error(p.err, kDevCandidates, (uint32_t)bh);
     for (int j = tid; j < p.k_max; j += THREADS) idx[j] = -1;
     return;
   }
 
-  bool waited_ok = true;
-  const bool in_smem = total <= (uint32_t)p.cand_smem;
-  if (in_smem) {
-    if (tid == 0) mbar_arrive_expect_tx(&S.bar, total * 8u);
-    __syncthreads();
-    uint32_t o = off;
-    for (int r = r0; r < r1; ++r) {
-      const uint2 rc = recs[r];
-      for (uint32_t e = 0; e < rc.y; e += (uint32_t)BR) {
-        const uint32_t cnt = min((uint32_t)BR, rc.y - e);
-        bulk_g2s(cs + o + e, cand + ((size_t)(rc.x & 0xffffffu) + (size_t)(e >> lbr) * (rc.x >> 24)) * BR, cnt * 8u,
-                 &S.bar);
-      }
-      o += rc.y;
-    }
-    if (!mbar_wait_bounded(&S.bar, 0u)) waited_ok = false;
-  }
-
-  // fn(key, position) over every candidate (sentinels included), this thread's share of them
-  auto for_each = [&](auto&& fn) {
-    if (in_smem) {
-      for (uint32_t e = tid; e < total; e += THREADS) {
-        const uint2 v = cs[e];
-        fn(v.x, v.y);
-      }
-    } else {
-      for (uint32_t r = 0; r < R; ++r) {
-        const uint2 rc = recs[r];
-        for (uint32_t e = tid; e < rc.y; e += THREADS) {
-          const uint2 v =
-              cand[((size_t)(rc.x & 0xffffffu) + (size_t)(e >> lbr) * (rc.x >> 24)) * BR + (e & (uint32_t)(BR - 1))];
-          fn(v.x, v.y);
+  const uint2* cand = p.cand + (size_t)bh * p.cand_stride;
+  const int BR = p.block_rows;
+  const int lbr = __ffs(BR) - 1;  // BR is a power of two
+  // fn(key, position) over every candidate, pairs of entries (16-byte loads; record counts and
+  // block pieces are even) taken by consecutive threads, eight loads in flight per thread
+  auto stream = [&](auto&& fn) {
+    const uint32_t pairs = total >> 1;
+    uint32_t r = 0u;
+    constexpr int U = 8;
+    for (uint32_t j0 = (uint32_t)tid; j0 < pairs; j0 += U * THREADS) {
+      uint4 v[U];
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const uint32_t j = j0 + (uint32_t)u * THREADS;
+        v[u] = make_uint4(0u, 0u, 0u, 0u);
+        if (j < pairs) {
+          const uint32_t e = 2u * j;
+          while (rpre[r + 1] <= e) ++r;  // entries only move forward
+          const uint32_t o = e - rpre[r];
+          const uint2 rc = rrec[r];
+          const size_t at = ((size_t)(rc.x & 0xffffffu) + (size_t)(o >> lbr) * (rc.x >> 24)) * BR + (o & (uint32_t)(BR - 1));
+          v[u] = __ldcg(reinterpret_cast<const uint4*>(cand + at));
         }
       }
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        fn(v[u].x, v[u].y);  // a zero pair (past the end) has key 0: below every real key
+        fn(v[u].z, v[u].w);
+      }
+    }
+  };
+  auto mark = [&](uint32_t pos) { atomicOr(&bm[pos >> 5], 1u << (pos & 31)); };
+
+  // ---- one pass: above digit 1 into the bitmap, digit 1's bin into the list ----
+  const bool listed = eq1 <= (uint32_t)kListCap;
+  stream([&](uint32_t key, uint32_t pos) {
+    const uint32_t dg = key >> (32 - kCandHistBits);
+    if (dg > d1) {
+      mark(pos);
+    } else if (dg == d1 && listed) {
+      const uint32_t slot = atomicAdd(&S.nlist, 1u);
+      if (slot < (uint32_t)kListCap) list[slot] = make_uint2(key, pos);
+    }
+  });
+  for (int i = tid; i < 1024; i += THREADS) S.hist[i] = 0u;
+  __syncthreads();
+  const uint32_t nl = min(S.nlist, (uint32_t)kListCap);
+  // fn over the keys in digit 1's bin: the list, or every candidate filtered again
+  auto over_bin = [&](auto&& fn) {
+    if (listed) {
+      for (uint32_t e = tid; e < nl; e += THREADS) fn(list[e].x, list[e].y);
+    } else {
+      stream([&](uint32_t key, uint32_t pos) {
+        if ((key >> (32 - kCandHistBits)) == d1) fn(key, pos);
+      });
     }
   };
   auto clear_hist = [&]() {
-    for (int i = tid; i < kCandBins; i += THREADS) S.hist[i] = 0u;
+    for (int i = tid; i < 1024; i += THREADS) S.hist[i] = 0u;
     __syncthreads();
   };
 
-  // ---- T as three digits of the key: 11, 11 and 10 bits ----
-  for_each([&](uint32_t key, uint32_t) { atomicAdd(&S.hist[key >> 21], 1u); });
+  // ---- digits 2 and 3 of T (10 bits each) ----
+  over_bin([&](uint32_t key, uint32_t) { atomicAdd(&S.hist[(key >> 10) & 1023u], 1u); });
   __syncthreads();
-  find_digit<kCandBins, THREADS>(S.hist, (uint32_t)k_eff, S.wsum, &S.found);
-  const uint32_t d1 = S.found.digit;
-  uint32_t k_rem = (uint32_t)k_eff - S.found.above;
-  clear_hist();
-  for_each([&](uint32_t key, uint32_t) {
-    if ((key >> 21) == d1) atomicAdd(&S.hist[(key >> 10) & (kCandBins - 1)], 1u);
-  });
-  __syncthreads();
-  find_digit<kCandBins, THREADS>(S.hist, k_rem, S.wsum, &S.found);
-  const uint32_t pre = (d1 << 11) | S.found.digit;
+  find_digit<1024, THREADS>(S.hist, k_rem, S.wsum, &S.found);
+  const uint32_t pre = (d1 << 10) | S.found.digit;
   k_rem -= S.found.above;
   clear_hist();
-  for_each([&](uint32_t key, uint32_t) {
+  over_bin([&](uint32_t key, uint32_t) {
     if ((key >> 10) == pre) atomicAdd(&S.hist[key & 1023u], 1u);
   });
   __syncthreads();
@@ -705,7 +744,7 @@ __global__ void __launch_bounds__(THREADS, 1) select_cand_kernel(const SelectPar
   uint32_t cut = 0xffffffffu;
   if (need < eq) {
     clear_hist();
-    for_each([&](uint32_t key, uint32_t pos) {
+    over_bin([&](uint32_t key, uint32_t pos) {
       if (key == T) atomicAdd(&S.hist[511u - (pos >> 9)], 1u);
     });
     __syncthreads();
@@ -713,7 +752,7 @@ __global__ void __launch_bounds__(THREADS, 1) select_cand_kernel(const SelectPar
     const uint32_t ph = 511u - S.found.digit;
     const uint32_t need2 = need - S.found.above;
     clear_hist();
-    for_each([&](uint32_t key, uint32_t pos) {
+    over_bin([&](uint32_t key, uint32_t pos) {
       if (key == T && (pos >> 9) == ph) atomicAdd(&S.hist[511u - (pos & 511u)], 1u);
     });
     __syncthreads();
@@ -721,9 +760,9 @@ __global__ void __launch_bounds__(THREADS, 1) select_cand_kernel(const SelectPar
     cut = (ph << 9) | (511u - S.found.digit);
   }
 
-  // ---- the chosen positions into the bitmap ----
-  for_each([&](uint32_t key, uint32_t pos) {
-    if (key > T || (key == T && pos <= cut)) atomicOr(&bm[pos >> 5], 1u << (pos & 31));
+  // ---- the chosen keys of digit 1's bin into the bitmap ----
+  over_bin([&](uint32_t key, uint32_t pos) {
+    if (key > T || (key == T && pos <= cut)) mark(pos);
   });
   __syncthreads();
 
@@ -746,24 +785,23 @@ __global__ void __launch_bounds__(THREADS, 1) select_cand_kernel(const SelectPar
     }
   }
   for (int j = k_eff + tid; j < p.k_max; j += THREADS) idx[j] = -1;
-  if (!waited_ok) record_error(p.err, kDevWaitTimeout, (uint32_t)bh);
 }
 
 }  // namespace
 
 bool plan_select(SelectParams& p, int num_sms) {
   if (p.cands) {
-    // one CTA per head; the candidates of a whole head in shared memory when they fit
+    // one CTA per head: the on-chip list of digit 1's bin, the head's records and its bitmap
     p.cluster = 1;
     p.threads = 1024;
     p.chunk = p.cap;
-    p.bm_words = (((p.cap + 31) / 32) + 3) & ~3;
-    const long long fixed = (long long)sizeof(CandCtl) + (long long)p.bm_words * 4;
-    long long want = fixed + (long long)p.cand_stride * 8;
-    if (want > kSmemLimitSel) want = kSmemLimitSel;
-    if (want < fixed + 16) return false;
-    p.smem_bytes = (int)want;
-    p.cand_smem = (int)((want - fixed) / 8);
+    p.rec_cap = 16 * (num_sms > 0 ? num_sms : 148);  // records per head: 16 warps of every scanning CTA
+    if (p.rec_cap > p.rec_stride) p.rec_cap = p.rec_stride;
+    p.bm_words = (p.cap + 31) / 32;
+    const long long bytes = (long long)sizeof(CandCtl) + (long long)kListCap * 8 + (long long)p.rec_cap * 8 +
+                            (long long)((p.rec_cap + 4) & ~3) * 4 + (long long)p.bm_words * 4;
+    if (bytes > kSmemLimitSel) return false;
+    p.smem_bytes = (int)bytes;
     return true;
   }
   const int heads = p.B * p.Hkv;
