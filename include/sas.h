@@ -110,17 +110,6 @@ const char* sas_last_error_detail(void);
 size_t sas_decode_workspace_bytes(const sas_shape* shape, int32_t k_max);
 size_t sas_dense_workspace_bytes(const sas_shape* shape);
 
-/* Which form the selection takes for a shape and budget bound on the current device (host-only,
- * no GPU work; the device's SM count is read when a device is present, else 148 is assumed):
- *   0  keys: the score scan writes the key of every cached token and the selection streams them
- *      (few heads, or short per-SM scan segments against k_max);
- *   1  candidates: the score scan keeps, per KV head, only the keys at or above a running lower
- *      bound of the head's k-th largest key (a few k pairs of key and position instead of N keys)
- *      and the selection ranks those (many heads: per-SM segments of at least 8 * k_max rows);
- *  -1  invalid shape or k_max < 1.
- * Both forms select the same positions; the workspace size covers either. */
-int sas_selection_mode(const sas_shape* shape, int32_t k_max);
-
 /* Zero a workspace.  Must be called once after the workspace is allocated (or any time
  * after a call was abandoned); the kernels leave it ready for the next call themselves.
  * Enqueued on `stream`. */

@@ -138,13 +138,7 @@ def test_append_matches_build(cuda_lib):
         assert torch.equal(kp_app, kp_build)
 
 
-# ------------------------------------------------- candidate mode (many heads, long segments)
-def _mode(p):
-    from token_level_sparse_head_b200 import lib, shape_of
-
-    return lib.sas_selection_mode(shape_of(p), p.k_max)
-
-
+# ------------------------------------------------------- many heads with ragged lengths
 def _many_heads_problem(paged, lam, seed, fp8=False):
     # 128 KV heads with ragged lengths, an empty sequence, N = 1, k >= N and k = 0 among them
     rng = np.random.default_rng(seed)
@@ -159,27 +153,22 @@ def _many_heads_problem(paged, lam, seed, fp8=False):
 
 @pytest.mark.parametrize("paged", [False, True])
 @pytest.mark.parametrize("lam", [0.0, 1.0])
-def test_candidate_mode_many_heads(cuda_lib, paged, lam):
-    # long per-SM scan segments against the budget: the scan keeps only per-head candidates
+def test_many_heads(cuda_lib, paged, lam):
+    # 128 heads: one CTA of the selection per head, scan shares spanning head boundaries
     p = _many_heads_problem(paged, lam, seed=41)
-    assert _mode(p) == 1
     run_small(p, dense=False, check_build=False)
 
 
-def test_candidate_mode_fp8(cuda_lib):
+def test_many_heads_fp8(cuda_lib):
     p = _many_heads_problem(False, 1.0, seed=42, fp8=True)
-    assert _mode(p) == 1
     run_small(p, dense=False, check_build=False)
 
 
-def test_candidate_mode_ties_and_rising_scores(cuda_lib):
-    # sequence 0: every key equal, so every row is a candidate and the ties are cut by position;
-    # sequence 1: scores rising with position (in bf16 steps, so with plateaus of ties), so the
-    # running threshold never drops a row.  Both heads hold more candidates than shared memory,
-    # which sends the selection down the path that reads them from L2 in every pass.
+def test_ties_and_rising_scores(cuda_lib):
+    # sequence 0: every key equal, so the ties are cut by position; sequence 1: scores rising with
+    # position in bf16 steps (plateaus of ties), the order a recency-biased head would show
     N = 40000
     p = make_problem(B=2, Hq=2, Hkv=1, d=64, r=16, seqlens=[N, N], k=[64, 64], basis="eye", seed=43)
-    assert _mode(p) == 1
     p.K[0, 0, :, :16] = 0.5
     p.K[1, 0, :, :16] = 0.0
     p.K[1, 0, :, 0] = torch.linspace(0.0, 4.0, N).to(torch.bfloat16)

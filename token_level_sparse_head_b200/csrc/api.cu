@@ -142,53 +142,30 @@ sas::AttendParams attend_plan(const sas_shape* s, int count_max, bool dense) {
   return a;
 }
 
-// Workspace: [0,256) error word | key histograms | record counts | split counters | attention
-// partials | score keys or candidates | candidate records.  The histograms, record counts and
-// counters sit at fixed offsets before the partials: they must stay zero between calls (the
+// Workspace: [0,256) error word | key histograms | split counters | attention partials | score keys.
+// The histograms and counters sit at fixed offsets: they must stay zero between calls (the
 // kernels clear them after use), whatever other calls (dense decode, other budgets) share the
-// workspace; everything from the partials on is rewritten by every call before it is read.
+// workspace; partials and keys are rewritten by every call.
 struct WsLayout {
-  size_t hist, rec_cnt, counters, partials, keys, recs, total;
+  size_t hist, counters, partials, keys, total;
 };
 
-// Candidate slots per head: the capacity rounded up to whole 256-row blocks (the largest block
-// of the score kernel), so every block's slot range lies inside its head's region.
-size_t cand_stride_of(int cap) { return ((size_t)cap + 255) & ~(size_t)255; }
-// Candidate records per head at most: one per block of the smallest block size (32 rows).
-size_t rec_stride_of(int cap) { return ((size_t)cap + 31) / 32; }
-
 WsLayout ws_layout(const sas::AttendParams& a, bool with_keys) {
-  const size_t heads = (size_t)a.B * a.Hkv;
   WsLayout w;
   size_t o = kErrBytes;
   w.hist = o;
-  o += heads * sas::kHistBins * 4;
-  w.rec_cnt = o;
-  o += (heads * 4 + 255) & ~(size_t)255;
+  o += (size_t)a.B * a.Hkv * sas::kHistBins * 4;
   w.counters = o;
   o += ((size_t)a.B * a.Hkv * a.ngz * 4 + 255) & ~(size_t)255;
   w.partials = o;
   o += (sas::attend_workspace_floats(a) * 4 + 255) & ~(size_t)255;
   w.keys = o;
-  w.recs = o;
-  if (with_keys) {
-    // keys mode uses 4 bytes per position, candidate mode 8 per candidate slot
-    o += (heads * cand_stride_of(a.cap) * 8 + 255) & ~(size_t)255;
-    w.recs = o;
-    o += (heads * rec_stride_of(a.cap) * 8 + 255) & ~(size_t)255;
-  }
+  if (with_keys) o += ((size_t)a.B * a.Hkv * a.cap * 4 + 255) & ~(size_t)255;
   w.total = o;
   return w;
 }
 
 size_t ws_bytes_for(const sas::AttendParams& a, bool with_keys) { return ws_layout(a, with_keys).total; }
-
-// Candidate mode pays when the score kernel's per-CTA segments are long against the budget: a
-// CTA then drops all but a few k keys of every head it scans.  Short segments keep every key.
-bool use_candidates(const sas_shape* s, int k_max, int sms) {
-  const long long rows = (long long)s->B * s->Hkv * cap_of(s);
-  return rows >= 8LL * k_max * sms;
-}
 
 void bind_workspace(sas::AttendParams& a, void* ws) {
   unsigned char* w = static_cast<unsigned char*>(ws);
@@ -239,12 +216,6 @@ sas_status plan_selection(const sas_shape* s, const void* q, const float* M, con
   sp.k_max = k_max;
   sp.sigma = 1.0f / sqrtf((float)s->d);
   sp.lam = lambda;
-  sp.cands = use_candidates(s, k_max, sms) ? 1 : 0;
-  sp.cand = reinterpret_cast<uint2*>(w + L.keys);
-  sp.recs = reinterpret_cast<uint2*>(w + L.recs);
-  sp.rec_cnt = reinterpret_cast<uint32_t*>(w + L.rec_cnt);
-  sp.cand_stride = (int)cand_stride_of(sp.cap);
-  sp.rec_stride = (int)rec_stride_of(sp.cap);
   sas::plan_score(sp, sms);
 
   sas::SelectParams& sl = out->sl;
@@ -256,13 +227,6 @@ sas_status plan_selection(const sas_shape* s, const void* q, const float* M, con
   sl.idx_out = idx_out;
   sl.err = sp.err;
   sl.B = s->B; sl.Hkv = s->Hkv; sl.cap = sp.cap; sl.k_max = k_max;
-  sl.cands = sp.cands;
-  sl.cand = sp.cand;
-  sl.recs = sp.recs;
-  sl.rec_cnt = sp.rec_cnt;
-  sl.cand_stride = sp.cand_stride;
-  sl.rec_stride = sp.rec_stride;
-  sl.block_rows = sp.block_rows;
   if (!sas::plan_select(sl, sms)) return fail(SAS_ERR_UNSUPPORTED, "no selection plan for this shape");
   return SAS_OK;
 }
@@ -333,11 +297,6 @@ const char* sas_last_error_detail(void) { return g_detail; }
 size_t sas_decode_workspace_bytes(const sas_shape* shape, int32_t k_max) {
   if (check_shape(shape) != SAS_OK || k_max < 1) return 0;
   return ws_bytes_for(attend_plan(shape, k_max, false), true);
-}
-
-int sas_selection_mode(const sas_shape* shape, int32_t k_max) {
-  if (check_shape(shape) != SAS_OK || k_max < 1) return -1;
-  return use_candidates(shape, k_max, num_sms()) ? 1 : 0;
 }
 
 size_t sas_dense_workspace_bytes(const sas_shape* shape) {

@@ -20,7 +20,6 @@ enum DeviceError : uint32_t {
   kDevBadIndex = 3,      // an index list entry outside [0, N_b)
   kDevKOverMax = 4,      // k[b] > k_max (clamped to k_max)
   kDevWaitTimeout = 5,   // a bounded mbarrier wait ran out
-  kDevCandidates = 6,    // fewer candidates than the budget, or too many records (not expected)
 };
 
 __device__ __forceinline__ void record_error(uint32_t* err, uint32_t code, uint32_t where) {

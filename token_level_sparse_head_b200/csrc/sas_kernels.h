@@ -14,8 +14,6 @@ constexpr int kHistShift = 19;
 constexpr int kHistBins = 1 << (32 - kHistShift);  // 8192
 constexpr int kDigit2Bits = 10;
 constexpr int kDigit3Bits = 9;
-// Candidate mode: the score kernel's running threshold is kept as a bin of the keys' top 12 bits.
-constexpr int kCandHistBits = 12;
 
 // ---------------------------------------------------------------------------- projection
 struct ProjParams {
@@ -46,23 +44,12 @@ struct ScoreParams {
   const int32_t* kvec;         // [B]
   const float* log_g;          // [B][Hkv][cap] or null
   uint32_t* keys;              // workspace: [B][Hkv][cap] order-preserving keys of u_i
-  uint32_t* hist;              // workspace, zero on entry: keys mode [B*Hkv][kHistBins] counts of the keys'
-                               // top 13 bits; candidate mode [B*Hkv][4096] counts of the candidates' top 12
+  uint32_t* hist;              // workspace: [B][Hkv][kHistBins] counts of the keys' first digit (zero on entry)
   float* scores_out;           // [B][Hkv][cap] or null
   uint32_t* err;
   int B, Hq, Hkv, G, d, r, cap, max_pages, num_pages, paged, k_max;
   float sigma, lam;
   int ctas;                    // persistent grid size
-  // candidate mode (cands = 1): (key, position) pairs at or above the running threshold instead
-  // of every key; each consumer warp stores its candidates of a head in the slot ranges of its
-  // own blocks of that head and appends a record (first block | warps << 24, even count) to the
-  // head's list
-  int cands;
-  uint2* cand;                 // workspace: [B*Hkv][cand_stride]
-  uint2* recs;                 // workspace: [B*Hkv][rec_stride]
-  uint32_t* rec_cnt;           // workspace: [B*Hkv] records per head (zero on entry)
-  int cand_stride, rec_stride;
-  int block_rows;              // set by plan_score: projected rows per block
 };
 void plan_score(ScoreParams& p, int num_sms);
 cudaError_t launch_score(const ScoreParams& p, cudaStream_t stream);
@@ -81,17 +68,8 @@ struct SelectParams {
   int chunk;                   // max positions per CTA (multiple of 512)
   int cand_cap;                // candidate list capacity per CTA
   int off_hist, off_ctl, smem_bytes;
-  // candidate mode (see ScoreParams)
-  int cands;
-  const uint2* cand;
-  const uint2* recs;
-  uint32_t* rec_cnt;           // cleared here after use
-  int cand_stride, rec_stride, block_rows;
-  int bm_words;                // bitmap words in shared memory
-  int rec_cap;                 // records per head held in shared memory (>= 16 * scan CTAs)
 };
-// Chooses cluster size and chunk (keys mode) or the shared-memory split (candidate mode) for a
-// shape; returns false if unsupported.
+// Chooses cluster size and chunk for a shape; returns false if unsupported.
 bool plan_select(SelectParams& p, int num_sms);
 cudaError_t launch_select(const SelectParams& p, cudaStream_t stream);
 

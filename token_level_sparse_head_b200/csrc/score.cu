@@ -4,20 +4,9 @@
 // s-hat_i = q-bar^T M^T (M k_i) = q-hat . Kproj_i, with q-bar the mean of the G query heads of
 // h; section Triton 内核的三个设计点: scoring is not sparse, it scans every candidate.  The gate
 // of the SAS page (section 2.1) adds lambda * log g_i.  Each score is turned into the
-// order-preserving uint32 key of u_i = sigma * s-hat_i (+ lambda log g_i) for the selection that
-// follows, in one of two forms chosen per launch:
-//
-//   keys mode        every key is written to the workspace (L2 evict-last hint) and a histogram
-//                    of the keys' top 13 bits is accumulated per (b, h);
-//   candidate mode   only keys at or above a running lower bound tau of the head's k-th largest
-//                    key are written, as (key, position) pairs.  Every written key is also counted
-//                    in a per-head histogram of its top 12 bits in global memory, shared by all
-//                    CTAs that scan the head.  The k-th largest of the keys counted so far can
-//                    only be at or below the k-th largest of the whole head, so a key below tau
-//                    can never be selected and is dropped.  A threshold warp per CTA keeps tau at
-//                    the bin of that k-th largest counted key, reading the shared histogram; with
-//                    many heads this writes a few k keys per head instead of N, and the selection
-//                    takes its first digit from the histogram.
+// order-preserving uint32 key of u_i = sigma * s-hat_i (+ lambda log g_i), written to the
+// workspace with an L2 evict-last hint for the selection that follows, and a histogram of the
+// keys' top 13 bits is accumulated per (b, h).
 //
 // Persistent kernel, one CTA per SM.  The work is the list of 4 KB blocks of projected rows
 // (64 rows at r = 32 in bf16) of every (b, h) that needs scores, in (b, h, position) order; each
@@ -28,13 +17,7 @@
 // compute, so a slot is out of flight only for the few shared-memory loads that empty it and no
 // warp waits on another.  Per 32-row batch the lanes form 16-byte dot products with q-hat and
 // meet in a transposing butterfly.
-//
-// Candidate storage: a warp writes the candidates of its blocks of one head, in order, into the
-// 64-row slot ranges of those same blocks (the n-th candidate into the (n / BR)-th of its blocks,
-// at offset n % BR); the count never outruns the rows scanned, so no space is shared.  At the end
-// of its part of a head the warp pads the count to even with a sentinel (key 0, which no score
-// maps to, never selected) and appends a record (first block | warps << 24, count) to the head's
-// record list; the warp count is the block stride of the record.
+
 #include <cuda_fp16.h>
 #include <cuda_fp8.h>
 
@@ -48,9 +31,7 @@ constexpr int kBlockBytes = 4096;   // projected bytes per block (one ring stage
 constexpr int kDepth = 2;           // ring slots per consumer warp
 constexpr int kMaxWarps = 16;       // consumer warps per CTA at most
 constexpr int kSmemLimit = 227 * 1024;
-constexpr int kSmemMisc = 2048;     // q-bar, q-hat, barriers, plan and threshold state (upper bound)
-constexpr uint32_t kTauDone = 0xffffffffu;  // generation that tells the threshold warp to stop
-constexpr uint32_t kTauPasses = 1u << 20;   // threshold passes at most (each ends in a short sleep)
+constexpr int kSmemMisc = 2048;     // q-bar, q-hat, barriers and plan (upper bound)
 
 // Row geometry of the projected cache: bf16 (KP8 = false) or FP8 E4M3 codes (KP8 = true).
 template <int R, bool KP8>
@@ -66,17 +47,17 @@ struct Geo {
 };
 
 // Block shape of one instantiation: as many consumer warps (two slots each) as shared memory
-// holds next to the histogram, at most 16; candidate mode adds the threshold warp.
-template <int R, bool GATED, bool KP8, bool CANDS>
+// holds next to the histogram, at most 16.
+template <int R, bool GATED, bool KP8>
 struct Cfg {
   using Gm = Geo<R, KP8>;
-  static constexpr int kBins = CANDS ? 4 : kHistBins;  // candidate mode counts in global memory
+  static constexpr int kBins = kHistBins;
   static constexpr int kSlotBytes = kBlockBytes + (GATED ? Gm::BLOCK_ROWS * 4 : 0);
   static constexpr int kMaxSlots = (kSmemLimit - kSmemMisc - kBins * 4) / kSlotBytes;
   static constexpr int kWarps = kMaxSlots / kDepth >= kMaxWarps ? kMaxWarps : kMaxSlots / kDepth;
   static constexpr int kSlots = kWarps * kDepth;
   static constexpr int kConsumers = kWarps * 32;
-  static constexpr int kThreads = kConsumers + (CANDS ? 32 : 0);
+  static constexpr int kThreads = kConsumers;
 };
 
 // Position of a CTA's share in the block list, computed once by warp 0.
@@ -86,61 +67,30 @@ struct Plan {
   int h0, c0; // KV head and block index within it
 };
 
-template <int R, int D, bool GATED, bool KP8, bool CANDS>
+template <int R, int D, bool GATED, bool KP8>
 struct Smem {
-  using C = Cfg<R, GATED, KP8, CANDS>;
+  using C = Cfg<R, GATED, KP8>;
   unsigned char ring[C::kSlots][C::kSlotBytes];
   uint32_t hist[C::kBins];
   float qbar[D];
   float qhat[R];
   uint64_t full[C::kSlots];
-  unsigned long long tau_state;  // candidate mode: (generation << 32) | threshold bin
-  int head_k;                    // candidate mode: k_eff of the head being scanned (0: none)
-  int head_bh;                   // candidate mode: that head's (b * Hkv + h)
   Plan plan;
 };
 
-template <int R, int D, bool GATED, bool KP8, bool CANDS>
+template <int R, int D, bool GATED, bool KP8>
 constexpr bool smem_fits() {
-  return sizeof(Smem<R, D, GATED, KP8, CANDS>) <= (size_t)kSmemLimit;
+  return sizeof(Smem<R, D, GATED, KP8>) <= (size_t)kSmemLimit;
 }
-static_assert(smem_fits<16, 128, true, true, true>() && smem_fits<16, 128, true, true, false>() &&
-                  smem_fits<32, 128, true, true, true>() && smem_fits<32, 128, true, true, false>() &&
-                  smem_fits<64, 128, true, true, true>() && smem_fits<64, 128, true, true, false>() &&
-                  smem_fits<16, 128, true, false, true>() && smem_fits<16, 128, true, false, false>() &&
-                  smem_fits<32, 128, true, false, true>() && smem_fits<32, 128, true, false, false>() &&
-                  smem_fits<64, 128, true, false, true>() && smem_fits<64, 128, true, false, false>() &&
-                  smem_fits<32, 128, false, false, false>() && smem_fits<32, 128, false, false, true>(),
+static_assert(smem_fits<16, 128, true, true>() && smem_fits<32, 128, true, true>() && smem_fits<64, 128, true, true>() &&
+                  smem_fits<16, 128, true, false>() && smem_fits<32, 128, true, false>() &&
+                  smem_fits<64, 128, true, false>() && smem_fits<32, 128, false, false>(),
               "score kernel shared memory");
 
 __device__ __forceinline__ void stg_hint(uint32_t* ptr, uint32_t v, uint64_t pol) {
   asm volatile("st.global.L2::cache_hint.u32 [%0], %1, %2;" ::"l"(ptr), "r"(v), "l"(pol) : "memory");
 }
-__device__ __forceinline__ void stg_hint_v2(uint2* ptr, uint32_t a, uint32_t b, uint64_t pol) {
-  asm volatile("st.global.L2::cache_hint.v2.u32 [%0], {%1, %2}, %3;" ::"l"(ptr), "r"(a), "r"(b), "l"(pol) : "memory");
-}
-__device__ __forceinline__ void red_add(uint32_t* p) {
-  asm volatile("red.relaxed.gpu.global.add.u32 [%0], 1;" ::"l"(p) : "memory");
-}
-__device__ __forceinline__ uint32_t ld_volatile_u32(const uint32_t* p) {
-  uint32_t v;
-  asm volatile("ld.volatile.shared.u32 %0, [%1];" : "=r"(v) : "r"(smem_u32(p)) : "memory");
-  return v;
-}
-__device__ __forceinline__ unsigned long long ld_volatile_u64(const unsigned long long* p) {
-  unsigned long long v;
-  asm volatile("ld.volatile.shared.u64 %0, [%1];" : "=l"(v) : "r"(smem_u32(p)) : "memory");
-  return v;
-}
-__device__ __forceinline__ uint4 ld_volatile_v4(const uint32_t* p) {
-  uint4 v;
-  asm volatile("ld.volatile.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-               : "r"(smem_u32(p))
-               : "memory");
-  return v;
-}
-// Barrier 1 among the consumer warps only (the threshold warp never joins it).
+// Barrier 1 among the consumer warps.
 template <int N>
 __device__ __forceinline__ void consumers_sync() {
   asm volatile("bar.sync 1, %0;" ::"n"(N) : "memory");
@@ -224,80 +174,20 @@ __device__ __forceinline__ void next_scored_seq(const ScoreParams& p, int& b, Se
   while (b < p.B && (si = seq_info<BR>(p, b, false)).blocks == 0) ++b;
 }
 
-// Candidate mode: keeps the CTA's threshold at the bin of the k-th largest key counted so far for
-// the head being scanned, over every CTA that scans it (the global histogram).  Counts read while
-// other warps still add to them are at most the true counts, so the bin found is never above the
-// true one; a pass that straddles a change of head (the generation moved on) is discarded by the
-// compare-and-swap.
-__device__ void threshold_warp(const uint32_t* ghist, unsigned long long* state, const int* head_k,
-                               const int* head_bh, int lane) {
-  constexpr int BINS = 1 << kCandHistBits;
-  constexpr int PER = BINS / 32;  // bins per lane, lane 0 holding the top ones
-  for (uint32_t it = 0; it < kTauPasses; ++it) {
-    const unsigned long long st = ld_volatile_u64(state);
-    const uint32_t gen = (uint32_t)(st >> 32);
-    if (gen == kTauDone) return;
-    const uint32_t cur = (uint32_t)st;
-    __threadfence_block();
-    const int kk = (int)ld_volatile_u32(reinterpret_cast<const uint32_t*>(head_k));
-    const int bh = (int)ld_volatile_u32(reinterpret_cast<const uint32_t*>(head_bh));
-    if (kk > 0) {
-      const uint32_t* H = ghist + (size_t)bh * BINS;
-      const int lo = BINS - (lane + 1) * PER;
-      uint32_t s = 0u;
-      if (lo + PER > (int)cur) {
-#pragma unroll 8
-        for (int i = 0; i < PER; i += 4) {
-          const uint4 v = __ldcg(reinterpret_cast<const uint4*>(H + lo + i));
-          const int bin = lo + i;
-          s += (bin + 0 >= (int)cur ? v.x : 0u) + (bin + 1 >= (int)cur ? v.y : 0u) +
-               (bin + 2 >= (int)cur ? v.z : 0u) + (bin + 3 >= (int)cur ? v.w : 0u);
-        }
-      }
-      uint32_t incl = s;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += y;
-      }
-      const uint32_t hit = __ballot_sync(0xffffffffu, incl >= (uint32_t)kk);
-      if (hit != 0u && lane == __ffs(hit) - 1) {
-        uint32_t acc = incl - s;  // counted keys in the bins above this lane's
-        int found = -1;
-        for (int bin = lo + PER - 1; bin >= lo && bin >= (int)cur; --bin) {
-          acc += __ldcg(H + bin);
-          if (acc >= (uint32_t)kk) {
-            found = bin;
-            break;
-          }
-        }
-        if (found > (int)cur)
-          atomicCAS(state, st, ((unsigned long long)gen << 32) | (unsigned long long)(uint32_t)found);
-      }
-    }
-    __syncwarp();
-    __nanosleep(128);
-  }
-}
-
-template <int R, int D, bool GATED, bool KP8, bool CANDS>
-__global__ void __launch_bounds__(Cfg<R, GATED, KP8, CANDS>::kThreads, 1) score_kernel(const ScoreParams p) {
-  using C = Cfg<R, GATED, KP8, CANDS>;
+template <int R, int D, bool GATED, bool KP8>
+__global__ void __launch_bounds__(Cfg<R, GATED, KP8>::kThreads, 1) score_kernel(const ScoreParams p) {
+  using C = Cfg<R, GATED, KP8>;
   using Gm = Geo<R, KP8>;
   constexpr int BR = Gm::BLOCK_ROWS;
   constexpr int NW = C::kWarps;
   constexpr int kConsumers = C::kConsumers;
-  constexpr int kBinShift = CANDS ? 32 - kCandHistBits : kHistShift;
   extern __shared__ __align__(128) unsigned char smem_raw[];
-  Smem<R, D, GATED, KP8, CANDS>& S = *reinterpret_cast<Smem<R, D, GATED, KP8, CANDS>*>(smem_raw);
+  Smem<R, D, GATED, KP8>& S = *reinterpret_cast<Smem<R, D, GATED, KP8>*>(smem_raw);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 
   if (tid == 0) {
     for (int s = 0; s < C::kSlots; ++s) mbar_init(&S.full[s], 1);
     fence_barrier_init();
-    S.tau_state = 0ull;
-    S.head_k = 0;
-    S.head_bh = 0;
   }
   for (int i = tid; i < C::kBins; i += C::kThreads) S.hist[i] = 0u;
 
@@ -356,20 +246,12 @@ __global__ void __launch_bounds__(Cfg<R, GATED, KP8, CANDS>::kThreads, 1) score_
     }
   }
   __syncthreads();
-  // The projected cache (appended to by the previous kernel), the keys or candidates, the
-  // histograms, the record lists and the error word are touched only from here on.
+  // The projected cache (appended to by the previous kernel), the keys, the histograms and the
+  // error word are touched only from here on.
   pdl_wait();
   pdl_trigger();
   const Plan pl = S.plan;
 
-  if constexpr (CANDS) {
-    if (warp == NW) {
-      threshold_warp(p.hist, &S.tau_state, &S.head_k, &S.head_bh, lane);
-      return;
-    }
-  }
-
-  // ------------------------------------------------------------------ consumer warps
   bool waited_ok = true;
   const unsigned char* kp = reinterpret_cast<const unsigned char*>(p.kproj);
   const int my_blocks = pl.count > warp ? (pl.count - warp + NW - 1) / NW : 0;
@@ -435,56 +317,15 @@ __global__ void __launch_bounds__(Cfg<R, GATED, KP8, CANDS>::kThreads, 1) score_
   float2 qv[Gm::CPL / 2];
   int cur_bh = -1;
   bool cur_ranked = false;
-  // candidate mode: this warp's candidates of the current head and its first block there
-  uint32_t m_cand = 0u;
-  int c_first = 0;
-  const uint32_t* tau_lo = reinterpret_cast<const uint32_t*>(&S.tau_state);  // low word: the bin
-
-  // Candidate mode: pad the warp's count of head `bh` to even and append its record.
-  auto close_record = [&](int bh) {
-    if constexpr (CANDS) {
-      if (m_cand > 0u) {
-        if (lane == 0) {
-          if (m_cand & 1u) {
-            uint2* dst = p.cand + (size_t)bh * p.cand_stride + (size_t)(c_first + (int)(m_cand / BR) * NW) * BR +
-                         m_cand % BR;
-            stg_hint_v2(dst, 0u, 0xffffffffu, pol_keep);
-          }
-          const uint32_t r = atomicAdd(&p.rec_cnt[bh], 1u);
-          if (r < (uint32_t)p.rec_stride)
-            p.recs[(size_t)bh * p.rec_stride + r] =
-                make_uint2((uint32_t)c_first | ((uint32_t)NW << 24), (m_cand + 1u) & ~1u);
-          else
-            record_error(p.err, kDevCandidates, (uint32_t)bh);
-        }
-        m_cand = 0u;
-      }
+  // The key of this lane's row of a 32-row batch (valid: the row is < N_b) into the keys buffer
+  // and the histogram (and the fp32 score into scores_out when asked for).
+  auto take_key = [&](float u, int bh, int pos, bool valid) {
+    if (valid) {
+      const uint32_t key = float_key(u);
+      stg_hint(p.keys + (size_t)bh * p.cap + pos, key, pol_keep);
+      if (cur_ranked) atomicAdd(&S.hist[key >> kHistShift], 1u);
+      if (p.scores_out != nullptr) p.scores_out[(size_t)bh * p.cap + pos] = u;
     }
-  };
-
-  // Scores of one 32-row batch: this lane's row is lr (< wrows are valid); the key goes to the
-  // keys buffer (keys mode) or, when at or above tau, to the warp's candidates.
-  auto take_key = [&](float u, int bh, int pos, bool valid, uint32_t tau) {
-    const uint32_t key = float_key(u);
-    if constexpr (!CANDS) {
-      if (valid) {
-        stg_hint(p.keys + (size_t)bh * p.cap + pos, key, pol_keep);
-        if (cur_ranked) atomicAdd(&S.hist[key >> kBinShift], 1u);
-      }
-    } else {
-      if (cur_ranked) {
-        const bool em = valid && key >= tau;
-        const uint32_t ball = __ballot_sync(0xffffffffu, em);
-        if (em) {
-          const uint32_t mm = m_cand + (uint32_t)__popc(ball & ((1u << lane) - 1u));
-          uint2* dst = p.cand + (size_t)bh * p.cand_stride + (size_t)(c_first + (int)(mm / BR) * NW) * BR + mm % BR;
-          stg_hint_v2(dst, key, (uint32_t)pos, pol_keep);
-          red_add(p.hist + (size_t)bh * (1 << kCandHistBits) + (key >> kBinShift));
-        }
-        m_cand += (uint32_t)__popc(ball);
-      }
-    }
-    if (valid && p.scores_out != nullptr) p.scores_out[(size_t)bh * p.cap + pos] = u;
   };
 
   int b = pl.b0, h = pl.h0, c = pl.c0;
@@ -506,14 +347,13 @@ __global__ void __launch_bounds__(Cfg<R, GATED, KP8, CANDS>::kThreads, 1) score_
       for (int i = 0; i < CH; ++i) mreg[i] = Mrow[i];
       consumers_sync<kConsumers>();  // every warp is done with the previous head's rows
       if (cur_bh >= 0) {
-        if constexpr (!CANDS) {
-          uint32_t* gh = p.hist + (size_t)cur_bh * kHistBins;
-          for (int i = tid; i < C::kBins; i += kConsumers) {
-            const uint32_t v = S.hist[i];
-            if (v) {
-              if (cur_ranked) atomicAdd(&gh[i], v);
-              S.hist[i] = 0u;
-            }
+        // the previous head's counts into its global histogram, then a clear histogram
+        uint32_t* gh = p.hist + (size_t)cur_bh * C::kBins;
+        for (int i = tid; i < C::kBins; i += kConsumers) {
+          const uint32_t v = S.hist[i];
+          if (v) {
+            if (cur_ranked) atomicAdd(&gh[i], v);
+            S.hist[i] = 0u;
           }
         }
       }
@@ -531,16 +371,6 @@ __global__ void __launch_bounds__(Cfg<R, GATED, KP8, CANDS>::kThreads, 1) score_
       for (int o = TPR / 2; o; o >>= 1) sp += __shfl_xor_sync(0xffffffffu, sp, o);
       // FP8: the head's scale multiplies q-hat, so the codes are used as they are
       if (qpart == 0 && qrow) S.qhat[qj] = sp * p.sigma * (KP8 ? p.kproj_scale[h] : 1.f);
-      if constexpr (CANDS) {
-        if (tid == 0) {
-          // a new generation restarts the threshold for the new head
-          *reinterpret_cast<volatile int*>(&S.head_k) = si.ranked ? si.k_eff : 0;
-          *reinterpret_cast<volatile int*>(&S.head_bh) = bh;
-          __threadfence_block();
-          const unsigned long long st = ld_volatile_u64(&S.tau_state);
-          atomicExch(&S.tau_state, ((st >> 32) + 1ull) << 32);
-        }
-      }
       consumers_sync<kConsumers>();
 #pragma unroll
       for (int e = 0; e < Gm::CPL / 2; ++e)
@@ -551,7 +381,6 @@ __global__ void __launch_bounds__(Cfg<R, GATED, KP8, CANDS>::kThreads, 1) score_
 
     // ---- this warp's blocks of the segment: CTA block indices j = t.. with j % NW == warp ----
     const int j0 = t + ((warp - t) % NW + NW) % NW;
-    if constexpr (CANDS) c_first = c + (j0 - t);
     for (int j = j0; j < t + seg; j += NW) {
       const int i = (j - warp) / NW;  // the warp's own block number
       const int slot = warp * kDepth + i % kDepth;
@@ -572,7 +401,6 @@ __global__ void __launch_bounds__(Cfg<R, GATED, KP8, CANDS>::kThreads, 1) score_
                                                        part * 16);
         if constexpr (GATED) lgv[bt] = reinterpret_cast<const float*>(st + kBlockBytes)[bt * 32 + part * Gm::RPI + rsub];
       }
-      const uint32_t tau = CANDS ? ld_volatile_u32(tau_lo) << (32 - kCandHistBits) : 0u;
       __syncwarp();  // every lane has read the slot
       if (lane == 0 && i + kDepth < my_blocks) issue(slot);
 #pragma unroll
@@ -587,11 +415,10 @@ __global__ void __launch_bounds__(Cfg<R, GATED, KP8, CANDS>::kThreads, 1) score_
           const float u0 = butterfly<Gm>(v, lane);
           const int lr = part * Gm::RPI + rsub;
           const float u = GATED ? fmaf(p.lam, lgv[bt], u0) : u0;
-          take_key(u, bh, row0 + bt * 32 + lr, lr < wrows, tau);
+          take_key(u, bh, row0 + bt * 32 + lr, lr < wrows);
         }
       }
     }
-    close_record(bh);
 
     // ---- next head ----
     t += seg;
@@ -603,25 +430,21 @@ __global__ void __launch_bounds__(Cfg<R, GATED, KP8, CANDS>::kThreads, 1) score_
     }
   }
   consumers_sync<kConsumers>();
-  if constexpr (!CANDS) {
-    if (cur_bh >= 0) {
-      uint32_t* gh = p.hist + (size_t)cur_bh * kHistBins;
-      for (int i = tid; i < C::kBins; i += kConsumers) {
-        const uint32_t v = S.hist[i];
-        if (v && cur_ranked) atomicAdd(&gh[i], v);
-      }
+  if (cur_bh >= 0 && cur_ranked) {
+    uint32_t* gh = p.hist + (size_t)cur_bh * C::kBins;
+    for (int i = tid; i < C::kBins; i += kConsumers) {
+      const uint32_t v = S.hist[i];
+      if (v) atomicAdd(&gh[i], v);
     }
-  } else {
-    if (tid == 0) atomicExch(&S.tau_state, (unsigned long long)kTauDone << 32);
   }
   if (!waited_ok) record_error(p.err, kDevWaitTimeout, blockIdx.x);
 }
 
-template <int R, int D, bool GATED, bool KP8, bool CANDS>
+template <int R, int D, bool GATED, bool KP8>
 cudaError_t launch_v(const ScoreParams& p, cudaStream_t stream) {
-  using C = Cfg<R, GATED, KP8, CANDS>;
-  auto kern = score_kernel<R, D, GATED, KP8, CANDS>;
-  const int smem = (int)sizeof(Smem<R, D, GATED, KP8, CANDS>);
+  using C = Cfg<R, GATED, KP8>;
+  auto kern = score_kernel<R, D, GATED, KP8>;
+  const int smem = (int)sizeof(Smem<R, D, GATED, KP8>);
   cudaError_t e = prepare_kernel((const void*)kern, smem);
   if (e != cudaSuccess) return e;
   return launch_pdl(kern, dim3((unsigned)p.ctas), dim3(C::kThreads), (size_t)smem, stream, p);
@@ -630,12 +453,8 @@ cudaError_t launch_v(const ScoreParams& p, cudaStream_t stream) {
 template <int R, int D>
 cudaError_t launch_rd(const ScoreParams& p, cudaStream_t stream) {
   const bool gated = p.log_g != nullptr;
-  if (p.cands) {
-    if (p.fp8) return gated ? launch_v<R, D, true, true, true>(p, stream) : launch_v<R, D, false, true, true>(p, stream);
-    return gated ? launch_v<R, D, true, false, true>(p, stream) : launch_v<R, D, false, false, true>(p, stream);
-  }
-  if (p.fp8) return gated ? launch_v<R, D, true, true, false>(p, stream) : launch_v<R, D, false, true, false>(p, stream);
-  return gated ? launch_v<R, D, true, false, false>(p, stream) : launch_v<R, D, false, false, false>(p, stream);
+  if (p.fp8) return gated ? launch_v<R, D, true, true>(p, stream) : launch_v<R, D, false, true>(p, stream);
+  return gated ? launch_v<R, D, true, false>(p, stream) : launch_v<R, D, false, false>(p, stream);
 }
 
 }  // namespace
@@ -647,7 +466,6 @@ void plan_score(ScoreParams& p, int num_sms) {
   long long ctas = num_sms;
   if (ctas > blocks) ctas = blocks;
   p.ctas = (int)(ctas < 1 ? 1 : ctas);
-  p.block_rows = br;
 }
 
 cudaError_t launch_score(const ScoreParams& p, cudaStream_t stream) {

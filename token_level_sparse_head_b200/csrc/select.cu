@@ -36,7 +36,6 @@ constexpr int kMaxWords = kChunkMax / 32;     // bitmap words per CTA
 constexpr int kCap = 4096;                    // candidate list entries (CTA 0: the whole head's)
 constexpr int kMaxTies = 256;                 // ties on T resolved by CTA 0; more take the slow path
 constexpr uint32_t kFast = 1u, kSlow = 2u;
-constexpr long long kSmemLimitSel = 227 * 1024;
 
 struct Found {
   uint32_t digit, above, eq, pad;
@@ -555,255 +554,9 @@ __global__ void __launch_bounds__(THREADS, 1) select_topk_kernel(const SelectPar
   if (!waited_ok) record_error(p.err, kDevWaitTimeout, (uint32_t)bh);
 }
 
-// ---------------------------------------------------------------------------------------------
-// Candidate mode.  The score kernel has left, per head, a list of records (first block and block
-// stride, even count) that point at (key, position) pairs: every key at or above a lower bound of
-// the head's k-th largest key, plus sentinels of key 0; and a histogram of the top 12 bits of those
-// keys.  The candidates hold every key that can be selected and at least k of them, so the k-th
-// largest candidate key is the head's k-th largest key T.  One CTA per head:
-//   1. digit 1 of T (12 bits) from the histogram;
-//   2. one pass over the candidates (read from L2, eight 16-byte loads in flight per thread): keys
-//      with a larger digit 1 are selected and set in a bitmap of the head's positions, keys with
-//      digit 1 equal to T's go to a list in shared memory;
-//   3. digits 2 and 3 of T (10 bits each) among the list, then, when T has more ties than the
-//      budget takes, the lowest positions among them as two 9-bit digits of the position;
-//   4. the chosen list entries into the bitmap, and the bitmap out as ascending positions.
-// If the list does not fit on chip (many keys share T's digit 1), steps 3 and 4 make their passes
-// over all candidates instead.
-constexpr int kCandBins1 = 1 << kCandHistBits;  // 4096: digit 1
-constexpr int kListCap = 8192;                  // on-chip entries of digit 1's bin
-
-struct CandCtl {
-  uint32_t hist[1024];
-  uint32_t wsum[32];
-  Found found;
-  uint32_t nlist;
-  uint32_t pad[3];
-};
-static_assert(sizeof(CandCtl) % 16 == 0, "shared-memory layout alignment");
-
-template <int THREADS>
-__global__ void __launch_bounds__(THREADS, 1) select_cand_kernel(const SelectParams p) {
-  extern __shared__ __align__(128) unsigned char smem_raw[];
-  CandCtl& S = *reinterpret_cast<CandCtl*>(smem_raw);
-  uint2* list = reinterpret_cast<uint2*>(smem_raw + sizeof(CandCtl));
-  uint2* rrec = list + kListCap;
-  uint32_t* rpre = reinterpret_cast<uint32_t*>(rrec + p.rec_cap);
-  uint32_t* bm = rpre + ((p.rec_cap + 4) & ~3);
-  const int tid = threadIdx.x;
-  const int bh = blockIdx.x;
-  const int b = bh / p.Hkv;
-
-  // per-sequence values (range errors were recorded by the score kernel)
-  int n = p.seqlens[b];
-  if (n < 0 || n > p.cap) n = 0;
-  const SeqSelection sel = seq_selection(min(p.kvec[b], p.k_max), n);
-  const int k_eff = sel.k_eff;
-  int32_t* idx = p.idx_out + (size_t)bh * p.k_max;
-
-  if (!sel.ranked) {
-    // Nothing to rank (the scan wrote no candidates): the first k_eff positions, or none.
-    pdl_wait();
-    pdl_trigger();
-    for (int j = tid; j < p.k_max; j += THREADS) idx[j] = (j < k_eff) ? j : -1;
-    return;
-  }
-
-  const int nwords = (n + 31) >> 5;
-  for (int i = tid; i < nwords; i += THREADS) bm[i] = 0u;
-  if (tid == 0) {
-    S.found = Found{};
-    S.nlist = 0u;
-  }
-  __syncthreads();
-  // The candidates, records, record counts and histograms of the score pass are read only from
-  // here on.
-  pdl_wait();
-  pdl_trigger();
-
-  // ---- records: copied on chip, with the offsets of their entries in one flat order ----
-  uint32_t R = p.rec_cnt[bh];
-  if (R > (uint32_t)p.rec_cap) {  // cannot happen: at most 16 warps of every scanning CTA
-    if (tid == 0) record_error(p.err, kDevCandidates, (uint32_t)bh);
-    R = (uint32_t)p.rec_cap;
-  }
-  const uint2* recs = p.recs + (size_t)bh * p.rec_stride;
-  const int rpt = (int)((R + THREADS - 1) / THREADS);
-  const int r0 = min(tid * rpt, (int)R), r1 = min(r0 + rpt, (int)R);
-  uint32_t mine = 0u;
-  for (int r = r0; r < r1; ++r) {
-    const uint2 rc = recs[r];
-    rrec[r] = rc;
-    mine += rc.y;
-  }
-  uint32_t total;
-  uint32_t off = block_excl_scan<THREADS>(mine, S.wsum, &total);
-  for (int r = r0; r < r1; ++r) {
-    rpre[r] = off;
-    off += rrec[r].y;
-  }
-  if (tid == 0) {
-    rpre[R] = total;
-    p.rec_cnt[bh] = 0u;  // every thread has read it: ready for the next scan
-  }
-
-  // ---- digit 1 from the score pass's histogram, which is then cleared for the next scan ----
-  uint32_t* gh = p.hist + (size_t)bh * kCandBins1;
-  find_digit<kCandBins1, THREADS>(gh, (uint32_t)k_eff, S.wsum, &S.found);  // ends with a barrier
-  const uint32_t d1 = S.found.digit;
-  const uint32_t eq1 = S.found.eq;
-  uint32_t k_rem = (uint32_t)k_eff - S.found.above;
-  for (int i = tid; i < kCandBins1 / 4; i += THREADS) reinterpret_cast<uint4*>(gh)[i] = make_uint4(0u, 0u, 0u, 0u);
-
-  if ((uint32_t)k_eff > total || eq1 == 0u) {
-    // Cannot happen (every key >= T is a candidate and counted); leave a defined output.
-    if (tid == 0) record_error(p.err, kDevCandidates, (uint32_t)bh);
-    for (int j = tid; j < p.k_max; j += THREADS) idx[j] = -1;
-    return;
-  }
-
-  const uint2* cand = p.cand + (size_t)bh * p.cand_stride;
-  const int BR = p.block_rows;
-  const int lbr = __ffs(BR) - 1;  // BR is a power of two
-  // fn(key, position) over every candidate, pairs of entries (16-byte loads; record counts and
-  // block pieces are even) taken by consecutive threads, eight loads in flight per thread
-  auto stream = [&](auto&& fn) {
-    const uint32_t pairs = total >> 1;
-    uint32_t r = 0u;
-    constexpr int U = 8;
-    for (uint32_t j0 = (uint32_t)tid; j0 < pairs; j0 += U * THREADS) {
-      uint4 v[U];
-#pragma unroll
-      for (int u = 0; u < U; ++u) {
-        const uint32_t j = j0 + (uint32_t)u * THREADS;
-        v[u] = make_uint4(0u, 0u, 0u, 0u);
-        if (j < pairs) {
-          const uint32_t e = 2u * j;
-          while (rpre[r + 1] <= e) ++r;  // entries only move forward
-          const uint32_t o = e - rpre[r];
-          const uint2 rc = rrec[r];
-          const size_t at = ((size_t)(rc.x & 0xffffffu) + (size_t)(o >> lbr) * (rc.x >> 24)) * BR + (o & (uint32_t)(BR - 1));
-          v[u] = __ldcg(reinterpret_cast<const uint4*>(cand + at));
-        }
-      }
-#pragma unroll
-      for (int u = 0; u < U; ++u) {
-        fn(v[u].x, v[u].y);  // a zero pair (past the end) has key 0: below every real key
-        fn(v[u].z, v[u].w);
-      }
-    }
-  };
-  auto mark = [&](uint32_t pos) { atomicOr(&bm[pos >> 5], 1u << (pos & 31)); };
-
-  // ---- one pass: above digit 1 into the bitmap, digit 1's bin into the list ----
-  const bool listed = eq1 <= (uint32_t)kListCap;
-  stream([&](uint32_t key, uint32_t pos) {
-    const uint32_t dg = key >> (32 - kCandHistBits);
-    if (dg > d1) {
-      mark(pos);
-    } else if (dg == d1 && listed) {
-      const uint32_t slot = atomicAdd(&S.nlist, 1u);
-      if (slot < (uint32_t)kListCap) list[slot] = make_uint2(key, pos);
-    }
-  });
-  for (int i = tid; i < 1024; i += THREADS) S.hist[i] = 0u;
-  __syncthreads();
-  const uint32_t nl = min(S.nlist, (uint32_t)kListCap);
-  // fn over the keys in digit 1's bin: the list, or every candidate filtered again
-  auto over_bin = [&](auto&& fn) {
-    if (listed) {
-      for (uint32_t e = tid; e < nl; e += THREADS) fn(list[e].x, list[e].y);
-    } else {
-      stream([&](uint32_t key, uint32_t pos) {
-        if ((key >> (32 - kCandHistBits)) == d1) fn(key, pos);
-      });
-    }
-  };
-  auto clear_hist = [&]() {
-    for (int i = tid; i < 1024; i += THREADS) S.hist[i] = 0u;
-    __syncthreads();
-  };
-
-  // ---- digits 2 and 3 of T (10 bits each) ----
-  over_bin([&](uint32_t key, uint32_t) { atomicAdd(&S.hist[(key >> 10) & 1023u], 1u); });
-  __syncthreads();
-  find_digit<1024, THREADS>(S.hist, k_rem, S.wsum, &S.found);
-  const uint32_t pre = (d1 << 10) | S.found.digit;
-  k_rem -= S.found.above;
-  clear_hist();
-  over_bin([&](uint32_t key, uint32_t) {
-    if ((key >> 10) == pre) atomicAdd(&S.hist[key & 1023u], 1u);
-  });
-  __syncthreads();
-  find_digit<1024, THREADS>(S.hist, k_rem, S.wsum, &S.found);
-  const uint32_t T = (pre << 10) | S.found.digit;
-  const uint32_t need = k_rem - S.found.above;  // ties on T to take, 1 <= need <= eq
-  const uint32_t eq = S.found.eq;
-
-  // ---- ties: the need lowest positions among the keys equal to T (positions < 2^18) ----
-  uint32_t cut = 0xffffffffu;
-  if (need < eq) {
-    clear_hist();
-    over_bin([&](uint32_t key, uint32_t pos) {
-      if (key == T) atomicAdd(&S.hist[511u - (pos >> 9)], 1u);
-    });
-    __syncthreads();
-    find_digit<512, THREADS>(S.hist, need, S.wsum, &S.found);
-    const uint32_t ph = 511u - S.found.digit;
-    const uint32_t need2 = need - S.found.above;
-    clear_hist();
-    over_bin([&](uint32_t key, uint32_t pos) {
-      if (key == T && (pos >> 9) == ph) atomicAdd(&S.hist[511u - (pos & 511u)], 1u);
-    });
-    __syncthreads();
-    find_digit<512, THREADS>(S.hist, need2, S.wsum, &S.found);
-    cut = (ph << 9) | (511u - S.found.digit);
-  }
-
-  // ---- the chosen keys of digit 1's bin into the bitmap ----
-  over_bin([&](uint32_t key, uint32_t pos) {
-    if (key > T || (key == T && pos <= cut)) mark(pos);
-  });
-  __syncthreads();
-
-  // ---- ordered output ----
-  {
-    const int wpt = (nwords + THREADS - 1) / THREADS;
-    const int w0 = min(tid * wpt, nwords), w1 = min(w0 + wpt, nwords);
-    uint32_t cnt = 0u;
-    for (int w = w0; w < w1; ++w) cnt += (uint32_t)__popc(bm[w]);
-    uint32_t tot;
-    uint32_t o = block_excl_scan<THREADS>(cnt, S.wsum, &tot);
-    for (int w = w0; w < w1; ++w) {
-      uint32_t bits = bm[w];
-      while (bits) {
-        const int e = __ffs(bits) - 1;
-        bits &= bits - 1u;
-        if (o < (uint32_t)k_eff) idx[o] = w * 32 + e;
-        ++o;
-      }
-    }
-  }
-  for (int j = k_eff + tid; j < p.k_max; j += THREADS) idx[j] = -1;
-}
-
 }  // namespace
 
 bool plan_select(SelectParams& p, int num_sms) {
-  if (p.cands) {
-    // one CTA per head: the on-chip list of digit 1's bin, the head's records and its bitmap
-    p.cluster = 1;
-    p.threads = 1024;
-    p.chunk = p.cap;
-    p.rec_cap = 16 * (num_sms > 0 ? num_sms : 148);  // records per head: 16 warps of every scanning CTA
-    if (p.rec_cap > p.rec_stride) p.rec_cap = p.rec_stride;
-    p.bm_words = (p.cap + 31) / 32;
-    const long long bytes = (long long)sizeof(CandCtl) + (long long)kListCap * 8 + (long long)p.rec_cap * 8 +
-                            (long long)((p.rec_cap + 4) & ~3) * 4 + (long long)p.bm_words * 4;
-    if (bytes > kSmemLimitSel) return false;
-    p.smem_bytes = (int)bytes;
-    return true;
-  }
   const int heads = p.B * p.Hkv;
   // One CTA per SM.  Split a head over a cluster while its chunk is too long, and while the
   // grid still leaves SMs idle (up to the portable cluster size).
@@ -822,12 +575,6 @@ bool plan_select(SelectParams& p, int num_sms) {
 }
 
 cudaError_t launch_select(const SelectParams& p, cudaStream_t stream) {
-  if (p.cands) {
-    auto kern = select_cand_kernel<1024>;
-    const cudaError_t e = prepare_kernel((const void*)kern, p.smem_bytes);
-    if (e != cudaSuccess) return e;
-    return launch_pdl(kern, dim3((unsigned)(p.B * p.Hkv)), dim3(1024u), (size_t)p.smem_bytes, stream, p);
-  }
   auto kern = p.threads == 512 ? select_topk_kernel<512> : select_topk_kernel<1024>;
   const cudaError_t e = prepare_kernel((const void*)kern, p.smem_bytes, p.cluster > 8);
   if (e != cudaSuccess) return e;

@@ -37,7 +37,6 @@ _SIGS = {
     "sas_last_error_detail": (ctypes.c_char_p, []),
     "sas_decode_workspace_bytes": (_sz, [ctypes.POINTER(sas_shape), _i32]),
     "sas_dense_workspace_bytes": (_sz, [ctypes.POINTER(sas_shape)]),
-    "sas_selection_mode": (ctypes.c_int, [ctypes.POINTER(sas_shape), _i32]),
     "sas_workspace_init": (ctypes.c_int, [_vp, _sz, _vp]),
     "sas_check_workspace": (ctypes.c_int, [_vp, _sz, _vp, ctypes.POINTER(ctypes.c_uint32),
                                            ctypes.POINTER(ctypes.c_uint32)]),
@@ -159,11 +158,6 @@ def sas_decode_workspace_bytes(shape: Shape, k_max: int) -> int:
 
 def sas_dense_workspace_bytes(shape: Shape) -> int:
     return int(load().sas_dense_workspace_bytes(ctypes.byref(shape.c())))
-
-
-def sas_selection_mode(shape: Shape, k_max: int) -> int:
-    """0: every key is written and streamed; 1: per-head candidates only; -1: invalid."""
-    return int(load().sas_selection_mode(ctypes.byref(shape.c()), int(k_max)))
 
 
 def sas_workspace_init(workspace, ws_bytes: int, stream=None):
