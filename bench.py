@@ -264,6 +264,30 @@ def timed_block(torch, fn, steps, dist=None):
     return max_over_ranks(e0.elapsed_time(e1) / 1e3, dist)
 
 
+def step_distribution(torch, fn, min_steps=50, min_seconds=1.0, flush_buf=None):
+    """Per-step device times of fn (CUDA events around each call), over at least min_steps
+    calls and at least min_seconds of calls; an L2 flush before each call when flush_buf is
+    given.  Returns {median, p10, p90, mean, n} in milliseconds."""
+    ts = []
+    t_end = time.perf_counter() + min_seconds
+    chunk = 50
+    while len(ts) < min_steps or time.perf_counter() < t_end:
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(chunk)]
+        for e0, e1 in evs:
+            if flush_buf is not None:
+                flush_l2(flush_buf)
+            e0.record()
+            fn()
+            e1.record()
+        torch.cuda.synchronize()
+        ts.extend(e0.elapsed_time(e1) for e0, e1 in evs)
+        if len(ts) >= 200000:
+            break
+    ts.sort()
+    q = lambda f: ts[min(len(ts) - 1, int(f * (len(ts) - 1) + 0.5))]
+    return {"median": q(0.5), "p10": q(0.1), "p90": q(0.9), "mean": statistics.mean(ts), "n": len(ts)}
+
+
 def flush_l2(flush_buf):
     """Evict L2: write a buffer twice the L2 size, then read it back, so the lines left in L2
     are clean and the timed step does not pay for the flush's write-back."""
@@ -387,9 +411,13 @@ def run_ours(args):
     # from a CUDA graph of the step (as a decode server runs it); the same K steps launched
     # call by call are reported beside it
     graph = capture_graph(torch, wl.step)
+    replay = graph.replay if graph is not None else wl.step
     t_stream = timed_block(torch, wl.step, args.steps, dist)
+    # clocks are sampled over a window of at least a second under load: the per-step
+    # distribution (each replay between two events) and then the headline block itself
     sampler = ClockSampler(smi_device_id(torch, local))
-    t = timed_block(torch, graph.replay if graph is not None else wl.step, args.steps, dist)
+    dist_ms = step_distribution(torch, replay, min_steps=50, min_seconds=1.0)
+    t = timed_block(torch, replay, args.steps, dist)
     clocks = sampler.stop()
     ms = t / args.steps * 1e3
     value = job_throughput(args.steps, world, t)
@@ -492,7 +520,9 @@ def run_ours(args):
         n1 = max(10, min(args.steps, 100))
         t1_stream = flushed_steps(torch, w1.step, n1, flush)
         g1 = capture_graph(torch, w1.step)
-        t1 = flushed_steps(torch, g1.replay, n1, flush) if g1 is not None else t1_stream
+        d1 = step_distribution(torch, g1.replay if g1 is not None else w1.step, min_steps=100, min_seconds=0.3,
+                               flush_buf=flush)
+        t1 = d1["median"] * 1e-3
         gd1 = capture_graph(torch, w1.dense)
         td1 = flushed_steps(torch, gd1.replay if gd1 is not None else w1.dense, 10, flush)
         # each kernel alone, replayed from its own graph after an L2 flush
@@ -501,7 +531,7 @@ def run_ours(args):
             gk = capture_graph(torch, fn)
             kt[kname] = flushed_steps(torch, gk.replay if gk is not None else fn, 20, flush) * 1e3
         secondary = {"workload": SECONDARY_WORKLOAD, "ms_per_step": t1 * 1e3, "steps_per_s": 1.0 / t1,
-                     "ms_per_step_stream": t1_stream * 1e3,
+                     "ms_per_step_stream": t1_stream * 1e3, "p10": d1["p10"], "p90": d1["p90"], "n": d1["n"],
                      "hbm_gbs": w1.bytes["step"] / t1 / 1e9, "dense_ms_per_step": td1 * 1e3,
                      "speedup_vs_dense": td1 / t1, "l2": "flushed between steps (2x L2 written, then read)",
                      "timing": "CUDA graph replay of the step" if g1 is not None else "stream launches",
@@ -533,6 +563,14 @@ def run_ours(args):
                "timing": "CUDA graph replay of the step" if g8 is not None else "stream launches"}
         wl = w8
 
+    # --- the other named workloads: 8B-shaped 32K, paged variable-length B=16, gated budget sweep
+    others = None
+    if not args.no_workloads and args.workload == DEFAULT_WORKLOAD:
+        wl.free()
+        del wl
+        wl = None
+        others = {name: time_workload(torch, name, dev) for name in OTHER_WORKLOADS}
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(args.workload, budget_s=args.cpu_seconds)
@@ -542,15 +580,14 @@ def run_ours(args):
         dist.destroy_process_group()
     if rank != 0:
         return
-    c = CONFIGS_VIEW(args.workload)
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms, "ms_per_step_stream": t_stream / args.steps * 1e3,
+        "ms_per_step_dist": dist_ms,
         "timing": "CUDA graph replay of the step" if graph is not None else "stream launches",
         "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f32", "storage_dtype": "bf16", "data": "synthetic",
-        "config": dict(workload=args.workload, **c, l2="inputs larger than L2: each step reads "
-                       f"{head_bytes['step'] / 1e9:.2f} GB, L2 is 0.13 GB", parallelism=f"replicas x{world}"),
+        "config": config_view(args.workload, world),
         "hbm_gbs": None, "speedup_vs_dense": dense_ms / ms,
         "dense": {"ms_per_step": dense_ms, "steps_per_s": 1e3 / dense_ms},
         "kernels_ms": k_ms,
@@ -570,29 +607,142 @@ def run_ours(args):
         line["fp8_kproj"] = fp8
     if foil:
         line["gather_foil"] = foil
+    if others:
+        line["workloads"] = others
     line["selection_recall"] = {"value": recall, "definition": "mean over (sequence, KV head) of the fraction of "
                                 "the exact top-k by q-bar . k_i (full dimension) that the projected selection keeps; "
                                 "synthetic data"}
     print(json.dumps(line), flush=True)
 
 
-def CONFIGS_VIEW(name):
+OTHER_WORKLOADS = ("8b-32k", "paged-b16", "gated-b4-k256", "gated-b4-k1024", "gated-b4-k4096", "gated-b4-k16384")
+
+
+def workload_bytes(name):
+    """Roofline bytes of one step of a named workload from its definition (the paged workload:
+    at the mean sequence length of its uniform draw)."""
+    from synth import CONFIGS
+
+    c = CONFIGS[name]
+    kp = 1 if c.get("kproj_fp8") else 2
+    n = c["N"] if c["N"] else (c["n_lo"] + c["n_hi"]) / 2
+    k = c["k"] if c["k"] else n / c["k_div"]
+    return roofline_bytes(c["B"], c["Hq"], c["Hkv"], c["d"], c["r"], [n] * c["B"], [k] * c["B"],
+                          c.get("lam", 0.0), kp_bytes=kp)["step"]
+
+
+def l2_policy(step_bytes):
+    """Steps that read less than twice the L2 are timed with an L2 flush before each step."""
+    return step_bytes < 2 * L2_BYTES
+
+
+def config_view(name, world):
+    """The config dict both arms print for a workload: its shape, the L2 treatment of the timing
+    and the parallelism."""
     from synth import CONFIGS
 
     c = dict(CONFIGS[name])
-    return {k: c[k] for k in ("B", "Hq", "Hkv", "d", "r", "N", "k") if k in c} | (
-        {"lam": c["lam"]} if "lam" in c else {})
+    v = {k: c[k] for k in ("B", "Hq", "Hkv", "d", "r", "N", "k") if k in c}
+    if c.get("lam"):
+        v["lam"] = c["lam"]
+    if c.get("paged"):
+        v.update(n_lo=c["n_lo"], n_hi=c["n_hi"], k="N_b/%d" % c["k_div"], page_size=64)
+    if c.get("kproj_fp8"):
+        v["kproj"] = "fp8_e4m3"
+    step = workload_bytes(name)
+    v["l2"] = (f"L2 flushed before each step (a step reads {step / 1e9:.3f} GB, L2 is 0.13 GB)" if l2_policy(step)
+               else f"inputs larger than L2: each step reads {step / 1e9:.2f} GB, L2 is 0.13 GB")
+    v["parallelism"] = f"replicas x{world}"
+    return dict(workload=name, **v)
+
+
+def time_workload(torch, name, dev):
+    """One named workload: the step (append + decode step, CUDA graph replay) and the dense decode,
+    each as a median over replays, with its roofline bytes and bandwidth."""
+    w = Workload(name, dev, torch)
+    step_bytes = w.bytes["step"]
+    flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev) if l2_policy(step_bytes) else None
+    for _ in range(3):
+        w.step()
+    g = capture_graph(torch, w.step)
+    st = step_distribution(torch, g.replay if g is not None else w.step, min_steps=50, min_seconds=0.2,
+                           flush_buf=flush)
+    gd = capture_graph(torch, w.dense)
+    dn = step_distribution(torch, gd.replay if gd is not None else w.dense, min_steps=20, min_seconds=0.1,
+                           flush_buf=flush)
+    out = {"ms_per_step": st["median"], "p10": st["p10"], "p90": st["p90"], "steps_per_s": 1e3 / st["median"],
+           "step_bytes": step_bytes, "hbm_gbs": step_bytes / (st["median"] * 1e-3) / 1e9,
+           "dense_ms_per_step": dn["median"], "dense_hbm_gbs": w.dense_bytes / (dn["median"] * 1e-3) / 1e9,
+           "speedup_vs_dense": dn["median"] / st["median"],
+           "l2": "flushed before each step" if flush is not None else "inputs larger than L2",
+           "timing": "median of CUDA graph replays"}
+    del g, gd, flush
+    w.free()
+    del w
+    return out
 
 
 # ------------------------------------------------------------------------------ oracle arm
-def _threads_used():
-    try:
-        from threadpoolctl import threadpool_info
+# The oracle runs one (sequence, KV head) pair at a time; a step is every pair of the workload.
+# Pairs are independent, so a pool of single-threaded worker processes (spawned, so nothing of
+# a CUDA context is inherited) takes them in parallel.  Each worker holds one seeded draw of the
+# workload's pair shape and runs the oracle on it for every pair it is handed: the oracle's
+# arithmetic does not depend on the values.
+_ORACLE_PAIR = None
 
-        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
-        return max(n) if n else 1
-    except Exception:
-        return 1
+
+def _oracle_worker_init(name):
+    import multiprocessing
+
+    global _ORACLE_PAIR
+    ident = multiprocessing.current_process()._identity
+    _ORACLE_PAIR = oracle_head_problem(name, seed=2000 + (ident[0] if ident else 0))
+
+
+def _oracle_worker_run(_):
+    return oracle_head_seconds(_ORACLE_PAIR)
+
+
+class OraclePool:
+    """Worker processes for whole oracle steps of a workload."""
+
+    THREAD_VARS = ("OMP_NUM_THREADS", "OPENBLAS_NUM_THREADS", "MKL_NUM_THREADS")
+
+    def __init__(self, name, workers=None):
+        import multiprocessing
+
+        from synth import CONFIGS
+
+        c = CONFIGS[name]
+        self.pairs = c["B"] * c["Hkv"]
+        self.workers = max(1, min(workers or (os.cpu_count() or 1), self.pairs, 32))
+        saved = {k: os.environ.get(k) for k in self.THREAD_VARS}
+        for k in self.THREAD_VARS:
+            os.environ[k] = "1"  # every worker single-threaded: cores = workers
+        try:
+            self.pool = multiprocessing.get_context("spawn").Pool(self.workers, initializer=_oracle_worker_init,
+                                                                 initargs=(name,))
+        finally:
+            for k, v in saved.items():
+                if v is None:
+                    os.environ.pop(k, None)
+                else:
+                    os.environ[k] = v
+
+    def step(self):
+        """Wall seconds of one step: the oracle on every (sequence, KV head) pair."""
+        t0 = time.perf_counter()
+        self.pool.map(_oracle_worker_run, range(self.pairs), chunksize=1)
+        return time.perf_counter() - t0
+
+    def close(self):
+        self.pool.close()
+        self.pool.join()
+
+    def sample(self, steps):
+        return (f"{steps} whole oracle steps; each step runs the oracle on all {self.pairs} (sequence, KV head) "
+                f"pairs, spread over {self.workers} single-threaded worker processes, each holding one seeded "
+                f"draw of the workload's pair")
 
 
 def oracle_head_problem(name, seed):
@@ -623,63 +773,44 @@ def oracle_head_seconds(h):
 
 
 def cpu_baseline(name, budget_s=15.0):
-    """The oracle, as it stands, on a bounded sample of the workload: whole heads (one sequence x
-    one KV head each) until about budget_s seconds of oracle time; steps/s extrapolates to all
-    B*Hkv heads of a step."""
-    from synth import CONFIGS
-
-    c = CONFIGS[name]
-    heads_per_step = c["B"] * c["Hkv"]
-    distinct = [oracle_head_problem(name, seed=1000 + i) for i in range(min(heads_per_step, 8))]
-    ts = []
-    while sum(ts) < budget_s and len(ts) < 100000:
-        ts.append(oracle_head_seconds(distinct[len(ts) % len(distinct)]))
-    per_head = statistics.mean(ts)
-    out = {"value": 1.0 / (per_head * heads_per_step), "unit": UNIT, "cores": _threads_used(),
-           "kind": "oracle", "sample": f"{len(ts)} oracle runs over {len(distinct)} distinct (sequence, KV head) "
-           f"pairs of the workload ({sum(ts):.1f} s of oracle time); one step = {heads_per_step} pairs"}
-    # the same oracle held to one thread, on a third of the budget
+    """The oracle, as it stands, on whole steps of the workload for about budget_s seconds of CPU
+    time (wall time x workers), at least one step."""
+    pool = OraclePool(name)
     try:
-        from threadpoolctl import threadpool_limits
-
-        t1 = []
-        with threadpool_limits(limits=1):
-            while sum(t1) < budget_s / 3 and len(t1) < 100000:
-                t1.append(oracle_head_seconds(distinct[len(t1) % len(distinct)]))
-        out["value_1_thread"] = 1.0 / (statistics.mean(t1) * heads_per_step)
-    except ImportError:
-        pass
-    return out
+        pool.step()  # warm-up: workers have loaded their pair
+        ts = []
+        while not ts or (sum(ts) * pool.workers < budget_s and len(ts) < 1000):
+            ts.append(pool.step())
+    finally:
+        pool.close()
+    per_step = statistics.mean(ts)
+    return {"value": 1.0 / per_step, "unit": UNIT, "cores": pool.workers, "kind": "oracle",
+            "sample": pool.sample(len(ts)), "ms_per_step": per_step * 1e3}
 
 
 def run_reference(args):
+    """The reference arm: the oracle (numpy, fp64) on whole steps of the workload on the host
+    cores, --warmup untimed steps then --steps timed ones; rank 0 only."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
-    from synth import CONFIGS
-
-    c = CONFIGS[args.workload]
-    heads_per_step = c["B"] * c["Hkv"]
-    h = oracle_head_problem(args.workload, seed=2000)
-    for _ in range(max(0, min(args.warmup, 3))):
-        oracle_head_seconds(h)
-    ts = []
-    t_start = time.perf_counter()
-    for i in range(args.steps):
-        ts.append(oracle_head_seconds(h))
-        if time.perf_counter() - t_start > args.cpu_seconds * 4:
-            break
-    per_head = statistics.mean(ts)
-    value = 1.0 / (per_head * heads_per_step)
+    pool = OraclePool(args.workload)
+    try:
+        for _ in range(args.warmup):
+            pool.step()
+        ts = [pool.step() for _ in range(args.steps)]
+    finally:
+        pool.close()
+    total = sum(ts)
+    value = args.steps / total
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
-        "steps": len(ts), "warmup": args.warmup, "ms_per_step": per_head * heads_per_step * 1e3,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": total / args.steps * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-        "data": "synthetic", "config": dict(workload=args.workload, **CONFIGS_VIEW(args.workload)),
-        "cpu_baseline": {"value": value, "unit": UNIT, "cores": _threads_used(), "kind": "oracle",
-                         "sample": f"{len(ts)} timed oracle runs of one (sequence, KV head) pair of "
-                                   f"the workload; each step = {heads_per_step} such pairs"},
+        "data": "synthetic", "config": config_view(args.workload, world),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": pool.workers, "kind": "oracle",
+                         "sample": pool.sample(args.steps)},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -697,6 +828,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-fp8", action="store_true", help="skip the FP8 projected-cache line")
     ap.add_argument("--no-foil", action="store_true", help="skip the gather-then-attend line")
+    ap.add_argument("--no-workloads", action="store_true", help="skip the other named workloads")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--recall-report", action="store_true",
                     help="print the selection recall of every named workload instead of timing")
