@@ -10,13 +10,13 @@
 //
 // Persistent kernel, one CTA per SM.  The work is the list of 4 KB blocks of projected rows
 // (64 rows at r = 32 in bf16) of every (b, h) that needs scores, in (b, h, position) order; each
-// CTA takes one contiguous, equal share of it.  Its consumer warps take the share's blocks in
-// turn; each warp owns two ring slots in shared memory and keeps them full itself: once its
-// lanes have moved a landed block into registers, lane 0 issues the bulk copy (TMA engine,
-// mbarrier completion) of the warp's next block into that slot, and only then does the warp
-// compute, so a slot is out of flight only for the few shared-memory loads that empty it and no
-// warp waits on another.  Per 32-row batch the lanes form 16-byte dot products with q-hat and
-// meet in a transposing butterfly.
+// CTA takes one contiguous, equal share of it.  A producer warp streams the blocks into a ring of
+// 32 shared-memory slots with bulk copies (TMA engine, mbarrier completion); each producer lane
+// owns one slot.  Sixteen consumer warps take the blocks in turn, two slots each: a consumer warp
+// moves a landed block into registers (eight 16-byte pieces per lane) and hands the slot straight
+// back to its producer lane before computing, so a slot is out of flight only for the few
+// shared-memory loads that empty it.  Per 32-row batch the lanes form 16-byte dot products with
+// q-hat and meet in a transposing butterfly.
 
 #include <cuda_fp16.h>
 #include <cuda_fp8.h>
@@ -47,7 +47,7 @@ struct Geo {
 };
 
 // Block shape of one instantiation: as many consumer warps (two slots each) as shared memory
-// holds next to the histogram, at most 16.
+// holds next to the histogram, at most 16, and one producer lane per slot.
 template <int R, bool GATED, bool KP8>
 struct Cfg {
   using Gm = Geo<R, KP8>;
@@ -57,7 +57,8 @@ struct Cfg {
   static constexpr int kWarps = kMaxSlots / kDepth >= kMaxWarps ? kMaxWarps : kMaxSlots / kDepth;
   static constexpr int kSlots = kWarps * kDepth;
   static constexpr int kConsumers = kWarps * 32;
-  static constexpr int kThreads = kConsumers;
+  static constexpr int kProducerWarps = (kSlots + 31) / 32;
+  static constexpr int kThreads = kConsumers + kProducerWarps * 32;
 };
 
 // Position of a CTA's share in the block list, computed once by warp 0.
@@ -75,6 +76,7 @@ struct Smem {
   float qbar[D];
   float qhat[R];
   uint64_t full[C::kSlots];
+  uint64_t empty[C::kSlots];
   Plan plan;
 };
 
@@ -90,7 +92,10 @@ static_assert(smem_fits<16, 128, true, true>() && smem_fits<32, 128, true, true>
 __device__ __forceinline__ void stg_hint(uint32_t* ptr, uint32_t v, uint64_t pol) {
   asm volatile("st.global.L2::cache_hint.u32 [%0], %1, %2;" ::"l"(ptr), "r"(v), "l"(pol) : "memory");
 }
-// Barrier 1 among the consumer warps.
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+// Barrier 1 among the consumer warps (the producer warp never joins it).
 template <int N>
 __device__ __forceinline__ void consumers_sync() {
   asm volatile("bar.sync 1, %0;" ::"n"(N) : "memory");
@@ -186,7 +191,10 @@ __global__ void __launch_bounds__(Cfg<R, GATED, KP8>::kThreads, 1) score_kernel(
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 
   if (tid == 0) {
-    for (int s = 0; s < C::kSlots; ++s) mbar_init(&S.full[s], 1);
+    for (int s = 0; s < C::kSlots; ++s) {
+      mbar_init(&S.full[s], 1);
+      mbar_init(&S.empty[s], 1);
+    }
     fence_barrier_init();
   }
   for (int i = tid; i < C::kBins; i += C::kThreads) S.hist[i] = 0u;
@@ -254,63 +262,73 @@ __global__ void __launch_bounds__(Cfg<R, GATED, KP8>::kThreads, 1) score_kernel(
 
   bool waited_ok = true;
   const unsigned char* kp = reinterpret_cast<const unsigned char*>(p.kproj);
-  const int my_blocks = pl.count > warp ? (pl.count - warp + NW - 1) / NW : 0;
 
-  // Issue cursor of this warp (lane 0): the warp's i-th block is block warp + i * NW of the share.
-  int ib = pl.b0, ih = pl.h0, ic = pl.c0;
-  SeqInfo isi = seq_info<BR>(p, ib < p.B ? ib : 0, false);
-  auto advance = [&](int k) {
-    while (k > 0 && ib < p.B) {
-      const int take = min(k, isi.blocks - ic);
-      ic += take;
-      k -= take;
-      if (ic == isi.blocks) {
-        ic = 0;
-        if (++ih == p.Hkv) {
-          ih = 0;
-          ++ib;
-          next_scored_seq<BR>(p, ib, isi);
+  if (warp >= NW) {
+    // ---------------------------------------------------------------- producers
+    // Producer lane L owns ring slot L and copies the CTA's blocks L, L + kSlots, ... into it,
+    // each once the consumer warp that read the slot's previous block has released it.
+    const int L = (warp - NW) * 32 + lane;
+    if (L < C::kSlots && pl.count > L) {
+      int b = pl.b0, h = pl.h0, c = pl.c0;
+      SeqInfo si = seq_info<BR>(p, b, false);
+      // move the walk k blocks forward
+      auto advance = [&](int k) {
+        while (k > 0 && b < p.B) {
+          const int take = min(k, si.blocks - c);
+          c += take;
+          k -= take;
+          if (c == si.blocks) {
+            c = 0;
+            if (++h == p.Hkv) {
+              h = 0;
+              ++b;
+              next_scored_seq<BR>(p, b, si);
+            }
+          }
         }
+      };
+      advance(L);
+      const int slot = L;
+      uint32_t phase = 0u;
+      for (int t = L; t < pl.count; t += C::kSlots) {
+        if (t >= C::kSlots) {
+          if (!mbar_wait_bounded(&S.empty[slot], phase)) waited_ok = false;
+          phase ^= 1u;
+        }
+        const int row0 = c * BR;
+        const int rows = min(BR, si.n - row0);
+        const int bh = b * p.Hkv + h;
+        // gate values: a whole number of 16-byte units, inside the [cap] row (cap % 4 == 0)
+        const uint32_t lg_bytes = GATED ? (uint32_t)((rows + 3) & ~3) * 4u : 0u;
+        unsigned char* dst = S.ring[slot];
+        mbar_arrive_expect_tx(&S.full[slot], (uint32_t)rows * Gm::ROW_BYTES + lg_bytes);
+        if (!p.paged) {
+          bulk_g2s(dst, kp + ((size_t)bh * p.cap + row0) * Gm::ROW_BYTES, (uint32_t)rows * Gm::ROW_BYTES,
+                   &S.full[slot]);
+        } else {
+          const int32_t* pt = p.page_table + (size_t)b * p.max_pages;
+          for (int g = row0; g < row0 + rows;) {
+            const int pr = min(64 - (g & 63), row0 + rows - g);  // rows in this page piece
+            int pg = pt[g >> 6];
+            if (pg < 0 || pg >= p.num_pages) {
+              record_error(p.err, kDevBadPage, (uint32_t)b);
+              pg = 0;
+            }
+            bulk_g2s(dst + (size_t)(g - row0) * Gm::ROW_BYTES,
+                     kp + (((size_t)pg * p.Hkv + h) * 64 + (g & 63)) * Gm::ROW_BYTES, (uint32_t)pr * Gm::ROW_BYTES,
+                     &S.full[slot]);
+            g += pr;
+          }
+        }
+        if (GATED) bulk_g2s(dst + kBlockBytes, p.log_g + (size_t)bh * p.cap + row0, lg_bytes, &S.full[slot]);
+        advance(C::kSlots);
       }
     }
-  };
-  // Copy the block under the cursor into slot `slot` (one bulk copy, or one per 64-token page
-  // piece for the paged layout, plus the block's gate values), then move the cursor to the warp's
-  // next block.
-  auto issue = [&](int slot) {
-    const int row0 = ic * BR;
-    const int rows = min(BR, isi.n - row0);
-    const int bh = ib * p.Hkv + ih;
-    // gate values: a whole number of 16-byte units, inside the [cap] row (cap % 4 == 0)
-    const uint32_t lg_bytes = GATED ? (uint32_t)((rows + 3) & ~3) * 4u : 0u;
-    unsigned char* dst = S.ring[slot];
-    mbar_arrive_expect_tx(&S.full[slot], (uint32_t)rows * Gm::ROW_BYTES + lg_bytes);
-    if (!p.paged) {
-      bulk_g2s(dst, kp + ((size_t)bh * p.cap + row0) * Gm::ROW_BYTES, (uint32_t)rows * Gm::ROW_BYTES, &S.full[slot]);
-    } else {
-      const int32_t* pt = p.page_table + (size_t)ib * p.max_pages;
-      for (int g = row0; g < row0 + rows;) {
-        const int pr = min(64 - (g & 63), row0 + rows - g);  // rows in this page piece
-        int pg = pt[g >> 6];
-        if (pg < 0 || pg >= p.num_pages) {
-          record_error(p.err, kDevBadPage, (uint32_t)ib);
-          pg = 0;
-        }
-        bulk_g2s(dst + (size_t)(g - row0) * Gm::ROW_BYTES,
-                 kp + (((size_t)pg * p.Hkv + ih) * 64 + (g & 63)) * Gm::ROW_BYTES, (uint32_t)pr * Gm::ROW_BYTES,
-                 &S.full[slot]);
-        g += pr;
-      }
-    }
-    if (GATED) bulk_g2s(dst + kBlockBytes, p.log_g + (size_t)bh * p.cap + row0, lg_bytes, &S.full[slot]);
-    advance(NW);
-  };
-  if (lane == 0) {
-    advance(warp);
-    for (int i = 0; i < min(kDepth, my_blocks); ++i) issue(warp * kDepth + i);
+    if (!waited_ok) record_error(p.err, kDevWaitTimeout, blockIdx.x);
+    return;
   }
-  __syncwarp();
 
+  // ------------------------------------------------------------------ consumer warps
   const uint64_t pol_keep = l2_evict_last();
   const int part = lane % Gm::LPR;  // this lane's 16-byte chunk of each row it loads
   const int rsub = lane / Gm::LPR;  // its row within each load instruction
@@ -382,14 +400,13 @@ __global__ void __launch_bounds__(Cfg<R, GATED, KP8>::kThreads, 1) score_kernel(
     // ---- this warp's blocks of the segment: CTA block indices j = t.. with j % NW == warp ----
     const int j0 = t + ((warp - t) % NW + NW) % NW;
     for (int j = j0; j < t + seg; j += NW) {
-      const int i = (j - warp) / NW;  // the warp's own block number
-      const int slot = warp * kDepth + i % kDepth;
-      if (!mbar_wait_bounded(&S.full[slot], (uint32_t)(i / kDepth) & 1u)) waited_ok = false;
+      const int slot = j % C::kSlots;  // the warp's blocks cycle through its kDepth slots
+      if (!mbar_wait_bounded(&S.full[slot], (uint32_t)(j / C::kSlots) & 1u)) waited_ok = false;
       const int row0 = (c + (j - t)) * BR;
       const int rows = min(BR, si.n - row0);
       const unsigned char* st = S.ring[slot];
       // The whole block into registers (8 16-byte pieces per lane) and the slot straight back to
-      // the copy engine, so the arithmetic below overlaps the copy of the warp's next blocks.
+      // its producer lane, so the arithmetic below overlaps the copy of the slot's next block.
       // Rows past a partial block's end hold older data; their results are dropped below.
       uint4 wv[Gm::NB][Gm::NI];
       float lgv[Gm::NB];
@@ -402,7 +419,7 @@ __global__ void __launch_bounds__(Cfg<R, GATED, KP8>::kThreads, 1) score_kernel(
         if constexpr (GATED) lgv[bt] = reinterpret_cast<const float*>(st + kBlockBytes)[bt * 32 + part * Gm::RPI + rsub];
       }
       __syncwarp();  // every lane has read the slot
-      if (lane == 0 && i + kDepth < my_blocks) issue(slot);
+      if (lane == 0) mbar_arrive(&S.empty[slot]);
 #pragma unroll
       for (int bt = 0; bt < Gm::NB; ++bt) {
         const int wrows = rows - bt * 32;  // rows of this 32-row batch (warp-uniform)

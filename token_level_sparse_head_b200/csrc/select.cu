@@ -84,10 +84,12 @@ struct SelSmem {
   Found found;
 };
 
-// Exclusive prefix sum over the block; *total receives the block sum.
+// Exclusive prefix sum over the block; *total receives the block sum.  Warp sums meet in shared
+// memory and every warp scans them with shuffles (at most 32 of them).
 template <int THREADS>
 __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t* wsum, uint32_t* total) {
   constexpr int kWarps = THREADS / 32;
+  static_assert(kWarps <= 32, "one warp sum per lane");
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   uint32_t x = v;
 #pragma unroll
@@ -97,15 +99,16 @@ __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t* wsum, 
   }
   if (lane == 31) wsum[warp] = x;
   __syncthreads();
-  uint32_t off = 0, tot = 0;
+  const uint32_t ws = lane < kWarps ? wsum[lane] : 0u;
+  uint32_t wi = ws;
 #pragma unroll
-  for (int w = 0; w < kWarps; ++w) {
-    const uint32_t s = wsum[w];
-    off += (w < warp) ? s : 0u;
-    tot += s;
+  for (int o = 1; o < kWarps; o <<= 1) {
+    const uint32_t y = __shfl_up_sync(0xffffffffu, wi, o);
+    if (lane >= o) wi += y;
   }
-  __syncthreads();
-  *total = tot;
+  const uint32_t off = __shfl_sync(0xffffffffu, wi - ws, warp);
+  *total = __shfl_sync(0xffffffffu, wi, kWarps - 1);
+  __syncthreads();  // wsum may be written again by the next scan
   return off + x - v;
 }
 
@@ -281,6 +284,12 @@ __global__ void __launch_bounds__(THREADS, 1) select_topk_kernel(const SelectPar
   const uint32_t above1 = S.found.above;  // keys of the head with a larger digit 1
   const uint32_t eq1 = S.found.eq;        // keys of the head with this digit 1: the candidates
   const bool fast = eq1 <= (uint32_t)kCap;
+  // One CTA per head: every thread has read the histogram (find_digit ends with a barrier), so
+  // it is cleared for the next call now, under the streaming pass; in a cluster, CTA 0 clears it
+  // once every CTA has passed the arrive below.
+  if (C == 1)
+    for (int i = tid; i < kHistBins / 4; i += kThreads)
+      reinterpret_cast<uint4*>(const_cast<uint32_t*>(ghist))[i] = make_uint4(0u, 0u, 0u, 0u);
   cluster_arrive();  // this CTA's set-up is done and it has read the global histogram
 
   bool waited_ok = true;
@@ -341,6 +350,9 @@ __global__ void __launch_bounds__(THREADS, 1) select_topk_kernel(const SelectPar
     if (lane == 0 && my_above) atomicAdd(&S.ctl.above, my_above);
     __syncthreads();
     cluster_wait();  // every CTA of the cluster is set up: CTA 0's list may now be appended to
+    if (C > 1 && rank == 0)
+      for (int i = tid; i < kHistBins / 4; i += kThreads)
+        reinterpret_cast<uint4*>(const_cast<uint32_t*>(ghist))[i] = make_uint4(0u, 0u, 0u, 0u);
 
     // ------------------------------------------------------------ gather into CTA 0
     const uint32_t mine = min(S.ctl.ccount, (uint32_t)kCap);
@@ -429,8 +441,6 @@ __global__ void __launch_bounds__(THREADS, 1) select_topk_kernel(const SelectPar
       }
     }
     cluster_sync();  // C: results are in every CTA
-    if (rank == 0)
-      for (int i = tid; i < kHistBins; i += kThreads) const_cast<uint32_t*>(ghist)[i] = 0u;  // for the next call
   } else {
     // Too many candidates for the list: drain the copies issued above, then take the slow path.
     if (lane == 0)
@@ -438,8 +448,9 @@ __global__ void __launch_bounds__(THREADS, 1) select_topk_kernel(const SelectPar
         if (!mbar_wait_bounded(&S.full[warp][j % kSlots], 0u)) waited_ok = false;
     __syncthreads();
     cluster_wait();
-    if (rank == 0)
-      for (int i = tid; i < kHistBins; i += kThreads) const_cast<uint32_t*>(ghist)[i] = 0u;
+    if (C > 1 && rank == 0)
+      for (int i = tid; i < kHistBins / 4; i += kThreads)
+        reinterpret_cast<uint4*>(const_cast<uint32_t*>(ghist))[i] = make_uint4(0u, 0u, 0u, 0u);
     if (tid == 0) S.ctl.flag = kSlow;
     __syncthreads();
   }
