@@ -416,7 +416,7 @@ def run_ours(args):
     # clocks are sampled over a window of at least a second under load: the per-step
     # distribution (each replay between two events) and then the headline block itself
     sampler = ClockSampler(smi_device_id(torch, local))
-    dist_ms = step_distribution(torch, replay, min_steps=50, min_seconds=1.0)
+    dist_ms = step_distribution(torch, replay, min_steps=50, min_seconds=args.dist_seconds)
     t = timed_block(torch, replay, args.steps, dist)
     clocks = sampler.stop()
     ms = t / args.steps * 1e3
@@ -829,6 +829,8 @@ def main():
     ap.add_argument("--no-fp8", action="store_true", help="skip the FP8 projected-cache line")
     ap.add_argument("--no-foil", action="store_true", help="skip the gather-then-attend line")
     ap.add_argument("--no-workloads", action="store_true", help="skip the other named workloads")
+    ap.add_argument("--dist-seconds", type=float, default=1.0,
+                    help="least wall time of the per-step distribution and clock window (0: 50 steps)")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--recall-report", action="store_true",
                     help="print the selection recall of every named workload instead of timing")

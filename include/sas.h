@@ -241,14 +241,18 @@ sas_status sas_gather_selected(const sas_shape* shape, const void* K, const void
  *
  * Size limit: the shape and k_max must need at most SAS_STATIC_SCRATCH_BYTES of workspace,
  * i.e. sas_decode_workspace_bytes(shape, k_max) <= SAS_STATIC_SCRATCH_BYTES.  For example
- * B=1, Hq=32, Hkv=8, d=128, r=32, 131072 tokens, k_max=4096 needs about 4.8 MiB and B=4 at
- * 65536 tokens about 11 MiB; B=16 at 131072 tokens needs 70 MiB and is rejected.  A shape
+ * B=1, Hq=32, Hkv=8, d=128, r=32, 131072 tokens, k_max=4096 needs 4,989,440 bytes (4.8 MiB) and
+ * B=4 at 65536 tokens 11,567,616 bytes (11.0 MiB); B=16 at 131072 tokens needs 79,823,616 bytes
+ * (76.1 MiB) and is rejected.  A shape
  * over the limit returns SAS_ERR_UNSUPPORTED before anything is launched, with the sizes in
  * sas_last_error_detail(); use sas_decode_step with a workspace for it.
  *
  * Setup: the first call on each device looks up the array's device address
- * (cudaGetSymbolAddress) with that device current, and caches it; make that first call before
- * any stream capture begins.  The current device selects which device's array is used.
+ * (cudaGetSymbolAddress) with that device current, and caches it with the id of the device's
+ * current CUDA context; make that first call before any stream capture begins.  If that context
+ * is later replaced (cudaDeviceReset, or the primary context torn down and created again), the
+ * next call looks the address up again, so it too should come before any capture.  The current
+ * device selects which device's array is used.
  *
  * Sharing: all calls on one device use the same array.  Calls that overlap in time on that
  * device (different streams, or different host threads, without ordering between them) race

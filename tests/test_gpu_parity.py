@@ -67,6 +67,16 @@ def test_exact_ties_take_lowest_positions(cuda_lib):
     run_small(p, dense=False)
 
 
+@pytest.mark.parametrize("n,k", [(512, 63), (512, 64), (512, 65), (512, 511), (512, 512), (512, 513),
+                                 (511, 64), (513, 64), (512, 1), (512, 0)])
+def test_selection_size_around_the_tiny_budget(cuda_lib, n, k):
+    # the budget either ranks (0 < k < n), takes every position (k >= n) or takes none (k <= 0);
+    # the tiny workload's k = 64, n = 512 and its neighbours, one head split over a cluster
+    p = make_problem(B=1, Hq=4, Hkv=1, d=64, r=16, seqlens=[n], k=[k], k_max=max(k, 1), basis="qr", seed=n + k,
+                     poison_tail=True)
+    run_small(p, dense=False)
+
+
 @pytest.mark.parametrize("B,Hkv,N", [(1, 2, 20000), (40, 2, 10000)])
 def test_candidate_overflow_takes_the_slow_path(cuda_lib, B, Hkv, N):
     # more than 4096 keys share the k-th key's first digit (half the positions tie), so the

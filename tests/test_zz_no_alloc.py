@@ -60,7 +60,8 @@ def test_static_scratch_matches_workspace_call(cuda_lib, case):
 
 
 def test_static_scratch_rejects_oversized_shape():
-    """B=16 at 131072 tokens needs 67 MiB of scratch: rejected on the host, nothing launched."""
+    """B=16 at 131072 tokens needs 79,823,616 bytes (76.1 MiB) of scratch: rejected on the host,
+    nothing launched."""
     lib.load()
     shape = lib.Shape(16, 32, 8, 128, 32, 131072)
     need = lib.sas_decode_workspace_bytes(shape, 4096)

@@ -8,6 +8,8 @@
 #include <mutex>
 #include <unordered_map>
 
+#include <cuda.h>  // driver types only (CUcontext, CUresult); no driver library is linked
+
 #include "sas.h"
 #include "sas_kernels.h"
 
@@ -531,10 +533,41 @@ namespace {
 
 constexpr int kMaxScratchDevices = 64;
 std::mutex g_scratch_mutex;
-void* g_scratch_ptr[kMaxScratchDevices] = {};
+// Per device: the address of g_static_scratch and the id of the CUDA context it was looked up
+// in.  A device reset (or any teardown of the primary context) loads the library's device image
+// again, possibly elsewhere, so the address is looked up again whenever the context changes.
+struct ScratchEntry {
+  void* ptr;
+  unsigned long long ctx_id;
+};
+ScratchEntry g_scratch[kMaxScratchDevices] = {};
 
-// Address of this device's copy of g_static_scratch.  The first call on a device looks it up
-// with that device current; later calls reuse the cached pointer.
+using PfnCtxGetCurrent = CUresult (*)(CUcontext*);
+using PfnCtxGetId = CUresult (*)(CUcontext, unsigned long long*);
+
+// Id of the context current on this thread (driver entry points resolved through the runtime,
+// so the library links no driver library); 0 when there is none yet.
+cudaError_t current_context_id(unsigned long long* id) {
+  static PfnCtxGetCurrent get_current = nullptr;
+  static PfnCtxGetId get_id = nullptr;
+  if (get_current == nullptr || get_id == nullptr) {
+    cudaDriverEntryPointQueryResult q1, q2;
+    cudaError_t e = cudaGetDriverEntryPoint("cuCtxGetCurrent", reinterpret_cast<void**>(&get_current),
+                                            cudaEnableDefault, &q1);
+    if (e == cudaSuccess)
+      e = cudaGetDriverEntryPoint("cuCtxGetId", reinterpret_cast<void**>(&get_id), cudaEnableDefault, &q2);
+    if (e != cudaSuccess) return e;
+    if (q1 != cudaDriverEntryPointSuccess || q2 != cudaDriverEntryPointSuccess) return cudaErrorNotSupported;
+  }
+  CUcontext ctx = nullptr;
+  if (get_current(&ctx) != CUDA_SUCCESS) return cudaErrorUnknown;
+  *id = 0;
+  if (ctx != nullptr && get_id(ctx, id) != CUDA_SUCCESS) return cudaErrorUnknown;
+  return cudaSuccess;
+}
+
+// Address of this device's copy of g_static_scratch, looked up with the device current the first
+// time and again after the device's context has been replaced; cached otherwise.
 sas_status static_scratch_ptr(void** out) {
   int dev = -1;
   cudaError_t e = cudaGetDevice(&dev);
@@ -543,13 +576,22 @@ sas_status static_scratch_ptr(void** out) {
     return fail(SAS_ERR_UNSUPPORTED, "device ordinal %d: the static scratch supports devices 0..%d", dev,
                 kMaxScratchDevices - 1);
   std::lock_guard<std::mutex> lock(g_scratch_mutex);
-  if (g_scratch_ptr[dev] == nullptr) {
+  unsigned long long id = 0;
+  e = current_context_id(&id);
+  if (e != cudaSuccess) return cuda_fail(e, "querying the current context");
+  ScratchEntry& ent = g_scratch[dev];
+  if (ent.ptr == nullptr || id == 0 || id != ent.ctx_id) {
     void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_static_scratch);
+    e = cudaGetSymbolAddress(&p, g_static_scratch);  // makes the device's primary context current
     if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress of the static scratch");
-    g_scratch_ptr[dev] = p;
+    if (id == 0) {
+      e = current_context_id(&id);
+      if (e != cudaSuccess) return cuda_fail(e, "querying the current context");
+    }
+    ent.ptr = p;
+    ent.ctx_id = id;
   }
-  *out = g_scratch_ptr[dev];
+  *out = ent.ptr;
   return SAS_OK;
 }
 
