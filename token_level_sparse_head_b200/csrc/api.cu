@@ -15,29 +15,75 @@
 
 namespace sas {
 
+namespace {
+using PfnCtxGetCurrent = CUresult (*)(CUcontext*);
+using PfnCtxGetId = CUresult (*)(CUcontext, unsigned long long*);
+struct CtxQuery {
+  PfnCtxGetCurrent get_current = nullptr;
+  PfnCtxGetId get_id = nullptr;
+  cudaError_t status = cudaErrorNotSupported;
+  CtxQuery() {
+    cudaDriverEntryPointQueryResult q1, q2;
+    cudaError_t e = cudaGetDriverEntryPoint("cuCtxGetCurrent", reinterpret_cast<void**>(&get_current),
+                                            cudaEnableDefault, &q1);
+    if (e == cudaSuccess)
+      e = cudaGetDriverEntryPoint("cuCtxGetId", reinterpret_cast<void**>(&get_id), cudaEnableDefault, &q2);
+    if (e != cudaSuccess) status = e;
+    else if (q1 != cudaDriverEntryPointSuccess || q2 != cudaDriverEntryPointSuccess) status = cudaErrorNotSupported;
+    else status = cudaSuccess;
+  }
+};
+}  // namespace
+
+// Id of the context current on this thread (driver entry points resolved once, thread-safely,
+// through the runtime, so the library links no driver library); 0 when there is none yet.
+cudaError_t current_context_id(unsigned long long* id) {
+  static const CtxQuery q;
+  if (q.status != cudaSuccess) return q.status;
+  CUcontext ctx = nullptr;
+  if (q.get_current(&ctx) != CUDA_SUCCESS) return cudaErrorUnknown;
+  *id = 0;
+  if (ctx != nullptr && q.get_id(ctx, id) != CUDA_SUCCESS) return cudaErrorUnknown;
+  return cudaSuccess;
+}
+
+// Kernel attributes belong to the context: the limit set for a kernel is remembered per device
+// together with the id of the context it was set in, and set again in a new context.
 cudaError_t prepare_kernel(const void* kern, int smem_bytes, bool nonportable_cluster) {
   constexpr int kDevices = 64;
+  struct Allowed {
+    int bytes;
+    unsigned long long ctx_id;
+  };
   static std::mutex mu;
-  static std::unordered_map<const void*, std::array<int, kDevices>> allowed;  // bytes allowed, per device
+  static std::unordered_map<const void*, std::array<Allowed, kDevices>> allowed;  // per device
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
+  unsigned long long ctx_id = 0;
+  e = current_context_id(&ctx_id);
+  if (e != cudaSuccess) return e;
   std::lock_guard<std::mutex> lock(mu);
-  int* lim = nullptr;
+  Allowed* lim = nullptr;
   if (dev >= 0 && dev < kDevices) {
     auto it = allowed.find(kern);
     if (it == allowed.end()) {
-      std::array<int, kDevices> none;
-      none.fill(-1);
+      std::array<Allowed, kDevices> none;
+      none.fill(Allowed{-1, 0});
       it = allowed.emplace(kern, none).first;
     }
     lim = &it->second[dev];
-    if (*lim >= smem_bytes) return cudaSuccess;
+    if (ctx_id != 0 && lim->ctx_id == ctx_id && lim->bytes >= smem_bytes) return cudaSuccess;
   }
   e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes);
   if (e == cudaSuccess && nonportable_cluster)
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-  if (e == cudaSuccess && lim != nullptr) *lim = smem_bytes;
+  if (e == cudaSuccess && lim != nullptr) {
+    if (ctx_id == 0) current_context_id(&ctx_id);  // the call above made the primary context current
+    if (lim->ctx_id != ctx_id) lim->bytes = -1;
+    if (smem_bytes > lim->bytes) lim->bytes = smem_bytes;
+    lim->ctx_id = ctx_id;
+  }
   return e;
 }
 
@@ -542,30 +588,6 @@ struct ScratchEntry {
 };
 ScratchEntry g_scratch[kMaxScratchDevices] = {};
 
-using PfnCtxGetCurrent = CUresult (*)(CUcontext*);
-using PfnCtxGetId = CUresult (*)(CUcontext, unsigned long long*);
-
-// Id of the context current on this thread (driver entry points resolved through the runtime,
-// so the library links no driver library); 0 when there is none yet.
-cudaError_t current_context_id(unsigned long long* id) {
-  static PfnCtxGetCurrent get_current = nullptr;
-  static PfnCtxGetId get_id = nullptr;
-  if (get_current == nullptr || get_id == nullptr) {
-    cudaDriverEntryPointQueryResult q1, q2;
-    cudaError_t e = cudaGetDriverEntryPoint("cuCtxGetCurrent", reinterpret_cast<void**>(&get_current),
-                                            cudaEnableDefault, &q1);
-    if (e == cudaSuccess)
-      e = cudaGetDriverEntryPoint("cuCtxGetId", reinterpret_cast<void**>(&get_id), cudaEnableDefault, &q2);
-    if (e != cudaSuccess) return e;
-    if (q1 != cudaDriverEntryPointSuccess || q2 != cudaDriverEntryPointSuccess) return cudaErrorNotSupported;
-  }
-  CUcontext ctx = nullptr;
-  if (get_current(&ctx) != CUDA_SUCCESS) return cudaErrorUnknown;
-  *id = 0;
-  if (ctx != nullptr && get_id(ctx, id) != CUDA_SUCCESS) return cudaErrorUnknown;
-  return cudaSuccess;
-}
-
 // Address of this device's copy of g_static_scratch, looked up with the device current the first
 // time and again after the device's context has been replaced; cached otherwise.
 sas_status static_scratch_ptr(void** out) {
@@ -577,7 +599,7 @@ sas_status static_scratch_ptr(void** out) {
                 kMaxScratchDevices - 1);
   std::lock_guard<std::mutex> lock(g_scratch_mutex);
   unsigned long long id = 0;
-  e = current_context_id(&id);
+  e = sas::current_context_id(&id);
   if (e != cudaSuccess) return cuda_fail(e, "querying the current context");
   ScratchEntry& ent = g_scratch[dev];
   if (ent.ptr == nullptr || id == 0 || id != ent.ctx_id) {
@@ -585,7 +607,7 @@ sas_status static_scratch_ptr(void** out) {
     e = cudaGetSymbolAddress(&p, g_static_scratch);  // makes the device's primary context current
     if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress of the static scratch");
     if (id == 0) {
-      e = current_context_id(&id);
+      e = sas::current_context_id(&id);
       if (e != cudaSuccess) return cuda_fail(e, "querying the current context");
     }
     ent.ptr = p;

@@ -44,9 +44,11 @@ __device__ __forceinline__ uint32_t float_key(float f) {
 __device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
 
 // Size of the selection, min(k_b, N_b) clamped at 0, and whether it needs ranking (neither
-// empty nor every position).  The ranking test is written on the inputs rather than as
-// (k_eff == 0 || k_eff == n): with nvcc 12.9 for sm_100a, an equality test between
-// max(0, min(k, n)) and n was observed to evaluate true for k = 64, n = 512.
+// empty nor every position).  The ranking test is written on the inputs (0 < k < n), which
+// means the same as (k_eff == 0 || k_eff == n) negated.  A build that used the latter form once
+// returned every position at k = 64, n = 512; no race or uninitialised value was found in that
+// code and the cause was not established.  The selection's parity tests cover n = 512 with k
+// around 64 and around n.
 struct SeqSelection {
   int k_eff;
   bool ranked;
