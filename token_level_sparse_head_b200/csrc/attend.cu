@@ -379,40 +379,63 @@ __global__ void __launch_bounds__(kThreads) attend_kernel(const AttendParams p) 
   // The merge buffer aliases the ring: every warp must be done with its stages (all issued
   // copies have been waited for) before any warp writes its totals.
   __syncthreads();
-  // merge[warp][g][0..D-1] = acc, [D] = m, [D+1] = l
-  float* mw = merge + (size_t)warp * GT * (D + 2);
+  // merge: acc [warp][g][D] (16-byte rows of lanes), then (m, l) [warp][g][2]
+  float* mml = merge + kWarps * GT * D;
+  float* mw = merge + (size_t)warp * GT * D;
 #pragma unroll
-  for (int g = 0; g < GT; ++g)
-#pragma unroll
-    for (int c = 0; c < Gm::CPL; ++c) mw[g * (D + 2) + lane * Gm::CPL + c] = acc[g][c];
+  for (int g = 0; g < GT; ++g) {
+    if constexpr (Gm::CPL == 4) {
+      *reinterpret_cast<float4*>(mw + g * D + lane * 4) = make_float4(acc[g][0], acc[g][1], acc[g][2], acc[g][3]);
+    } else {
+      *reinterpret_cast<float2*>(mw + g * D + lane * 2) = make_float2(acc[g][0], acc[g][1]);
+    }
+  }
   if (owner && my_tl == 0) {
-    mw[my_g * (D + 2) + D] = m_run;
-    mw[my_g * (D + 2) + D + 1] = l_tot;
+    mml[(warp * GT + my_g) * 2] = m_run;
+    mml[(warp * GT + my_g) * 2 + 1] = l_tot;
   }
   __syncthreads();
 
   // ---- CTA partial for this split: acc [GT][D] and (m, l) [GT][2] ----
+  // Per head: M = max over the warps of m, weights f_w = exp(m_w - M) (0 for an empty warp),
+  // L = sum f_w l_w; then acc = sum f_w acc_w, four channels per thread and step.
   const size_t nheads = (size_t)p.B * p.Hkv * p.ngz;
   float* pacc = p.partials + ((size_t)bhz * p.splits + split) * GT * D;
   float* pml = p.partials + nheads * p.splits * GT * D + ((size_t)bhz * p.splits + split) * GT * 2;
-  for (int e = tid; e < GT * (D + 2); e += kThreads) {
-    const int g = e / (D + 2), c = e % (D + 2);
+  float* cw = pbuf_all;   // [kWarps][GT] weights, then [GT] M (the tile buffers are idle now)
+  if (tid < GT) {
+    const int g = tid;
     float M = -INFINITY;
 #pragma unroll
-    for (int w = 0; w < kWarps; ++w) M = fmaxf(M, merge[(w * GT + g) * (D + 2) + D]);
-    float val = 0.f;
-    if (c == D) {
-      val = M;
-    } else if (M != -INFINITY) {
+    for (int w = 0; w < kWarps; ++w) M = fmaxf(M, mml[(w * GT + g) * 2]);
+    float Lc = 0.f;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) {
+      const float mwv = mml[(w * GT + g) * 2];
+      const float f = (M == -INFINITY || mwv == -INFINITY) ? 0.f : __expf(mwv - M);
+      cw[w * GT + g] = f;
+      Lc += f * mml[(w * GT + g) * 2 + 1];
+    }
+    cw[kWarps * GT + g] = M;
+    pml[g * 2] = M;
+    pml[g * 2 + 1] = Lc;
+  }
+  __syncthreads();
+  for (int e = tid; e < GT * D / 4; e += kThreads) {
+    const int g = (e * 4) / D;
+    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (cw[kWarps * GT + g] != -INFINITY) {
 #pragma unroll
       for (int w = 0; w < kWarps; ++w) {
-        const float mwv = merge[(w * GT + g) * (D + 2) + D];
-        const float f = (mwv == -INFINITY) ? 0.f : __expf(mwv - M);
-        val += f * merge[(w * GT + g) * (D + 2) + c];
+        const float f = cw[w * GT + g];
+        const float4 a = *reinterpret_cast<const float4*>(merge + (size_t)w * GT * D + e * 4);
+        v.x += f * a.x;
+        v.y += f * a.y;
+        v.z += f * a.z;
+        v.w += f * a.w;
       }
     }
-    if (c < D) pacc[g * D + c] = val;
-    else pml[g * 2 + (c - D)] = val;
+    *reinterpret_cast<float4*>(pacc + e * 4) = v;
   }
   __threadfence();
   __syncthreads();
@@ -454,19 +477,26 @@ __global__ void __launch_bounds__(kThreads) attend_kernel(const AttendParams p) 
   for (int i = 0; i < OPL; ++i) racc[i] = 0.f;
   int s = warp;
   if constexpr (OPL % 4 == 0) {
-    for (; s + kWarps < p.splits; s += 2 * kWarps) {
-      const float4* a = reinterpret_cast<const float4*>(bacc + (size_t)s * GT * D + e0);
-      const float4* bb = reinterpret_cast<const float4*>(bacc + (size_t)(s + kWarps) * GT * D + e0);
-      float4 va[OPL / 4], vb[OPL / 4];
+    // four splits per step: their 16-byte loads are all in flight before the sums
+    constexpr int kU = 4;
+    for (; s + (kU - 1) * kWarps < p.splits; s += kU * kWarps) {
+      float4 va[kU][OPL / 4];
 #pragma unroll
-      for (int i = 0; i < OPL / 4; ++i) { va[i] = __ldcg(a + i); vb[i] = __ldcg(bb + i); }
-      const float wa = wts[s * GT + gl], wb = wts[(s + kWarps) * GT + gl];
+      for (int u = 0; u < kU; ++u) {
+        const float4* a = reinterpret_cast<const float4*>(bacc + (size_t)(s + u * kWarps) * GT * D + e0);
 #pragma unroll
-      for (int i = 0; i < OPL / 4; ++i) {
-        racc[4 * i + 0] += wa * va[i].x + wb * vb[i].x;
-        racc[4 * i + 1] += wa * va[i].y + wb * vb[i].y;
-        racc[4 * i + 2] += wa * va[i].z + wb * vb[i].z;
-        racc[4 * i + 3] += wa * va[i].w + wb * vb[i].w;
+        for (int i = 0; i < OPL / 4; ++i) va[u][i] = __ldcg(a + i);
+      }
+#pragma unroll
+      for (int u = 0; u < kU; ++u) {
+        const float wa = wts[(s + u * kWarps) * GT + gl];
+#pragma unroll
+        for (int i = 0; i < OPL / 4; ++i) {
+          racc[4 * i + 0] += wa * va[u][i].x;
+          racc[4 * i + 1] += wa * va[u][i].y;
+          racc[4 * i + 2] += wa * va[u][i].z;
+          racc[4 * i + 3] += wa * va[u][i].w;
+        }
       }
     }
   }
