@@ -241,8 +241,8 @@ sas_status sas_gather_selected(const sas_shape* shape, const void* K, const void
  *
  * Size limit: the shape and k_max must need at most SAS_STATIC_SCRATCH_BYTES of workspace,
  * i.e. sas_decode_workspace_bytes(shape, k_max) <= SAS_STATIC_SCRATCH_BYTES.  For example
- * B=1, Hq=32, Hkv=8, d=128, r=32, 131072 tokens, k_max=4096 needs 4,989,440 bytes (4.8 MiB) and
- * B=4 at 65536 tokens 11,567,616 bytes (11.0 MiB); B=16 at 131072 tokens needs 79,823,616 bytes
+ * B=1, Hq=32, Hkv=8, d=128, r=32, 131072 tokens, k_max=4096 needs 4,989,184 bytes (4.8 MiB) and
+ * B=4 at 65536 tokens 11,567,360 bytes (11.0 MiB); B=16 at 131072 tokens needs 79,823,104 bytes
  * (76.1 MiB) and is rejected.  A shape
  * over the limit returns SAS_ERR_UNSUPPORTED before anything is launched, with the sizes in
  * sas_last_error_detail(); use sas_decode_step with a workspace for it.
@@ -257,8 +257,8 @@ sas_status sas_gather_selected(const sas_shape* shape, const void* K, const void
  * Sharing: all calls on one device use the same array.  Calls that overlap in time on that
  * device (different streams, or different host threads, without ordering between them) race
  * on it and give wrong results; order them on one stream.  Each call first clears, on
- * `stream`, the part of the array that must start at zero (the device error word, the
- * per-head histograms and the split counters); the rest is written before it is read.
+ * `stream`, the part of the array that must start at zero (the device error word and the
+ * per-head histograms); the rest is written before it is read.
  *
  * Device-side checks still run, but their error word lives in the shared array, is cleared by
  * the next call and cannot be read with sas_check_workspace: callers that need the device

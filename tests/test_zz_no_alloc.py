@@ -60,7 +60,7 @@ def test_static_scratch_matches_workspace_call(cuda_lib, case):
 
 
 def test_static_scratch_rejects_oversized_shape():
-    """B=16 at 131072 tokens needs 79,823,616 bytes (76.1 MiB) of scratch: rejected on the host,
+    """B=16 at 131072 tokens needs 79,823,104 bytes (76.1 MiB) of scratch: rejected on the host,
     nothing launched."""
     lib.load()
     shape = lib.Shape(16, 32, 8, 128, 32, 131072)

@@ -190,12 +190,12 @@ sas::AttendParams attend_plan(const sas_shape* s, int count_max, bool dense) {
   return a;
 }
 
-// Workspace: [0,256) error word | key histograms | split counters | attention partials | score keys.
-// The histograms and counters sit at fixed offsets: they must stay zero between calls (the
-// kernels clear them after use), whatever other calls (dense decode, other budgets) share the
-// workspace; partials and keys are rewritten by every call.
+// Workspace: [0,256) error word | key histograms | attention partials | score keys.
+// The histograms sit at a fixed offset: they must stay zero between calls (the selection clears
+// them after use), whatever other calls (dense decode, other budgets) share the workspace;
+// partials and keys are rewritten by every call.
 struct WsLayout {
-  size_t hist, counters, partials, keys, total;
+  size_t hist, partials, keys, total;
 };
 
 WsLayout ws_layout(const sas::AttendParams& a, bool with_keys) {
@@ -203,8 +203,6 @@ WsLayout ws_layout(const sas::AttendParams& a, bool with_keys) {
   size_t o = kErrBytes;
   w.hist = o;
   o += (size_t)a.B * a.Hkv * sas::kHistBins * 4;
-  w.counters = o;
-  o += ((size_t)a.B * a.Hkv * a.ngz * 4 + 255) & ~(size_t)255;
   w.partials = o;
   o += (sas::attend_workspace_floats(a) * 4 + 255) & ~(size_t)255;
   w.keys = o;
@@ -219,7 +217,6 @@ void bind_workspace(sas::AttendParams& a, void* ws) {
   unsigned char* w = static_cast<unsigned char*>(ws);
   const WsLayout L = ws_layout(a, false);
   a.err = reinterpret_cast<uint32_t*>(w);
-  a.counters = reinterpret_cast<uint32_t*>(w + L.counters);
   a.partials = reinterpret_cast<float*>(w + L.partials);
 }
 
@@ -648,9 +645,9 @@ sas_status sas_decode_step_static_scratch(const sas_shape* shape, const void* q,
   void* ws = nullptr;
   SAS_TRY(static_scratch_ptr(&ws));
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  // The error word, the per-head histograms and the split counters must start at zero; a
-  // previous call may have been cut short, so every call clears them.  The score keys and
-  // the attention partials that follow are written before they are read.
+  // The error word and the per-head histograms must start at zero; a previous call may have
+  // been cut short, so every call clears them.  The score keys and the attention partials that
+  // follow are written before they are read.
   const WsLayout L = ws_layout(attend_plan(shape, k_max, false), true);
   const cudaError_t e = cudaMemsetAsync(ws, 0, L.partials, st);
   if (e != cudaSuccess) return cuda_fail(e, "clearing the static scratch");

@@ -12,10 +12,11 @@
 // gt query heads of h; its 4 warps take 8-token tiles of the slice in turn, each warp with its
 // own ring of stages and its own online-softmax state (running max m, sum l, accumulator), in
 // fp32.  Logits z = sigma q.K_i (+ lambda log g_i, SAS page section 2.1).  The warps merge in
-// shared memory, the CTA writes one partial (m, l, acc) per query head to the workspace, and
-// the last CTA of each (b, h, head group) to finish merges all splits in split order
-// (deterministic) and writes the output.  The dense variant (idx = 0..N_b-1) is the full-KV
-// baseline.
+// shared memory and the CTA writes one partial (m, l, acc) per query head to the workspace; a
+// second kernel, one CTA per (b, h, head group), merges the splits in split order
+// (deterministic) and writes the output.  The split CTAs wait on no counter or fence, so each
+// frees its SM slot as soon as its partial is written.  The dense variant (idx = 0..N_b-1) is
+// the full-KV baseline.
 #include "sas_device.cuh"
 #include "sas_kernels.h"
 
@@ -52,7 +53,7 @@ struct Geo {
 };
 
 struct Smem {
-  int off_rows, off_lg, off_ring, off_pbuf, off_sbuf, off_merge, off_bars, off_w, off_flag, total;
+  int off_rows, off_lg, off_ring, off_pbuf, off_sbuf, off_merge, off_bars, total;
 };
 
 template <int D, int GT>
@@ -73,8 +74,6 @@ __host__ __device__ inline Smem smem_layout(int split_len, int splits) {
   s.off_sbuf = o;  o += kWarps * GT * 4;
   o = (o + 7) & ~7;
   s.off_bars = o;  o += kWarps * kStages * 8;
-  s.off_w = o;     o += splits * GT * 4 + GT * 8;
-  s.off_flag = o;  o += 16;
   s.total = o;
   return s;
 }
@@ -91,8 +90,6 @@ __global__ void __launch_bounds__(kThreads) attend_kernel(const AttendParams p) 
   float* sbuf_all = reinterpret_cast<float*>(smem + L.off_sbuf);
   float* merge = reinterpret_cast<float*>(smem + L.off_merge);
   uint64_t* bars_all = reinterpret_cast<uint64_t*>(smem + L.off_bars);
-  float* wts = reinterpret_cast<float*>(smem + L.off_w);
-  int* flag = reinterpret_cast<int*>(smem + L.off_flag);
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int split = blockIdx.x;
@@ -437,19 +434,63 @@ __global__ void __launch_bounds__(kThreads) attend_kernel(const AttendParams p) 
     }
     *reinterpret_cast<float4*>(pacc + e * 4) = v;
   }
-  __threadfence();
-  __syncthreads();
-  if (tid == 0) {
-    const uint32_t prev = atomicAdd(&p.counters[bhz], 1u);
-    flag[0] = (prev == (uint32_t)(p.splits - 1)) ? 1 : 0;
-  }
-  __syncthreads();
-  if (flag[0] == 0) return;
+}
 
-  // ---- last CTA: merge the splits (fixed order: deterministic) ----
-  __threadfence();
+
+
+// Merge of each head group's split partials, in split order (deterministic), and the output.
+// Launched after the split kernel on the same stream with programmatic dependent launch: its
+// wait returns once every split CTA has finished and its partial is visible.
+template <int D, int GT>
+__host__ __device__ inline int combine_smem_floats(int splits) {
+  return ((splits * GT + GT + 3) & ~3) + kWarps * GT * D;
+}
+
+template <int D, int GT>
+__global__ void __launch_bounds__(kThreads) combine_kernel(const AttendParams p) {
+  extern __shared__ __align__(16) float csm[];
+  float* wts = csm;                                          // [splits][GT] weights, [GT] 1/L
+  float* red = csm + ((p.splits * GT + GT + 3) & ~3);       // [kWarps][GT * D] warp sums
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int bhz = blockIdx.x;
+  const int bh = bhz / p.ngz, gz = bhz % p.ngz;
+  const int b = bh / p.Hkv, h = bh % p.Hkv;
+  const size_t nheads = (size_t)p.B * p.Hkv * p.ngz;
+  pdl_wait();
+  pdl_trigger();
   const float* bacc = p.partials + (size_t)bhz * p.splits * GT * D;
   const float* bml = p.partials + nheads * p.splits * GT * D + (size_t)bhz * p.splits * GT * 2;
+
+  // Warp w sums splits w, w + 4, ... in order, kU splits per step with all their loads in flight;
+  // lane owns OPL consecutive outputs (one head).  The first step's loads are issued before the
+  // weights are computed, so the two reads of the partials overlap.
+  constexpr int OPL = GT * D / 32;
+  constexpr int VW = (OPL % 4 == 0) ? 4 : 2;   // floats per load
+  constexpr int kU = 4;
+  const int e0 = lane * OPL;
+  const int gl = e0 / D;
+  float va[kU][OPL];
+  auto load_step = [&](int s0) {
+#pragma unroll
+    for (int u = 0; u < kU; ++u) {
+      const int s = s0 + u * kWarps;
+      if (s < p.splits) {
+        const float* a = bacc + (size_t)s * GT * D + e0;
+#pragma unroll
+        for (int i = 0; i < OPL; i += VW) {
+          if constexpr (VW == 4) {
+            const float4 x = __ldcg(reinterpret_cast<const float4*>(a + i));
+            va[u][i] = x.x; va[u][i + 1] = x.y; va[u][i + 2] = x.z; va[u][i + 3] = x.w;
+          } else {
+            const float2 x = __ldcg(reinterpret_cast<const float2*>(a + i));
+            va[u][i] = x.x; va[u][i + 1] = x.y;
+          }
+        }
+      }
+    }
+  };
+  load_step(warp);
+
   if (warp < GT) {
     const int g = warp;
     float M = -INFINITY;
@@ -468,48 +509,30 @@ __global__ void __launch_bounds__(kThreads) attend_kernel(const AttendParams p) 
     if (lane == 0) wts[p.splits * GT + g] = (Lsum > 0.f) ? 1.f / Lsum : 0.f;
   }
   __syncthreads();
-  // Warp w sums splits w, w+4, ...; lane owns OPL consecutive outputs (one head).
-  constexpr int OPL = GT * D / 32;
-  const int e0 = lane * OPL;
-  const int gl = e0 / D;
+
   float racc[OPL];
 #pragma unroll
   for (int i = 0; i < OPL; ++i) racc[i] = 0.f;
-  int s = warp;
-  if constexpr (OPL % 4 == 0) {
-    // four splits per step: their 16-byte loads are all in flight before the sums
-    constexpr int kU = 4;
-    for (; s + (kU - 1) * kWarps < p.splits; s += kU * kWarps) {
-      float4 va[kU][OPL / 4];
+  for (int s0 = warp; s0 < p.splits; s0 += kU * kWarps) {
+    if (s0 != warp) load_step(s0);
 #pragma unroll
-      for (int u = 0; u < kU; ++u) {
-        const float4* a = reinterpret_cast<const float4*>(bacc + (size_t)(s + u * kWarps) * GT * D + e0);
+    for (int u = 0; u < kU; ++u) {
+      const int s = s0 + u * kWarps;
+      if (s < p.splits) {
+        const float wa = wts[s * GT + gl];
 #pragma unroll
-        for (int i = 0; i < OPL / 4; ++i) va[u][i] = __ldcg(a + i);
-      }
-#pragma unroll
-      for (int u = 0; u < kU; ++u) {
-        const float wa = wts[(s + u * kWarps) * GT + gl];
-#pragma unroll
-        for (int i = 0; i < OPL / 4; ++i) {
-          racc[4 * i + 0] += wa * va[u][i].x;
-          racc[4 * i + 1] += wa * va[u][i].y;
-          racc[4 * i + 2] += wa * va[u][i].z;
-          racc[4 * i + 3] += wa * va[u][i].w;
-        }
+        for (int i = 0; i < OPL; ++i) racc[i] += wa * va[u][i];
       }
     }
   }
-  for (; s < p.splits; s += kWarps) {
-    const float* a = bacc + (size_t)s * GT * D + e0;
-    const float wa = wts[s * GT + gl];
 #pragma unroll
-    for (int i = 0; i < OPL; ++i) racc[i] += wa * __ldcg(a + i);
+  for (int i = 0; i < OPL; i += VW) {
+    if constexpr (VW == 4) {
+      *reinterpret_cast<float4*>(red + warp * GT * D + e0 + i) = make_float4(racc[i], racc[i + 1], racc[i + 2], racc[i + 3]);
+    } else {
+      *reinterpret_cast<float2*>(red + warp * GT * D + e0 + i) = make_float2(racc[i], racc[i + 1]);
+    }
   }
-  float* red = merge;  // reuse: [kWarps][GT * D]
-  __syncthreads();
-#pragma unroll
-  for (int i = 0; i < OPL; ++i) red[warp * GT * D + e0 + i] = racc[i];
   __syncthreads();
   for (int e = tid; e < GT * D; e += kThreads) {
     const int g = e / D, c = e % D;
@@ -519,7 +542,6 @@ __global__ void __launch_bounds__(kThreads) attend_kernel(const AttendParams p) 
     const int hq = h * p.G + gz * GT + g;
     p.out[((size_t)b * p.Hq + hq) * D + c] = v * wts[p.splits * GT + g];
   }
-  if (tid == 0) p.counters[bhz] = 0u;
 }
 
 // Shared-memory bytes of a plan.
@@ -565,7 +587,13 @@ cudaError_t launch_t(const AttendParams& p0, cudaStream_t stream) {
   cudaError_t e = prepare_kernel((const void*)kern, p.smem_bytes);
   if (e != cudaSuccess) return e;
   dim3 grid((unsigned)p.splits, (unsigned)(p.B * p.Hkv), (unsigned)p.ngz);
-  return launch_pdl(kern, grid, dim3(kThreads), (size_t)p.smem_bytes, stream, p);
+  e = launch_pdl(kern, grid, dim3(kThreads), (size_t)p.smem_bytes, stream, p);
+  if (e != cudaSuccess) return e;
+  auto ck = combine_kernel<D, GT>;
+  const int csm = combine_smem_floats<D, GT>(p.splits) * 4;
+  e = prepare_kernel((const void*)ck, csm);
+  if (e != cudaSuccess) return e;
+  return launch_pdl(ck, dim3((unsigned)(p.B * p.Hkv * p.ngz)), dim3(kThreads), (size_t)csm, stream, p);
 }
 
 template <int D, int GT>

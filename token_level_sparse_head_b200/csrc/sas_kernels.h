@@ -100,7 +100,6 @@ struct AttendParams {
   const float* log_g;          // [B][Hkv][cap] or null
   float* out;                  // [B][Hq][d]
   float* partials;             // workspace: [B*Hkv*ngz][splits][gt][d + 2]
-  uint32_t* counters;          // workspace: [B*Hkv*ngz]
   uint32_t* err;
   int B, Hq, Hkv, G, d, cap, max_pages, num_pages, paged, k_max;
   float sigma, lam;
