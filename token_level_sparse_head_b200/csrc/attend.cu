@@ -56,13 +56,14 @@ struct Smem {
   int off_rows, off_lg, off_ring, off_pbuf, off_sbuf, off_merge, off_bars, total;
 };
 
+// The gate terms' buffer (lg) is laid out only for the gated variant.
 template <int D, int GT>
-__host__ __device__ inline Smem smem_layout(int split_len, int splits) {
+__host__ __device__ inline Smem smem_layout(int split_len, int splits, bool with_lg) {
   using Gm = Geo<D, GT>;
   Smem s;
   int o = 0;
   s.off_rows = o;  o += split_len * 4;
-  s.off_lg = o;    o += split_len * 4;
+  s.off_lg = o;    o += with_lg ? split_len * 4 : 0;
   o = (o + 127) & ~127;
   s.off_ring = o;
   // After the tile loop the ring is idle: the warp merge (and the split merge) reuse it.
@@ -82,7 +83,7 @@ template <int D, int GT, bool GATED, bool PAGED, bool DENSE>
 __global__ void __launch_bounds__(kThreads) attend_kernel(const AttendParams p) {
   using Gm = Geo<D, GT>;
   extern __shared__ __align__(128) unsigned char smem[];
-  const Smem L = smem_layout<D, GT>(p.split_len, p.splits);
+  const Smem L = smem_layout<D, GT>(p.split_len, p.splits, GATED);
   uint32_t* rows_s = reinterpret_cast<uint32_t*>(smem + L.off_rows);
   float* lg_s = reinterpret_cast<float*>(smem + L.off_lg);
   unsigned char* ring = smem + L.off_ring;
@@ -546,23 +547,24 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(const AttendParams p)
 
 // Shared-memory bytes of a plan.
 template <int D, int GT>
-int plan_smem(int split_len, int splits) {
-  return smem_layout<D, GT>(split_len, splits).total;
+int plan_smem(int split_len, int splits, bool with_lg = true) {
+  return smem_layout<D, GT>(split_len, splits, with_lg).total;
 }
 
 template <int D, int GT, bool GATED, bool PAGED, bool DENSE>
 cudaError_t launch_t(const AttendParams& p0, cudaStream_t stream) {
   auto kern = attend_kernel<D, GT, GATED, PAGED, DENSE>;
   AttendParams p = p0;
-  if (!DENSE && p.sms > 0) {
+  if (p.sms > 0) {
     // Re-split for whole waves: CTAs resident per SM at the largest slice, then the split count
     // in [s_lo, max_splits] whose grid fills its last wave best (the most splits when even
-    // max_splits does not fill one wave).
+    // max_splits does not fill one wave).  The dense variant's count is the cache capacity.
     const int count_max = p.k_max;
-    const int occ = ctas_per_sm((const void*)kern, kThreads, plan_smem<D, GT>(kMaxSplitLen, p.max_splits));
+    const int max_len = DENSE ? kMaxSplitLenDense : kMaxSplitLen;
+    const int occ = ctas_per_sm((const void*)kern, kThreads, plan_smem<D, GT>(max_len, p.max_splits, GATED));
     const long heads = (long)p.B * p.Hkv * p.ngz;
     const long slots = (long)p.sms * occ;
-    const int s_lo = (count_max + kMaxSplitLen - 1) / kMaxSplitLen;
+    const int s_lo = (count_max + max_len - 1) / max_len;
     int best = p.max_splits;
     if (heads * p.max_splits > slots) {
       double best_eff = -1.0;
@@ -582,8 +584,8 @@ cudaError_t launch_t(const AttendParams& p0, cudaStream_t stream) {
     if (len < 32) len = 32;
     p.split_len = len;
     p.splits = (count_max + len - 1) / len;
-    p.smem_bytes = plan_smem<D, GT>(p.split_len, p.splits);
   }
+  p.smem_bytes = plan_smem<D, GT>(p.split_len, p.splits, GATED);
   cudaError_t e = prepare_kernel((const void*)kern, p.smem_bytes);
   if (e != cudaSuccess) return e;
   dim3 grid((unsigned)p.splits, (unsigned)(p.B * p.Hkv), (unsigned)p.ngz);
