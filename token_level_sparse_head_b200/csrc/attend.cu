@@ -566,7 +566,26 @@ cudaError_t launch_t(const AttendParams& p0, cudaStream_t stream) {
     const long slots = (long)p.sms * occ;
     const int s_lo = (count_max + max_len - 1) / max_len;
     int best = p.max_splits;
-    if (heads * p.max_splits > slots) {
+    if (DENSE) {
+      // The dense slices are long and bandwidth-bound: balance the rows per SM (CTAs a multiple
+      // of the SM count) and keep the resident slots filled; one wave when one can hold them.
+      // Each candidate is scored on its split count after the slice length is rounded.
+      const bool one_wave = heads * s_lo <= slots;
+      double best_eff = -1.0;
+      for (int s = s_lo < 1 ? 1 : s_lo; s <= p.max_splits; ++s) {
+        int len = (count_max + s - 1) / s;
+        len = (len + 31) & ~31;
+        const long ctas = heads * (long)((count_max + len - 1) / len);
+        if (one_wave && ctas > slots) break;
+        const long per_sm = (ctas + p.sms - 1) / p.sms;
+        const double fill = (double)(ctas < slots ? ctas : slots) / (double)slots;
+        const double eff = fill * (double)ctas / (double)(per_sm * p.sms);
+        if (eff > best_eff + 1e-9) {
+          best_eff = eff;
+          best = s;
+        }
+      }
+    } else if (heads * p.max_splits > slots) {
       double best_eff = -1.0;
       for (int s = s_lo < 1 ? 1 : s_lo; s <= p.max_splits; ++s) {
         const long ctas = heads * s;
