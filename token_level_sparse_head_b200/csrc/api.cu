@@ -53,6 +53,7 @@ cudaError_t prepare_kernel(const void* kern, int smem_bytes, bool nonportable_cl
   constexpr int kDevices = 64;
   struct Allowed {
     int bytes;
+    bool nonportable;
     unsigned long long ctx_id;
   };
   static std::mutex mu;
@@ -69,19 +70,27 @@ cudaError_t prepare_kernel(const void* kern, int smem_bytes, bool nonportable_cl
     auto it = allowed.find(kern);
     if (it == allowed.end()) {
       std::array<Allowed, kDevices> none;
-      none.fill(Allowed{-1, 0});
+      none.fill(Allowed{-1, false, 0});
       it = allowed.emplace(kern, none).first;
     }
     lim = &it->second[dev];
-    if (ctx_id != 0 && lim->ctx_id == ctx_id && lim->bytes >= smem_bytes) return cudaSuccess;
+    if (ctx_id != 0 && lim->ctx_id == ctx_id && lim->bytes >= smem_bytes && (lim->nonportable || !nonportable_cluster))
+      return cudaSuccess;
   }
-  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes);
+  // Never lower a limit already set in this context (another launch of the kernel may need it).
+  const int bytes = (lim != nullptr && ctx_id != 0 && lim->ctx_id == ctx_id && lim->bytes > smem_bytes) ? lim->bytes
+                                                                                                     : smem_bytes;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
   if (e == cudaSuccess && nonportable_cluster)
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
   if (e == cudaSuccess && lim != nullptr) {
     if (ctx_id == 0) current_context_id(&ctx_id);  // the call above made the primary context current
-    if (lim->ctx_id != ctx_id) lim->bytes = -1;
-    if (smem_bytes > lim->bytes) lim->bytes = smem_bytes;
+    if (lim->ctx_id != ctx_id) {
+      lim->bytes = -1;
+      lim->nonportable = false;
+    }
+    if (bytes > lim->bytes) lim->bytes = bytes;
+    if (nonportable_cluster) lim->nonportable = true;
     lim->ctx_id = ctx_id;
   }
   return e;
