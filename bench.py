@@ -210,7 +210,8 @@ class Workload:
         ev[4].record()
 
     def parts(self):
-        """The step's four kernels as separate calls of the component entry points."""
+        """The step's four component calls (append, score scan, selection, attention with its split
+        merge) as separate entry-point calls."""
         p, L, s = self.p, self.lib, self.sess
         return {
             "append": lambda: L.sas_append_proj(self.shape, self.knew, p.M, self.kproj, p.page_table, p.seqlens),
