@@ -441,19 +441,23 @@ __global__ void __launch_bounds__(kThreads) attend_kernel(const AttendParams p) 
 
 // Merge of each head group's split partials, in split order (deterministic), and the output.
 // Launched after the split kernel on the same stream with programmatic dependent launch: its
-// wait returns once every split CTA has finished and its partial is visible.
-template <int D, int GT>
+// wait returns once every split CTA has finished and its partial is visible.  NQ CTAs share a
+// head group, each taking D / NQ of its channels (NQ = 4 when there are few head groups, so that
+// more SMs read the partials and each warp has fewer loads in flight to wait for).
+template <int D, int GT, int NQ>
 __host__ __device__ inline int combine_smem_floats(int splits) {
-  return ((splits * GT + GT + 3) & ~3) + kWarps * GT * D;
+  return ((splits * GT + GT + 3) & ~3) + kWarps * GT * (D / NQ);
 }
 
-template <int D, int GT>
+template <int D, int GT, int NQ>
 __global__ void __launch_bounds__(kThreads) combine_kernel(const AttendParams p) {
+  constexpr int DC = D / NQ;                   // channels of this CTA
   extern __shared__ __align__(16) float csm[];
   float* wts = csm;                                          // [splits][GT] weights, [GT] 1/L
-  float* red = csm + ((p.splits * GT + GT + 3) & ~3);       // [kWarps][GT * D] warp sums
+  float* red = csm + ((p.splits * GT + GT + 3) & ~3);       // [kWarps][GT * DC] warp sums
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int bhz = blockIdx.x;
+  const int c_base = blockIdx.y * DC;
   const int bh = bhz / p.ngz, gz = bhz % p.ngz;
   const int b = bh / p.Hkv, h = bh % p.Hkv;
   const size_t nheads = (size_t)p.B * p.Hkv * p.ngz;
@@ -465,18 +469,20 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(const AttendParams p)
   // Warp w sums splits w, w + 4, ... in order, kU splits per step with all their loads in flight;
   // lane owns OPL consecutive outputs (one head).  The first step's loads are issued before the
   // weights are computed, so the two reads of the partials overlap.
-  constexpr int OPL = GT * D / 32;
+  constexpr int OPL = GT * DC / 32;
+  static_assert(OPL >= 2 && OPL % 2 == 0, "two or more outputs per lane");
   constexpr int VW = (OPL % 4 == 0) ? 4 : 2;   // floats per load
-  constexpr int kU = 4;
+  constexpr int kU = OPL <= 4 ? 8 : 4;         // splits per step (registers: kU * OPL)
   const int e0 = lane * OPL;
-  const int gl = e0 / D;
+  const int gl = e0 / DC;
+  const int coff = gl * D + c_base + e0 % DC;  // offset of the lane's outputs in a [GT][D] partial
   float va[kU][OPL];
   auto load_step = [&](int s0) {
 #pragma unroll
     for (int u = 0; u < kU; ++u) {
       const int s = s0 + u * kWarps;
       if (s < p.splits) {
-        const float* a = bacc + (size_t)s * GT * D + e0;
+        const float* a = bacc + (size_t)s * GT * D + coff;
 #pragma unroll
         for (int i = 0; i < OPL; i += VW) {
           if constexpr (VW == 4) {
@@ -529,17 +535,17 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(const AttendParams p)
 #pragma unroll
   for (int i = 0; i < OPL; i += VW) {
     if constexpr (VW == 4) {
-      *reinterpret_cast<float4*>(red + warp * GT * D + e0 + i) = make_float4(racc[i], racc[i + 1], racc[i + 2], racc[i + 3]);
+      *reinterpret_cast<float4*>(red + warp * GT * DC + e0 + i) = make_float4(racc[i], racc[i + 1], racc[i + 2], racc[i + 3]);
     } else {
-      *reinterpret_cast<float2*>(red + warp * GT * D + e0 + i) = make_float2(racc[i], racc[i + 1]);
+      *reinterpret_cast<float2*>(red + warp * GT * DC + e0 + i) = make_float2(racc[i], racc[i + 1]);
     }
   }
   __syncthreads();
-  for (int e = tid; e < GT * D; e += kThreads) {
-    const int g = e / D, c = e % D;
+  for (int e = tid; e < GT * DC; e += kThreads) {
+    const int g = e / DC, c = c_base + e % DC;
     float v = 0.f;
 #pragma unroll
-    for (int w = 0; w < kWarps; ++w) v += red[w * GT * D + e];
+    for (int w = 0; w < kWarps; ++w) v += red[w * GT * DC + e];
     const int hq = h * p.G + gz * GT + g;
     p.out[((size_t)b * p.Hq + hq) * D + c] = v * wts[p.splits * GT + g];
   }
@@ -610,11 +616,22 @@ cudaError_t launch_t(const AttendParams& p0, cudaStream_t stream) {
   dim3 grid((unsigned)p.splits, (unsigned)(p.B * p.Hkv), (unsigned)p.ngz);
   e = launch_pdl(kern, grid, dim3(kThreads), (size_t)p.smem_bytes, stream, p);
   if (e != cudaSuccess) return e;
-  auto ck = combine_kernel<D, GT>;
-  const int csm = combine_smem_floats<D, GT>(p.splits) * 4;
+  // Few head groups: four CTAs per group, each merging a quarter of the channels.
+  const unsigned groups = (unsigned)(p.B * p.Hkv * p.ngz);
+  if constexpr (GT * D / 4 >= 64) {
+    if (p.sms > 0 && groups * 2 < (unsigned)p.sms) {
+      auto ck = combine_kernel<D, GT, 4>;
+      const int csm = combine_smem_floats<D, GT, 4>(p.splits) * 4;
+      e = prepare_kernel((const void*)ck, csm);
+      if (e != cudaSuccess) return e;
+      return launch_pdl(ck, dim3(groups, 4), dim3(kThreads), (size_t)csm, stream, p);
+    }
+  }
+  auto ck = combine_kernel<D, GT, 1>;
+  const int csm = combine_smem_floats<D, GT, 1>(p.splits) * 4;
   e = prepare_kernel((const void*)ck, csm);
   if (e != cudaSuccess) return e;
-  return launch_pdl(ck, dim3((unsigned)(p.B * p.Hkv * p.ngz)), dim3(kThreads), (size_t)csm, stream, p);
+  return launch_pdl(ck, dim3(groups), dim3(kThreads), (size_t)csm, stream, p);
 }
 
 template <int D, int GT>
