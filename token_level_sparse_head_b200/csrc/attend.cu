@@ -13,8 +13,9 @@
 // own ring of stages and its own online-softmax state (running max m, sum l, accumulator), in
 // fp32.  Logits z = sigma q.K_i (+ lambda log g_i, SAS page section 2.1).  The warps merge in
 // shared memory and the CTA writes one partial (m, l, acc) per query head to the workspace; a
-// second kernel, one CTA per (b, h, head group), merges the splits in split order
-// (deterministic) and writes the output.  The split CTAs wait on no counter or fence, so each
+// second kernel, one CTA per (b, h, head group) (four, each with a quarter of the channels,
+// when head groups are few), merges the splits in split order (deterministic) and writes the
+// output.  The split CTAs wait on no counter or fence, so each
 // frees its SM slot as soon as its partial is written.  The dense variant (idx = 0..N_b-1) is
 // the full-KV baseline.
 #include "sas_device.cuh"
