@@ -37,6 +37,16 @@ def test_head_shapes(cuda_lib, d, r, Hq, Hkv):
     run_small(p)
 
 
+@pytest.mark.parametrize("d,r,Hq,Hkv", [(64, 16, 8, 2), (128, 32, 4, 2), (128, 32, 8, 2)])
+def test_split_merge_many_splits(cuda_lib, d, r, Hq, Hkv):
+    # one sequence and two KV heads, so the split merge takes four CTAs per head group (a quarter
+    # of the channels each); k = 6000 gives 47 sparse splits (two load steps per merge warp) and
+    # the dense decode of 20000 rows more still; head groups of 4 and of 2 query heads
+    p = make_problem(B=1, Hq=Hq, Hkv=Hkv, d=d, r=r, seqlens=[20000], k=[6000], basis="qr", aniso=True,
+                     seed=d + Hq, poison_tail=True)
+    run_small(p, check_build=False)
+
+
 def test_multi_cta_clusters(cuda_lib):
     # capacity 40000 with 2 heads -> clusters of 16 CTAs; with 32 heads -> clusters of 4
     p = make_problem(B=1, Hq=8, Hkv=2, d=128, r=32, seqlens=[40000], k=[2500], basis="eye", aniso=True, seed=3)
